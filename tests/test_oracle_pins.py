@@ -1,0 +1,437 @@
+"""Pins of the fp64 oracle to things other than itself (CPU only).
+
+Each test names what fixes the expected value: the pages' worked example or
+printed figures (fixtures under tests/golden/, with their citations), the
+E4M3 format's closed forms, a library routine, brute force, or an invariant
+the pages state.  Together they are chosen so that a dropped scale, a wrong
+GQA head map, a transposed operand, an off-by-one in the gather or a wrong
+block index fails at least one of them (see the planted-mistake tests at
+the end).
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+import oracle
+from oracle import codecs, paged, memory
+from paged_kv_cache_416_b200.alloc import BlockAllocator
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# --------------------------------------------------------------------------
+# the pages' worked example and printed figures
+# --------------------------------------------------------------------------
+
+def test_worked_example_block_table_and_gather():
+    g = _golden("worked_example.json")
+    bs, d = g["block_size"], g["head_dim"]
+    alloc = BlockAllocator(g["pool_blocks"], bs, free_list=g["free_list"])
+    n = g["num_tokens"]
+    assert memory.blocks_needed(n, bs) == g["expected_blocks"]
+    table = alloc.allocate(0, n)
+    assert table == g["expected_block_table"]
+    assert list(alloc.free) == g["expected_free_after"]
+    # keys written through the table and read back are intact (bit-equal)
+    rng = np.random.default_rng(0)
+    keys = rng.standard_normal((n, 1, d)).astype(np.float32)
+    pool = np.zeros((g["pool_blocks"], bs, 1, d), dtype=np.float32)
+    slots = [oracle.slot_of(table, p, bs) for p in range(n)]
+    assert slots == [alloc.slot(0, p) for p in range(n)]
+    paged.write_kv(keys, keys, "f32", slots, pool, pool.copy(), "f32")
+    back = paged.gather(pool, table, n)
+    assert np.array_equal(back, keys) == g["expected_keys_intact"]
+    # the rows live in the blocks the table names, at pos // bs, pos % bs
+    assert np.array_equal(pool[41, :16], keys[:16]) and np.array_equal(pool[19, :8], keys[32:40])
+    assert memory.paged_unused_slots([n], bs) == g["expected_unused_paged"]
+    assert memory.reservation_unused_slots(n, g["reservation_tokens"]) == g["expected_unused_reserved"]
+
+
+def test_printed_memory_figures():
+    g = _golden("memory_figures.json")
+    a = g["llama13b_one_sequence"]
+    b13 = memory.kv_bytes(a["tokens"], a["layers"], a["kv_heads"], a["head_dim"], a["elem_bytes"])
+    assert b13 == 2048 * 40 * 2 * 40 * 128 * 2
+    assert round(b13 / 1e9, 1) == a["printed_gb"]
+    b = g["llama31_70b_4096_tokens"]
+    b70 = memory.kv_bytes(b["tokens"], b["layers"], b["kv_heads"], b["head_dim"], b["elem_bytes"])
+    assert round(b70 / 1e9, 1) == b["printed_gb"]
+    c = g["internal_fragmentation_4096"]
+    waste = memory.reservation_unused_slots(c["used"], c["reserved"]) / c["reserved"]
+    assert round(100 * waste) == c["printed_percent_wasted"]
+    e = g["internal_fragmentation_1000"]
+    assert memory.reservation_unused_slots(e["used"], e["reserved"]) == e["printed_unused"]
+
+
+def test_paged_waste_is_below_one_block_per_sequence():
+    rng = np.random.default_rng(3)
+    lens = rng.integers(1, 5000, size=200)
+    for bs in (16, 32):
+        w = memory.paged_unused_slots(lens, bs)
+        assert 0 <= w < bs * len(lens)
+        assert w == sum((-(-int(n) // bs)) * bs - int(n) for n in lens)
+
+
+# --------------------------------------------------------------------------
+# codecs
+# --------------------------------------------------------------------------
+
+def test_e4m3_decode_closed_forms():
+    dec = codecs.e4m3_decode
+    assert dec(np.uint8(0x00)) == 0.0 and np.signbit(dec(np.uint8(0x80)))
+    assert dec(np.uint8(0x01)) == 2.0 ** -9            # smallest subnormal
+    assert dec(np.uint8(0x07)) == 7 * 2.0 ** -9        # largest subnormal
+    assert dec(np.uint8(0x08)) == 2.0 ** -6            # smallest normal
+    assert dec(np.uint8(0x38)) == 1.0                  # e = bias, m = 0
+    assert dec(np.uint8(0x3C)) == 1.5
+    assert dec(np.uint8(0x7E)) == 448.0                # largest finite
+    assert dec(np.uint8(0xFE)) == -448.0
+    assert np.isnan(dec(np.uint8(0x7F))) and np.isnan(dec(np.uint8(0xFF)))
+    vals = codecs.e4m3_finite_values()
+    assert len(vals) == 127 and np.all(np.diff(vals) > 0)
+    # every normal binade holds 8 evenly spaced values
+    for e in range(1, 16):
+        seg = vals[8 * e: 8 * e + 8] if 8 * e + 8 <= 127 else vals[8 * e:]
+        step = 2.0 ** (e - 7) / 8
+        assert np.allclose(np.diff(seg), step)
+
+
+def test_e4m3_roundtrip_every_finite_code():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    vals = codecs.e4m3_decode(codes).astype(np.float32)
+    assert np.array_equal(codecs.e4m3_encode_f32(vals), codes)
+
+
+def test_e4m3_encode_matches_library_cast():
+    rng = np.random.default_rng(7)
+    vals = codecs.e4m3_finite_values()
+    mids = (vals[:-1] + vals[1:]) / 2  # exact ties
+    x = np.concatenate([
+        rng.standard_normal(400_000) * 3,
+        rng.standard_normal(200_000) * 100,
+        rng.uniform(-2.0 ** -6, 2.0 ** -6, 200_000),     # subnormal range
+        mids, -mids, vals, -vals,
+        np.nextafter(mids.astype(np.float32), np.float32(np.inf)),
+        np.nextafter(mids.astype(np.float32), np.float32(-np.inf)),
+        [0.0, -0.0, 463.99, -463.99, 448.0, 449.0],
+    ]).astype(np.float32)
+    x = x[np.abs(x) < 464.0]  # the library cast overflows to NaN beyond here
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = codecs.e4m3_encode_f32(x)
+    assert np.array_equal(got, ref)
+
+
+def test_e4m3_encode_saturates_and_nan():
+    x = np.array([464.0, 480.0, 1e6, np.inf, -464.0, -np.inf, np.nan], dtype=np.float32)
+    assert codecs.e4m3_encode_f32(x).tolist() == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0xFE, 0x7F]
+
+
+def test_16bit_decoders_match_library():
+    rng = np.random.default_rng(1)
+    w = rng.integers(0, 1 << 16, size=100_000, dtype=np.uint16)
+    tf = torch.from_numpy(w.view(np.int16)).view(torch.float16).double().numpy()
+    tb = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(codecs.f16_bits_to_f64(w), tf)
+    np.testing.assert_array_equal(codecs.bf16_bits_to_f64(w), tb)
+
+
+# --------------------------------------------------------------------------
+# attention: library routine, brute force, closed forms
+# --------------------------------------------------------------------------
+
+def _contiguous_case(rng, B, hq, hkv, d, bs, lens):
+    """Pools holding each sequence's tokens in blocks 0.. in order
+    (identity table), as fp64 values stored in float64 'raw' arrays."""
+    nbs = [-(-n // bs) for n in lens]
+    N = sum(nbs)
+    kp = rng.standard_normal((N, bs, hkv, d))
+    vp = rng.standard_normal((N, bs, hkv, d))
+    tables = np.full((B, max(nbs)), -1, dtype=np.int64)
+    o = 0
+    for s, nb in enumerate(nbs):
+        tables[s, :nb] = np.arange(o, o + nb)
+        o += nb
+    q = rng.standard_normal((B, hq, d))
+    return q, kp, vp, tables
+
+
+def _oracle_f64(q, kp, vp, tables, lens, scale, hkv):
+    out = np.zeros_like(q)
+    for s in range(q.shape[0]):
+        out[s] = paged.decode_one(q[s], kp, vp, tables[s], int(lens[s]), scale, hkv)
+    return out
+
+
+@pytest.mark.parametrize("hq,hkv,d,bs", [(4, 4, 64, 16), (64, 8, 128, 16), (32, 8, 128, 32), (8, 1, 64, 16)])
+def test_decode_matches_library_sdpa(hq, hkv, d, bs):
+    rng = np.random.default_rng(hq * 131 + d)
+    lens = [1, bs, bs + 1, 3 * bs - 5, 77]
+    B = len(lens)
+    q, kp, vp, tables = _contiguous_case(rng, B, hq, hkv, d, bs, lens)
+    scale = 1.0 / math.sqrt(d)
+    got = _oracle_f64(q, kp, vp, tables, lens, scale, hkv)
+    for s, n in enumerate(lens):
+        nb = -(-n // bs)
+        K = torch.from_numpy(kp[tables[s, :nb]].reshape(-1, hkv, d)[:n]).permute(1, 0, 2)[None]
+        V = torch.from_numpy(vp[tables[s, :nb]].reshape(-1, hkv, d)[:n]).permute(1, 0, 2)[None]
+        Q = torch.from_numpy(q[s])[None, :, None, :]
+        ref = F.scaled_dot_product_attention(Q, K, V, scale=scale, enable_gqa=True)[0, :, 0, :]
+        np.testing.assert_allclose(got[s], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_decode_matches_brute_force_on_tiny():
+    """Pure-Python loops (math.exp), addressing each token through the table
+    as the pages' sketch does, on scattered blocks."""
+    rng = np.random.default_rng(11)
+    hq, hkv, d, bs, N = 4, 2, 8, 4, 20
+    lens = [1, 4, 5, 11]
+    kp = rng.standard_normal((N, bs, hkv, d))
+    vp = rng.standard_normal((N, bs, hkv, d))
+    perm = rng.permutation(N)
+    tables, o = [], 0
+    for n in lens:
+        nb = -(-n // bs)
+        tables.append(list(perm[o:o + nb]) + [-1] * (3 - nb))
+        o += nb
+    q = rng.standard_normal((len(lens), hq, d))
+    scale = 0.37
+    got = _oracle_f64(q, kp, vp, np.array(tables), lens, scale, hkv)
+    for s, n in enumerate(lens):
+        for h in range(hq):
+            kv = h // (hq // hkv)
+            z = []
+            for pos in range(n):
+                b, off = tables[s][pos // bs], pos % bs
+                z.append(scale * sum(q[s, h, i] * kp[b, off, kv, i] for i in range(d)))
+            m = max(z)
+            e = [math.exp(x - m) for x in z]
+            tot = sum(e)
+            for i in range(d):
+                ref = sum(e[pos] / tot * vp[tables[s][pos // bs], pos % bs, kv, i] for pos in range(n))
+                assert abs(got[s, h, i] - ref) < 1e-12
+
+
+def test_decode_closed_forms():
+    rng = np.random.default_rng(5)
+    hq, hkv, d, bs = 4, 2, 16, 16
+    q, kp, vp, tables = _contiguous_case(rng, 1, hq, hkv, d, bs, [40])
+    t = tables[0]
+    # one token: the output is that token's value row, exactly
+    out = paged.decode_one(q[0], kp, vp, t, 1, 0.25, hkv)
+    for h in range(hq):
+        assert np.array_equal(out[h], vp[t[0], 0, h // 2])
+    # q = 0: uniform weights, the mean of the value rows
+    out = paged.decode_one(np.zeros((hq, d)), kp, vp, t, 40, 0.25, hkv)
+    V = paged.gather(vp, t, 40)
+    for h in range(hq):
+        np.testing.assert_allclose(out[h], V[:, h // 2].mean(0), rtol=1e-12, atol=1e-13)
+    # all keys equal: also the mean, whatever q is
+    kp2 = kp.copy()
+    kp2[t[:3]] = kp[t[0], 0]
+    out = paged.decode_one(q[0], kp2, vp, t, 40, 0.25, hkv)
+    for h in range(hq):
+        np.testing.assert_allclose(out[h], V[:, h // 2].mean(0), rtol=1e-12, atol=1e-13)
+    # one key far above the rest: its value row
+    kp3 = np.zeros_like(kp)
+    kp3[t[1], 5] = 1.0
+    qd = np.ones((hq, d)) * 100.0
+    out = paged.decode_one(qd, kp3, vp, t, 40, 1.0, hkv)
+    for h in range(hq):
+        np.testing.assert_allclose(out[h], vp[t[1], 5, h // 2], rtol=1e-12, atol=1e-12)
+    # empty context: zeros
+    assert not paged.decode_one(q[0], kp, vp, t, 0, 0.25, hkv).any()
+
+
+def test_softmax_weights_sum_to_one():
+    rng = np.random.default_rng(9)
+    for n in (1, 2, 17, 4096):
+        K = rng.standard_normal((n, 128)) * 3
+        w = paged.attention_weights(rng.standard_normal(128), K, 1 / math.sqrt(128))
+        assert abs(w.sum() - 1.0) < 1e-12 and (w >= 0).all()
+
+
+# --------------------------------------------------------------------------
+# paging invariants the pages state
+# --------------------------------------------------------------------------
+
+def test_physical_placement_does_not_change_the_result():
+    """Blocks may sit wherever they are free: permuting physical ids (and
+    moving the contents with them) gives the identical output."""
+    rng = np.random.default_rng(21)
+    hq, hkv, d, bs = 8, 2, 32, 16
+    lens = [5, 16, 33, 100]
+    q, kp, vp, tables = _contiguous_case(rng, 4, hq, hkv, d, bs, lens)
+    base = _oracle_f64(q, kp, vp, tables, lens, 0.2, hkv)
+    N = kp.shape[0]
+    perm = rng.permutation(N)  # old id i -> new id perm[i]
+    kp2, vp2 = np.empty_like(kp), np.empty_like(vp)
+    kp2[perm], vp2[perm] = kp, vp
+    t2 = np.where(tables >= 0, perm[np.maximum(tables, 0)], -1)
+    assert np.array_equal(_oracle_f64(q, kp2, vp2, t2, lens, 0.2, hkv), base)
+
+
+def test_shared_blocks_equal_unshared_copies():
+    rng = np.random.default_rng(22)
+    hq, hkv, d, bs = 4, 4, 16, 16
+    # two sequences share 3 prefix blocks; the unshared version has copies
+    kp = rng.standard_normal((12, bs, hkv, d))
+    vp = rng.standard_normal((12, bs, hkv, d))
+    shared = np.array([[0, 1, 2, 3], [0, 1, 2, 4]])
+    kp[5:8], vp[5:8] = kp[0:3], vp[0:3]
+    unshared = np.array([[0, 1, 2, 3], [5, 6, 7, 4]])
+    q = rng.standard_normal((2, hq, d))
+    lens = [60, 55]
+    assert np.array_equal(_oracle_f64(q, kp, vp, shared, lens, 0.3, hkv),
+                          _oracle_f64(q, kp, vp, unshared, lens, 0.3, hkv))
+
+
+def test_unused_slots_and_table_entries_are_never_read():
+    rng = np.random.default_rng(23)
+    hq, hkv, d, bs = 4, 2, 16, 16
+    q, kp, vp, tables = _contiguous_case(rng, 2, hq, hkv, d, bs, [20, 7])
+    base = _oracle_f64(q, kp, vp, tables, [20, 7], 0.3, hkv)
+    kp[tables[0, 1], 4:] = np.nan
+    vp[tables[0, 1], 4:] = np.nan
+    kp[tables[1, 0], 7:] = np.nan
+    t = tables.copy()
+    t[1, 1:] = 10**6  # past the sequence: never read
+    assert np.array_equal(_oracle_f64(q, kp, vp, t, [20, 7], 0.3, hkv), base)
+
+
+def test_copy_on_write_semantics():
+    rng = np.random.default_rng(24)
+    k = rng.integers(0, 1 << 16, size=(8, 16, 2, 8), dtype=np.uint16)
+    v = rng.integers(0, 1 << 16, size=(8, 16, 2, 8), dtype=np.uint16)
+    k0, v0 = k.copy(), v.copy()
+    paged.copy_blocks(k, v, [[1, 5], [5, 6]])  # pairs read the state before any copy
+    assert np.array_equal(k[5], k0[1]) and np.array_equal(v[5], v0[1])
+    assert np.array_equal(k[6], k0[5]) and np.array_equal(v[6], v0[5])
+    assert np.array_equal(k[1], k0[1])
+    # a later write into the copy leaves the source untouched
+    new = rng.integers(0, 1 << 16, size=(1, 2, 8), dtype=np.uint16)
+    paged.write_kv(new, new, "bf16", [5 * 16 + 3], k, v, "bf16")
+    assert np.array_equal(k[5, 3], new[0]) and np.array_equal(k[1], k0[1])
+
+
+def test_allocator_copy_on_write_and_free():
+    a = BlockAllocator(10, 4, free_list=range(10))
+    a.allocate(0, 6)                      # blocks 0, 1 (second partial)
+    a.fork(0, 1)
+    a.fork(0, 2)
+    assert a.refcount[0] == 3 and a.refcount[1] == 3
+    s, cow = a.append_token(1)            # shared partial block -> copy first
+    assert cow == (1, 2) and s == 2 * 4 + 2
+    s, cow = a.append_token(2)
+    assert cow == (1, 3)
+    s, cow = a.append_token(0)            # last holder writes in place
+    assert cow is None and s == 1 * 4 + 2 and a.refcount[1] == 1
+    for _ in range(2):
+        a.append_token(0)                 # fills block 1, then takes a new one
+    assert a.tables[0] == [0, 1, 4] and a.lengths[0] == 9
+    a.free_seq(1)
+    assert a.refcount[0] == 2 and list(a.free)[-1] == 2
+    a.free_seq(2)
+    a.free_seq(0)
+    assert a.used_blocks() == 0 and sorted(a.free) == list(range(10))
+
+
+def test_write_kv_skips_padding_and_quantises_in_fp32():
+    rng = np.random.default_rng(25)
+    x = rng.standard_normal((3, 2, 8)).astype(np.float32)
+    raw = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    kp = np.zeros((4, 4, 2, 8), dtype=np.uint8)
+    vp = np.zeros((4, 4, 2, 8), dtype=np.uint8)
+    paged.write_kv(raw, raw, "bf16", [5, -1, 15], kp, vp, "e4m3", k_scale=0.01, v_scale=0.02)
+    xv = codecs.bf16_bits_to_f64(raw).astype(np.float32)
+    assert np.array_equal(kp[1, 1], codecs.e4m3_encode_f32(xv[0] / np.float32(0.01)))
+    assert np.array_equal(vp[3, 3], codecs.e4m3_encode_f32(xv[2] / np.float32(0.02)))
+    assert kp.sum() == kp[1, 1].sum() + kp[3, 3].sum()  # the padding token wrote nothing
+
+
+def test_fp8_decode_dequantises_with_the_scales():
+    """An e4m3 cache decodes to code value * scale: attention over it equals
+    attention over the dequantised fp64 cache (here checked via SDPA)."""
+    rng = np.random.default_rng(26)
+    hq, hkv, d, bs, n = 4, 2, 16, 16, 23
+    kc = rng.integers(0, 0x7E, size=(2, bs, hkv, d), dtype=np.uint8) | (rng.integers(0, 2, size=(2, bs, hkv, d), dtype=np.uint8) << 7)
+    vc = rng.integers(0, 0x7E, size=(2, bs, hkv, d), dtype=np.uint8)
+    qf = rng.standard_normal((1, hq, d)).astype(np.float32)
+    qraw = torch.from_numpy(qf).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    out = paged.decode(qraw, "bf16", kc, vc, "e4m3", np.array([[1, 0]]), [n], 0.25, hkv,
+                       k_scale=0.003, v_scale=0.5)
+    K = codecs.e4m3_decode(kc[[1, 0]]).reshape(-1, hkv, d)[:n] * 0.003
+    V = codecs.e4m3_decode(vc[[1, 0]]).reshape(-1, hkv, d)[:n] * 0.5
+    Q = codecs.bf16_bits_to_f64(qraw)
+    ref = F.scaled_dot_product_attention(torch.from_numpy(Q)[:, :, None, :],
+                                         torch.from_numpy(K).permute(1, 0, 2)[None],
+                                         torch.from_numpy(V).permute(1, 0, 2)[None],
+                                         scale=0.25, enable_gqa=True)[0, :, 0, :]
+    np.testing.assert_allclose(out[0], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# planted mistakes: each pin above catches at least one plausible error
+# --------------------------------------------------------------------------
+
+def _sdpa_pin_fails(monkeypatch, patch):
+    patch(monkeypatch)
+    try:
+        test_decode_matches_library_sdpa(64, 8, 128, 16)
+    except AssertionError:
+        return True
+    return False
+
+
+def test_planted_wrong_gqa_map_is_caught(monkeypatch):
+    def patch(mp):
+        orig = paged.decode_one
+
+        def bad(q_f64, k_vals, v_vals, table_row, n, scale, hkv):
+            out = orig(q_f64, k_vals, v_vals, table_row, n, scale, hkv)
+            hq = q_f64.shape[0]
+            # strided instead of consecutive grouping
+            for h in range(hq):
+                kv = h % hkv
+                K = paged.gather(k_vals, table_row, n)[:, kv]
+                V = paged.gather(v_vals, table_row, n)[:, kv]
+                out[h] = paged.attention_weights(q_f64[h], K, scale) @ V
+            return out
+        mp.setattr(paged, "decode_one", bad)
+    assert _sdpa_pin_fails(monkeypatch, patch)
+
+
+def test_planted_dropped_scale_is_caught(monkeypatch):
+    def patch(mp):
+        orig = paged.attention_weights
+        mp.setattr(paged, "attention_weights", lambda q, K, scale: orig(q, K, 1.0))
+    assert _sdpa_pin_fails(monkeypatch, patch)
+
+
+def test_planted_gather_off_by_one_is_caught(monkeypatch):
+    orig = paged.gather
+    monkeypatch.setattr(paged, "gather", lambda pool, row, n: orig(pool, row, n + 1)[1:])
+    with pytest.raises(AssertionError):
+        test_decode_matches_brute_force_on_tiny()
+
+
+def test_planted_e4m3_tie_rule_is_caught(monkeypatch):
+    orig = codecs.e4m3_encode_f32
+
+    def ties_away(x):
+        x = np.asarray(x, dtype=np.float32)
+        nudged = np.nextafter(x, np.copysign(np.float32(np.inf), x)).astype(np.float32)
+        return orig(nudged)
+    monkeypatch.setattr(codecs, "e4m3_encode_f32", ties_away)
+    with pytest.raises(AssertionError):
+        test_e4m3_encode_matches_library_cast()
