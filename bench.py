@@ -1,0 +1,512 @@
+#!/usr/bin/env python
+"""Benchmark of the paged decode step on B200; prints ONE JSON line (rank 0).
+
+A step is one pass of the whole hot path over one batch: copy-on-write block
+copies (none in the default workload), the cache write of every sequence's
+new token (pa_write_kv), and paged decode attention over all sequences
+(pa_decode: plan + main kernel + merge when contexts are split).
+
+Default workload: the Llama-3-70B-shaped GQA decode layer -- 256 sequences
+x 4096 tokens, 64 query / 8 KV heads, head_dim 128, bf16, block_size 16,
+physical blocks randomly permuted (4 GiB of K+V read per step).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME]
+
+Multi-GPU (torchrun, one process per GPU): replicas only -- every rank runs
+its own copy of the workload, no collective touches the data path; the
+barrier and the max-over-ranks timing use the process group.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attn: KV-read GB/s (% of HBM peak), seq-tokens/s"
+NOMINAL_HBM_GBS = 8000.0      # the "~8 TB/s" B200 figure the target is stated against
+FALLBACK_HBM_GBS = 6650.0     # used only when MEASURED_PEAKS.json is absent
+DEFAULT_WORKLOAD = "llama70b_gqa"
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_kernel_llama70b_gqa.md")
+DECODE_SOURCES = [os.path.join(ROOT, "paged_kv_cache_416_b200", "csrc", f)
+                  for f in ("decode.cuh", "common.cuh")]
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--seed", type=int, default=3)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    return ap.parse_args(argv)
+
+
+# ------------------------------------------------------------ distributed
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+def dist_init(backend: str, timeout_s: int = 300):
+    import torch.distributed as dist
+    rank, local, world = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return rank, local, world
+
+
+def barrier(world: int, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def reduce_max(x: float, world: int, device) -> float:
+    """Max of x over ranks (x itself at world 1)."""
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x: float, world: int, device) -> float:
+    if world == 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def aggregate(bytes_per_step_per_rank: float, tokens_per_step_per_rank: float, steps: int,
+              max_seconds: float, world: int, device):
+    """Whole-job throughput: units all ranks processed / the slowest rank's time."""
+    total_bytes = reduce_sum(bytes_per_step_per_rank * steps, world, device)
+    total_tokens = reduce_sum(tokens_per_step_per_rank * steps, world, device)
+    return total_bytes / max_seconds / 1e9, total_tokens / max_seconds
+
+
+# ----------------------------------------------------------------- clocks
+NVML_REASONS = {
+    0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+    0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+    0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting",
+}
+
+
+class ClockSampler:
+    """Reads the SM clock and clock-event reasons through NVML on a thread
+    while running (read-only queries; no setting is changed)."""
+
+    def __init__(self, torch_device_index: int = 0, period_s: float = 0.002):
+        self.samples = []
+        self.period = period_s
+        self.max_mhz = None
+        self.ok = False
+        self._stop = threading.Event()
+        self._th = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            h = None
+            try:
+                uuid = str(torch.cuda.get_device_properties(torch_device_index).uuid)
+                h = pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid) if not uuid.startswith("GPU-") else uuid)
+            except Exception:
+                h = pynvml.nvmlDeviceGetHandleByIndex(torch_device_index)
+            self.h = h
+            self.nv = pynvml
+            self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            self.ok = True
+        except Exception as e:  # pragma: no cover - depends on the box
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        get_r = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                r = get_r(self.h)
+                self.samples.append((float(sm), int(r)))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._th = threading.Thread(target=self._run, daemon=True)
+            self._th.start()
+
+    def stop(self):
+        if self._th is not None:
+            self._stop.set()
+            self._th.join()
+
+    def summary(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "note": "NVML unavailable"}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        mhz = sorted(s[0] for s in self.samples)
+        mask = 0
+        for _, r in self.samples:
+            mask |= r
+        reasons = [n for b, n in NVML_REASONS.items() if mask & b and n != "gpu_idle"]
+        return {"sm_mhz": mhz[len(mhz) // 2], "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(mhz)}
+
+
+# ----------------------------------------------------------------- helpers
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def decode_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in DECODE_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic():
+    """DRAM bytes per decode launch from the committed ncu summary, if it was
+    taken on the current kernel source (else None)."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    src, traffic = None, None
+    with open(PROFILE_SUMMARY) as f:
+        for line in f:
+            if line.startswith("decode_source_sha256:"):
+                src = line.split(":", 1)[1].strip()
+            if line.startswith("dram_bytes_per_launch:"):
+                traffic = int(float(line.split(":", 1)[1].strip()))
+    return traffic if (src == decode_source_hash() and traffic) else None
+
+
+# ------------------------------------------------------------ CPU baseline
+def oracle_rate(name: str, seed: int, target_seconds: float, workers: int):
+    """Time the oracle (as it stands) on a bounded sample of sequences of the
+    workload on the host's cores.  Returns (GB/s of KV read, seq-tokens/s,
+    description, cores, seconds)."""
+    import numpy as np
+    from oracle.parallel import run_decode_tasks
+    from paged_kv_cache_416_b200 import workloads as W
+    from paged_kv_cache_416_b200.workloads import raw
+
+    def tasks_for(n):
+        w = W.make(name, seed=seed, device="cpu", **_sample_kw(name, n))
+        ts = []
+        bs = w.block_size
+        for s in range(w.num_seqs):
+            nb = -(-int(w.context_lens[s]) // bs)
+            ids = w.block_tables[s, :nb].astype(np.int64)
+            ts.append((raw(w.q[s:s + 1]), w.q_dtype, raw(w.k_pool)[ids], raw(w.v_pool)[ids],
+                       w.cache_dtype, np.arange(nb)[None], w.context_lens[s:s + 1], w.scale,
+                       w.num_kv_heads, w.k_scale, w.v_scale))
+        return w, ts
+
+    # calibrate on one sequence per worker, then size the sample
+    w, ts = tasks_for(workers)
+    _, wall = run_decode_tasks(ts, workers)
+    per_round = max(wall, 1e-3)
+    rounds = max(1, int(target_seconds / per_round))
+    n = min(workers * rounds, _full_seqs(name))
+    if n > workers:
+        w, ts = tasks_for(n)
+        _, wall = run_decode_tasks(ts, workers)
+    gbs = w.kv_bytes / wall / 1e9
+    tps = w.seq_tokens / wall
+    desc = (f"oracle (numpy fp64) decode of {w.num_seqs} of the workload's {_full_seqs(name)} "
+            f"sequences (same shapes and lengths), {workers} spawned workers, 1 BLAS thread each")
+    return gbs, tps, desc, workers, wall
+
+
+def _full_seqs(name):
+    return {"llama70b_gqa": 256, "llama13b_mha": 64, "fp8_longtail_bs16": 128,
+            "fp8_longtail_bs32": 128, "shared_prefix_tails": 128, "shared_prefix_fork": 128,
+            "tiny": 4}[name]
+
+
+def _sample_kw(name, n):
+    if name in ("llama70b_gqa", "llama13b_mha", "fp8_longtail_bs16", "fp8_longtail_bs32"):
+        return {"num_seqs": n}
+    if name.startswith("shared_prefix"):
+        return {"prompts": max(1, n // 4)}
+    return {}
+
+
+# ----------------------------------------------------------------- our arm
+def run_ours(args, rank, local, world):
+    import numpy as np
+    import torch
+
+    from paged_kv_cache_416_b200 import build as _build
+    _build.build()
+    from paged_kv_cache_416_b200 import pagedattn as pa
+    from paged_kv_cache_416_b200 import workloads as W
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = W.make(args.workload, seed=args.seed + rank, device=device)
+    stream = torch.cuda.current_stream()
+    kp, vp = w.k_pool, w.v_pool
+    q = w.q.contiguous()
+    new_k, new_v = w.new_k.contiguous(), w.new_v.contiguous()
+    slots = torch.from_numpy(w.slot_mapping).to(device)
+    tables = torch.from_numpy(w.block_tables).to(device)
+    lens = torch.from_numpy(w.context_lens).to(device)
+    pairs = torch.from_numpy(w.cow_pairs).to(device)
+    out = torch.empty_like(q)
+    split = pa.decode_split_tokens(w.num_seqs, w.num_kv_heads, w.block_size, w.max_context_len)
+    ws = torch.empty(max(256, pa.decode_workspace_size(
+        w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, w.max_context_len)),
+        dtype=torch.uint8, device=device)
+    launches_per_step = (1 if len(w.cow_pairs) else 0) + 1 + 2 + (1 if split < w.max_context_len else 0)
+
+    def step(dec_events=None):
+        if len(w.cow_pairs):
+            pa.copy_blocks(kp, vp, pairs)
+        pa.write_kv(new_k, new_v, slots, kp, vp, w.k_scale, w.v_scale)
+        if dec_events is not None:
+            dec_events[0].record(stream)
+        pa.decode(q, kp, vp, tables, lens, w.scale, w.max_context_len, k_scale=w.k_scale,
+                  v_scale=w.v_scale, out=out, workspace=ws)
+        if dec_events is not None:
+            dec_events[1].record(stream)
+
+    # correctness of the run itself: no device-side error
+    step()
+    pa.sync_status()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    K = args.steps
+    dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier(world, device)
+    torch.cuda.synchronize()
+    clocks.start()
+    t0.record(stream)
+    for i in range(K):
+        step(dec_ev[i])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clocks.stop()
+    barrier(world, device)
+    pa.sync_status()
+    sec = t0.elapsed_time(t1) / 1e3
+    dec_ms = [a.elapsed_time(b) for a, b in dec_ev]
+    max_sec = reduce_max(sec, world, device)
+    value, tok_s = aggregate(w.kv_bytes, w.seq_tokens, K, max_sec, world, device)
+
+    # ---- end to end through the public API with host buffers
+    E = args.e2e_steps or K
+    host_in = {n: t.detach().cpu().pin_memory() for n, t in
+               (("q", q), ("new_k", new_k), ("new_v", new_v), ("slots", slots),
+                ("tables", tables), ("lens", lens), ("pairs", pairs))}
+    dev_in = {n: torch.empty_like(t, device=device) for n, t in host_in.items()}
+    out_host = torch.empty(out.shape, dtype=out.dtype, pin_memory=True)
+    h2d = sum(t.numel() * t.element_size() for n, t in host_in.items() if n != "pairs" or len(w.cow_pairs))
+    d2h = out.numel() * out.element_size()
+
+    def e2e_step():
+        for n, t in host_in.items():
+            if n == "pairs" and not len(w.cow_pairs):
+                continue
+            dev_in[n].copy_(t, non_blocking=True)
+        if len(w.cow_pairs):
+            pa.copy_blocks(kp, vp, dev_in["pairs"])
+        pa.write_kv(dev_in["new_k"], dev_in["new_v"], dev_in["slots"], kp, vp, w.k_scale, w.v_scale)
+        pa.decode(dev_in["q"], kp, vp, dev_in["tables"], dev_in["lens"], w.scale, w.max_context_len,
+                  k_scale=w.k_scale, v_scale=w.v_scale, out=out, workspace=ws)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(max(3, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world, device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, device)
+    pa.sync_status()
+    e2e_sec = reduce_max(e0.elapsed_time(e1) / 1e3, world, device)
+    e2e_value, _ = aggregate(w.kv_bytes, w.seq_tokens, E, e2e_sec, world, device)
+
+    peak, peak_kind = measured_peaks()
+    dec_mean_s = float(np.mean(dec_ms)) / 1e3
+    achieved = w.kv_bytes / dec_mean_s / 1e9
+
+    if rank != 0:
+        return None
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        from oracle.parallel import host_cores
+        gbs, tps, desc, cores, wall = oracle_rate(args.workload, args.seed, args.cpu_seconds,
+                                                  host_cores())
+        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": desc, "seq_tokens_per_s": round(tps, 1), "seconds": round(wall, 2)}
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(max_sec / K * 1e3, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": {"f16": "f16", "bf16": "bf16", "e4m3": "e4m3"}[w.cache_dtype],
+        "data": "synthetic",
+        "config": {
+            "workload": w.name, "num_seqs": w.num_seqs, "context_lens": _lens_desc(w),
+            "num_q_heads": w.num_q_heads, "num_kv_heads": w.num_kv_heads,
+            "head_dim": w.head_dim, "block_size": w.block_size, "cache_dtype": w.cache_dtype,
+            "num_blocks": w.num_blocks, "split_tokens": split,
+            "kv_bytes_per_step": w.kv_bytes, "parallelism": f"replicas x{world}",
+            "l2": f"inputs larger than L2: {w.kv_bytes / 2**30:.2f} GiB of K/V streamed per step "
+                  f"vs 126 MB L2; no flush",
+        },
+        "seq_tokens_per_s": round(tok_s, 1),
+        "pct_of_8tbs": round(100 * value / NOMINAL_HBM_GBS, 2),
+        "roofline": {
+            "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
+            "frac": round(achieved / peak, 4), "traffic": profiled_traffic(),
+            "kernel": "pa_decode (plan + decode_kernel" + (" + merge" if split < w.max_context_len else "") + ")",
+            "algorithmic_bytes_per_launch": w.kv_bytes, "peak_kind": peak_kind,
+            "mean_launch_us": round(dec_mean_s * 1e6, 2),
+        },
+        "cpu_baseline": cpu,
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_sec / E * 1e3, 4)},
+        "gpu_launches": launches_per_step * K,
+        "clocks": clocks.summary(),
+    }
+    return line
+
+
+def _lens_desc(w):
+    import numpy as np
+    c = w.context_lens
+    if (c == c[0]).all():
+        return f"all {int(c[0])}"
+    return f"min {int(c.min())} median {int(np.median(c))} max {int(c.max())} sum {int(c.sum())}"
+
+
+# ---------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    """The oracle as it stands, timed on the host's cores, on a bounded sample
+    of the workload per step."""
+    if rank != 0:
+        return None
+    from oracle.parallel import host_cores, run_decode_tasks
+    import numpy as np
+    from paged_kv_cache_416_b200 import workloads as W
+    from paged_kv_cache_416_b200.workloads import raw
+
+    cores = host_cores()
+    n = min(_full_seqs(args.workload), cores)  # one sequence per core per step
+    w = W.make(args.workload, seed=args.seed, device="cpu", **_sample_kw(args.workload, n))
+    bs = w.block_size
+    tasks = []
+    for s in range(w.num_seqs):
+        nb = -(-int(w.context_lens[s]) // bs)
+        ids = w.block_tables[s, :nb].astype(np.int64)
+        tasks.append((raw(w.q[s:s + 1]), w.q_dtype, raw(w.k_pool)[ids], raw(w.v_pool)[ids],
+                      w.cache_dtype, np.arange(nb)[None], w.context_lens[s:s + 1], w.scale,
+                      w.num_kv_heads, w.k_scale, w.v_scale))
+    for _ in range(args.warmup):
+        run_decode_tasks(tasks[:1], 1)
+    total = 0.0
+    for _ in range(args.steps):
+        _, wall = run_decode_tasks(tasks, cores)
+        total += wall
+    gbs = w.kv_bytes * args.steps / total / 1e9
+    desc = (f"oracle (numpy fp64) decode of {w.num_seqs} of the workload's "
+            f"{_full_seqs(args.workload)} sequences per step, {cores} spawned workers")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total / args.steps * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "sample_seqs": w.num_seqs},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, local, world = dist_env()
+    if args.impl == "reference":
+        if world > 1:
+            import torch.distributed as dist
+            if rank != 0:
+                return 0
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return 0
+    import torch
+    if world > 1:
+        torch.cuda.set_device(local)
+    rank, local, world = dist_init("nccl")
+    try:
+        line = run_ours(args, rank, local, world)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,217 @@
+/*
+ * pagedattn.h -- C ABI of the paged KV-cache decode-attention library
+ * (libpagedattn.so, hand-written CUDA for sm_100a / B200).
+ *
+ * The method: a KV cache split into fixed-size physical blocks that sit
+ * wherever they were free in one shared pool, addressed per sequence by a
+ * block table that maps logical block i to a physical block id; the attention
+ * kernel follows the table to gather keys and values block by block, so a
+ * sequence's cache need not be contiguous ("PagedAttention", Ultralytics
+ * glossary, section "Sayfalama Nasil Calisir" and its PyTorch sketch).  Blocks
+ * may be shared by several sequences and are copied before a write while
+ * others still use them (same page, section "Diziler Arasinda Bloklari
+ * Paylasma").  Grouped-query attention and FP8 caches are named as companion
+ * techniques (same page, section "Ilgili Teknikler").
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *    never frees, retains or allocates device memory.
+ *  - Every tensor is dense and row-major with the layout stated below.
+ *  - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and the call returns without synchronising.
+ *  - Arguments are validated on the host before any launch; a failed check
+ *    returns a PA_ERR_* code, launches nothing and sets pa_last_error().
+ *  - Kernels never trap: an out-of-range index met on the device (a block id
+ *    outside the pool, a slot outside the pool, a context length above the
+ *    stated maximum) skips that access and records PA_ERR_DEVICE_BOUNDS in a
+ *    device error word that pa_sync_status() reports.
+ *  - Nothing throws across the ABI.
+ *
+ * Layouts (B = num_seqs, Hq = num_q_heads, Hkv = num_kv_heads, D = head_dim,
+ * bs = block_size, N = num_blocks, T = num_tokens):
+ *   q, out        [B, Hq, D]          q dtype (out has q's dtype)
+ *   k, v (write)  [T, Hkv, D]
+ *   k_pool/v_pool [N, bs, Hkv, D]     the sketch's key_pool[block, slot, dim]
+ *                                     with the head axis before dim
+ *   block_tables  int32 [B, max_blocks_per_seq]; entries at or past
+ *                 ceil(context_lens[s] / bs) are never read
+ *   context_lens  int32 [B]
+ *   slot_mapping  int64 [T]; slot = physical_block * bs + offset; < 0 skips
+ *   src_dst_pairs int64 [P, 2]
+ *
+ * Supported: D in {64, 128}; bs in {16, 32}; Hq a multiple of Hkv with
+ * Hq / Hkv <= 8; cache dtype f16 (q f16), bf16 (q bf16) or e4m3 (q f16 or
+ * bf16).  With an e4m3 cache the query is converted to fp16 for the tensor-
+ * core products, so |q| must stay inside the fp16 range (< 65504).
+ */
+#ifndef PAGEDATTN_H_
+#define PAGEDATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A CUDA stream handle (the same object as cudaStream_t / CUstream). */
+typedef struct CUstream_st* pa_stream_t;
+
+typedef enum pa_dtype {
+  PA_F16 = 0,      /* IEEE binary16 */
+  PA_BF16 = 1,     /* bfloat16 */
+  PA_FP8_E4M3 = 2  /* OCP 8-bit E4M3 ("fn": no infinities, 0x7F/0xFF NaN, max 448) */
+} pa_dtype;
+
+typedef enum pa_status {
+  PA_OK = 0,
+  PA_ERR_NULL = 1,          /* a required pointer is NULL */
+  PA_ERR_DTYPE = 2,         /* unsupported dtype or dtype combination */
+  PA_ERR_SHAPE = 3,         /* unsupported or inconsistent size */
+  PA_ERR_HEADS = 4,         /* Hq not a multiple of Hkv, or Hq / Hkv > 8 */
+  PA_ERR_RANGE = 5,         /* an index is out of range (pa_validate_*) */
+  PA_ERR_ALIAS = 6,         /* duplicate destinations, or a destination that is
+                               also a source (pa_validate_*) */
+  PA_ERR_CUDA = 7,          /* a CUDA runtime call failed; see pa_last_error() */
+  PA_ERR_DEVICE_BOUNDS = 8, /* a kernel met an out-of-range index and skipped it */
+  PA_ERR_WORKSPACE = 9,     /* workspace missing or smaller than required */
+  PA_ERR_TIMEOUT = 10       /* a kernel gave up waiting for an asynchronous copy
+                               (about one second) and skipped that block */
+} pa_status;
+
+/*
+ * pa_write_kv -- scatter new keys and values into the pools by slot.
+ * Defined by the pages' sketch, where token `pos` of a request is stored at
+ * key_pool[block_table[pos // bs], pos % bs]; the caller folds the table into
+ * slot = block_table[pos // bs] * bs + pos % bs ("Sayfalama Nasil Calisir").
+ *
+ * For each token t with slot_mapping[t] >= 0 and every kv head h:
+ *   k_pool[slot / bs][slot % bs][h][:] = enc(k[t][h][:])   (same for v)
+ * enc is the identity when cache_dtype == in_dtype (f16 or bf16), and for an
+ * e4m3 cache enc(x) = e4m3_rne_satfinite(fp32(x) / k_scale) (v: v_scale),
+ * with the division in IEEE fp32.  Tokens with slot < 0 are padding and are
+ * skipped.  A slot >= num_blocks * bs is skipped and reported as
+ * PA_ERR_DEVICE_BOUNDS.  Two tokens with the same slot race (undefined which
+ * value lands); pa_validate_slot_mapping() detects that case.
+ * k_scale / v_scale are ignored for 16-bit caches and must be finite and
+ * > 0 for e4m3.
+ */
+pa_status pa_write_kv(const void* k, const void* v, pa_dtype in_dtype,
+                      const int64_t* slot_mapping, int32_t num_tokens,
+                      void* k_pool, void* v_pool, pa_dtype cache_dtype,
+                      int32_t num_blocks, int32_t block_size,
+                      int32_t num_kv_heads, int32_t head_dim,
+                      float k_scale, float v_scale, pa_stream_t stream);
+
+/*
+ * pa_copy_blocks -- copy-on-write block copy ("Diziler Arasinda Bloklari
+ * Paylasma": a block that others still use is copied before it is written).
+ * For each pair p: k_pool[dst] = k_pool[src] and v_pool[dst] = v_pool[src],
+ * all bs * Hkv * D elements, with (src, dst) = src_dst_pairs[p].
+ * Pairs must not chain or collide (no dst equal to another pair's src or
+ * dst); pa_validate_copy_pairs() checks that.  An id outside [0, num_blocks)
+ * skips the pair and reports PA_ERR_DEVICE_BOUNDS.  num_pairs == 0 is a no-op.
+ */
+pa_status pa_copy_blocks(void* k_pool, void* v_pool, pa_dtype cache_dtype,
+                         int32_t num_blocks, int32_t block_size,
+                         int32_t num_kv_heads, int32_t head_dim,
+                         const int64_t* src_dst_pairs, int32_t num_pairs,
+                         pa_stream_t stream);
+
+/*
+ * pa_decode_split_tokens -- the context-split length pa_decode uses for these
+ * sizes when split_tokens == 0 (always a multiple of block_size).  A value >=
+ * max_context_len means every (sequence, kv head) is one work item and no
+ * merge pass runs.  Returns 0 on invalid arguments.
+ */
+int32_t pa_decode_split_tokens(int32_t num_seqs, int32_t num_kv_heads,
+                               int32_t block_size, int32_t max_context_len,
+                               int32_t split_tokens);
+
+/*
+ * pa_decode_workspace_size -- bytes of device workspace pa_decode needs for
+ * these sizes (work counter, per-sequence item offsets, and the split
+ * partials: one fp32 log-sum-exp and one fp32 [D] vector per (item, q head)).
+ * Returns 0 on invalid arguments.
+ */
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                int32_t num_kv_heads, int32_t head_dim,
+                                int32_t block_size, int32_t max_context_len,
+                                int32_t split_tokens);
+
+/*
+ * pa_decode -- single-query decode attention over the paged cache.
+ * The attention kernel follows each sequence's block table to gather keys and
+ * values block by block ("Sayfalama Nasil Calisir"), in the tiled
+ * FlashAttention style that never writes the score matrix to memory ("Ilgili
+ * Teknikler", Flash Attention bullet), with the query heads of one KV head
+ * packed together (same section, grouped-query attention bullet).
+ *
+ * For every sequence s and query head h (kv head kvh = h / (Hq / Hkv)), with
+ * n = context_lens[s] and K_s, V_s the first n token rows gathered through
+ * block_tables[s]:
+ *   z_t    = scale * k_scale * <q[s][h], K_s[t][kvh]>          t < n
+ *   out[s][h] = v_scale * sum_t softmax(z)_t * V_s[t][kvh]
+ * (k_scale = v_scale = 1 for 16-bit caches), accumulated in fp32 and
+ * rounded to q's dtype (round to nearest even).  n == 0 gives zeros.
+ *
+ * Contexts longer than the split length are cut into ranges of split_tokens
+ * tokens (0 = automatic, see pa_decode_split_tokens); each range writes a
+ * partial (log-sum-exp, normalised vector) into the workspace and a merge
+ * pass combines them.  Results depend only on the arguments (not on the grid
+ * or on timing): the same call gives bit-identical outputs.
+ *
+ * max_context_len must bound every context_lens[s]; a larger length, or one
+ * above max_blocks_per_seq * bs, makes that sequence's output zero and
+ * reports PA_ERR_DEVICE_BOUNDS.  A table entry outside [0, num_blocks) is
+ * skipped (its tokens masked) and reported the same way.
+ * workspace: device memory of at least pa_decode_workspace_size(...) bytes,
+ * 256-byte aligned, used only during the call (stream-ordered).
+ */
+pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype,
+                    const void* k_pool, const void* v_pool, pa_dtype cache_dtype,
+                    const int32_t* block_tables, int32_t max_blocks_per_seq,
+                    const int32_t* context_lens, int32_t max_context_len,
+                    int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                    int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                    float scale, float k_scale, float v_scale,
+                    int32_t split_tokens,
+                    void* workspace, size_t workspace_bytes, pa_stream_t stream);
+
+/*
+ * pa_sync_status -- synchronise `stream`, then read and clear the device
+ * error word of the current device.  Returns PA_OK, PA_ERR_DEVICE_BOUNDS,
+ * PA_ERR_TIMEOUT or PA_ERR_CUDA (an asynchronous CUDA error).
+ */
+pa_status pa_sync_status(pa_stream_t stream);
+
+/* Message of the last failing call on this host thread ("" if none).  The
+ * pointer stays valid until the next call on this thread. */
+const char* pa_last_error(void);
+
+/*
+ * Debug checks of index contents (they copy the indices to the host and
+ * synchronise `stream`; not for the hot path):
+ *  pa_validate_slot_mapping: every slot < num_blocks * bs, no slot twice
+ *    (negative slots ignored)                -> PA_ERR_RANGE / PA_ERR_ALIAS
+ *  pa_validate_copy_pairs: ids in [0, num_blocks), no dst twice, no dst that
+ *    is also a src                           -> PA_ERR_RANGE / PA_ERR_ALIAS
+ *  pa_validate_block_tables: 0 <= context_lens[s] <= max_context_len,
+ *    ceil(len / bs) <= max_blocks_per_seq, and every entry the sequence
+ *    reads in [0, num_blocks)                -> PA_ERR_RANGE
+ */
+pa_status pa_validate_slot_mapping(const int64_t* slot_mapping, int32_t num_tokens,
+                                   int32_t num_blocks, int32_t block_size,
+                                   pa_stream_t stream);
+pa_status pa_validate_copy_pairs(const int64_t* src_dst_pairs, int32_t num_pairs,
+                                 int32_t num_blocks, pa_stream_t stream);
+pa_status pa_validate_block_tables(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                   const int32_t* context_lens, int32_t num_seqs,
+                                   int32_t max_context_len, int32_t block_size,
+                                   int32_t num_blocks, pa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDATTN_H_ */

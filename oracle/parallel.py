@@ -1,0 +1,55 @@
+"""Run the oracle's decode over many sequences in a process pool.
+
+TEST / BASELINE INFRASTRUCTURE ONLY (see the package docstring).  Used by
+the CPU-baseline and reference legs of bench.py to time the oracle on the
+host's cores.  Each task is one sequence with its own compact pools, so a
+worker needs only numpy and this package.  The pool uses the "spawn" start
+method and pins BLAS to one thread per worker.
+"""
+
+from __future__ import annotations
+
+import multiprocessing as mp
+import os
+import time
+
+import numpy as np
+
+from .paged import decode
+
+
+def _init_worker():
+    for v in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ[v] = "1"
+
+
+def decode_task(task):
+    """task = (q_raw [1,Hq,D], q_dtype, k_raw, v_raw, cache_dtype, table [1,W],
+    lens [1], scale, Hkv, k_scale, v_scale) -> (out [1,Hq,D], seconds)."""
+    t0 = time.perf_counter()
+    out = decode(*task)
+    return out, time.perf_counter() - t0
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def run_decode_tasks(tasks, workers: int):
+    """Run tasks on `workers` spawned processes; returns (outputs, wall seconds)."""
+    for v in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        os.environ.setdefault(v, "1")
+    ctx = mp.get_context("spawn")
+    with ctx.Pool(processes=workers, initializer=_init_worker) as pool:
+        pool.map(_noop, range(workers))  # start-up outside the timed region
+        t0 = time.perf_counter()
+        res = pool.map(decode_task, tasks, chunksize=1)
+        wall = time.perf_counter() - t0
+    return [r[0] for r in res], wall
+
+
+def _noop(_):
+    return np.zeros(1)

@@ -1,0 +1,93 @@
+// Cache maintenance kernels: the slot-mapping scatter of new keys/values and
+// the copy-on-write block copy.
+//
+// Both are pure data movement in 16-byte vectors (HBM-bound, and at decode
+// sizes launch-bound).  "PagedAttention" (Ultralytics glossary): token `pos`
+// of a request is stored at key_pool[block_table[pos // bs], pos % bs]
+// (section "Sayfalama Nasil Calisir", PyTorch sketch); a block that other
+// sequences still use is copied before it is written (section "Diziler
+// Arasinda Bloklari Paylasma").
+#pragma once
+
+#include "common.cuh"
+
+namespace pa {
+
+// One thread moves one 16-byte vector of one (token, kv head) row of K or V.
+// 16-bit cache: the words are copied unchanged.  kFP8: the thread reads 8
+// 16-bit inputs (16 bytes) and stores 8 e4m3 codes (8 bytes), each
+// e4m3_rne_satfinite(fp32(x) / scale) with an IEEE fp32 division.
+template <bool kFP8, bool kInBF16>
+__global__ void __launch_bounds__(256) write_kv_kernel(
+    const uint16_t* __restrict__ k, const uint16_t* __restrict__ v,
+    const int64_t* __restrict__ slots, int num_tokens, uint8_t* __restrict__ k_pool,
+    uint8_t* __restrict__ v_pool, int64_t num_slots, int hkv, int D, float k_scale,
+    float v_scale) {
+  const int vec_per_row = D / 8;  // 8 input elements per vector
+  const int64_t per_tensor = static_cast<int64_t>(num_tokens) * hkv * vec_per_row;
+  const int64_t total = 2 * per_tensor;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const bool isv = i >= per_tensor;
+    const int64_t e = isv ? i - per_tensor : i;
+    const int c = static_cast<int>(e % vec_per_row);
+    const int64_t th = e / vec_per_row;  // token * hkv + head
+    const int h = static_cast<int>(th % hkv);
+    const int64_t t = th / hkv;
+    const int64_t slot = slots[t];
+    if (slot < 0) continue;  // padding token
+    if (slot >= num_slots) {
+      record_error(PA_ERR_DEVICE_BOUNDS);
+      continue;
+    }
+    const uint4 x = *reinterpret_cast<const uint4*>((isv ? v : k) + th * D + c * 8);
+    const int64_t dst_elem = (slot * hkv + h) * D + c * 8;
+    uint8_t* pool = isv ? v_pool : k_pool;
+    if constexpr (!kFP8) {
+      *reinterpret_cast<uint4*>(pool + dst_elem * 2) = x;
+    } else {
+      const float s = isv ? v_scale : k_scale;
+      const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+      uint32_t outw[2];
+#pragma unroll
+      for (int p = 0; p < 2; ++p) {
+        const float f0 = __fdiv_rn(to_float<kInBF16>(w[2 * p] & 0xffff), s);
+        const float f1 = __fdiv_rn(to_float<kInBF16>(w[2 * p] >> 16), s);
+        const float f2 = __fdiv_rn(to_float<kInBF16>(w[2 * p + 1] & 0xffff), s);
+        const float f3 = __fdiv_rn(to_float<kInBF16>(w[2 * p + 1] >> 16), s);
+        outw[p] = static_cast<uint32_t>(f32x2_to_e4m3x2(f0, f1)) |
+                  (static_cast<uint32_t>(f32x2_to_e4m3x2(f2, f3)) << 16);
+      }
+      *reinterpret_cast<uint2*>(pool + dst_elem) = make_uint2(outw[0], outw[1]);
+    }
+  }
+}
+
+// Grid (x: pair, y: CTAs per pair).  Each pair copies block_bytes of K and of
+// V from src to dst in 16-byte vectors.
+__global__ void __launch_bounds__(256) copy_blocks_kernel(uint8_t* __restrict__ k_pool,
+                                                          uint8_t* __restrict__ v_pool,
+                                                          const int64_t* __restrict__ pairs,
+                                                          int64_t num_blocks,
+                                                          int64_t block_bytes) {
+  const int64_t p = blockIdx.x;
+  const int64_t src = pairs[2 * p], dst = pairs[2 * p + 1];
+  if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+    if (blockIdx.y == 0 && threadIdx.x == 0) record_error(PA_ERR_DEVICE_BOUNDS);
+    return;
+  }
+  const int64_t nvec = block_bytes / 16;
+  const uint4* ks = reinterpret_cast<const uint4*>(k_pool + src * block_bytes);
+  const uint4* vs = reinterpret_cast<const uint4*>(v_pool + src * block_bytes);
+  uint4* kd = reinterpret_cast<uint4*>(k_pool + dst * block_bytes);
+  uint4* vd = reinterpret_cast<uint4*>(v_pool + dst * block_bytes);
+  for (int64_t i = blockIdx.y * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nvec;
+       i += static_cast<int64_t>(gridDim.y) * blockDim.x) {
+    const uint4 a = ks[i];
+    const uint4 b = vs[i];
+    kd[i] = a;
+    vd[i] = b;
+  }
+}
+
+}  // namespace pa

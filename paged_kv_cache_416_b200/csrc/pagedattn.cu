@@ -1,0 +1,430 @@
+// Host side of libpagedattn.so: argument validation, kernel selection,
+// workspace layout and the C entry points declared in include/pagedattn.h.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <vector>
+
+#include "cache_ops.cuh"
+#include "common.cuh"
+#include "decode.cuh"
+
+namespace {
+
+thread_local char g_msg[1024] = "";
+
+pa_status fail(pa_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+pa_status ok() {
+  g_msg[0] = '\0';
+  return PA_OK;
+}
+
+pa_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(PA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+constexpr int kMaxDevices = 64;
+
+int current_device(int* dev) {
+  const cudaError_t e = cudaGetDevice(dev);
+  if (e != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) return -1;
+  return 0;
+}
+
+// SM count of the current device (cached per device).
+int device_sms(int dev) {
+  static int cache[kMaxDevices] = {0};
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 1;
+  }
+  return cache[dev];
+}
+
+int elem_bytes(pa_dtype t) { return t == PA_FP8_E4M3 ? 1 : 2; }
+
+bool valid_dtype(int t) { return t == PA_F16 || t == PA_BF16 || t == PA_FP8_E4M3; }
+
+bool cache_shape_ok(int32_t num_blocks, int32_t bs, int32_t hkv, int32_t d) {
+  return num_blocks > 0 && (bs == 16 || bs == 32) && hkv > 0 && (d == 64 || d == 128);
+}
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+int64_t round_up(int64_t a, int64_t b) { return cdiv(a, b) * b; }
+
+// ------------------------------------------------------------- split rule
+// Persistent CTAs the split rule plans for (two per SM of a 148-SM B200);
+// fixed so that the split, and so the rounding of every result, depends on
+// the call's arguments only and not on the device it runs on.
+constexpr int64_t kPlanCtas = 296;
+constexpr int64_t kMinSplit = 256;        // shortest range worth its partial
+constexpr int64_t kLongContext = 4096;    // above this, cap ranges ...
+constexpr int64_t kLongSplit = 1024;      // ... at this many tokens
+
+int32_t choose_split(int32_t B, int32_t hkv, int32_t bs, int32_t max_ctx, int32_t user) {
+  if (user > 0) return static_cast<int32_t>(round_up(user, bs));
+  if (max_ctx <= 0) return bs;
+  const int64_t units = static_cast<int64_t>(B) * hkv;
+  // enough ranges for two waves of persistent CTAs ...
+  int64_t s = cdiv(units * max_ctx, 2 * kPlanCtas);
+  s = std::max<int64_t>(kMinSplit, std::min<int64_t>(max_ctx, s));
+  // ... and no single range much longer than the typical one when lengths
+  // can spread far (long contexts): the longest sequence is cut up
+  if (max_ctx > kLongContext) s = std::min<int64_t>(s, kLongSplit);
+  return static_cast<int32_t>(round_up(s, bs));
+}
+
+struct WsLayout {
+  size_t counter = 0, total = 4, seq_off = 256, lse = 0, o = 0, bytes = 0;
+  bool split = false;
+};
+
+WsLayout ws_layout(int32_t B, int32_t hq, int32_t D, int32_t max_ctx, int32_t S) {
+  WsLayout w;
+  w.lse = w.seq_off + static_cast<size_t>(round_up(static_cast<int64_t>(B + 1) * 4, 256));
+  w.split = S < max_ctx;
+  if (!w.split) {
+    w.o = w.lse;
+    w.bytes = w.lse;
+    return w;
+  }
+  const int64_t ranges = static_cast<int64_t>(B) * cdiv(max_ctx, S);
+  w.o = w.lse + static_cast<size_t>(round_up(ranges * hq * 4, 256));
+  w.bytes = w.o + static_cast<size_t>(ranges * hq * D * 4);
+  return w;
+}
+
+// ------------------------------------------------------ decode dispatch
+template <int CK, bool kQBF16, int D, int BS>
+pa_status launch_decode_main(const pa::DecodeArgs& args, int64_t items_upper, int dev,
+                             cudaStream_t stream) {
+  using C = pa::DecodeCfg<CK, D, BS>;
+  auto kern = pa::decode_kernel<CK, kQBF16, D, BS>;
+  static int occ[kMaxDevices] = {0};
+  if (occ[dev] == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, pa::kDecodeThreads, C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "occupancy(decode)");
+    occ[dev] = n > 0 ? n : 1;
+  }
+  const int64_t grid = std::max<int64_t>(
+      1, std::min<int64_t>(items_upper, static_cast<int64_t>(device_sms(dev)) * occ[dev]));
+  kern<<<static_cast<unsigned>(grid), pa::kDecodeThreads, C::kSmemBytes, stream>>>(args);
+  return PA_OK;
+}
+
+template <int CK, bool kQBF16>
+pa_status dispatch_shape(const pa::DecodeArgs& a, int D, int BS, int64_t items, int dev,
+                         cudaStream_t st) {
+  if (D == 128 && BS == 16) return launch_decode_main<CK, kQBF16, 128, 16>(a, items, dev, st);
+  if (D == 128 && BS == 32) return launch_decode_main<CK, kQBF16, 128, 32>(a, items, dev, st);
+  if (D == 64 && BS == 16) return launch_decode_main<CK, kQBF16, 64, 16>(a, items, dev, st);
+  if (D == 64 && BS == 32) return launch_decode_main<CK, kQBF16, 64, 32>(a, items, dev, st);
+  return fail(PA_ERR_SHAPE, "head_dim %d / block_size %d not supported", D, BS);
+}
+
+// Copy n indices to the host (debug checks only).
+template <typename T>
+pa_status fetch(std::vector<T>& h, const T* d, size_t n, cudaStream_t st, const char* what) {
+  h.resize(n);
+  if (n == 0) return PA_OK;
+  cudaError_t e = cudaMemcpyAsync(h.data(), d, n * sizeof(T), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return PA_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* pa_last_error(void) { return g_msg; }
+
+pa_status pa_write_kv(const void* k, const void* v, pa_dtype in_dtype,
+                      const int64_t* slot_mapping, int32_t num_tokens, void* k_pool,
+                      void* v_pool, pa_dtype cache_dtype, int32_t num_blocks,
+                      int32_t block_size, int32_t num_kv_heads, int32_t head_dim,
+                      float k_scale, float v_scale, pa_stream_t stream) {
+  if (!valid_dtype(in_dtype) || !valid_dtype(cache_dtype))
+    return fail(PA_ERR_DTYPE, "pa_write_kv: unknown dtype");
+  if (in_dtype == PA_FP8_E4M3)
+    return fail(PA_ERR_DTYPE, "pa_write_kv: inputs must be f16 or bf16");
+  if (cache_dtype != PA_FP8_E4M3 && cache_dtype != in_dtype)
+    return fail(PA_ERR_DTYPE, "pa_write_kv: a 16-bit cache must have the input dtype");
+  if (num_tokens < 0 || !cache_shape_ok(num_blocks, block_size, num_kv_heads, head_dim))
+    return fail(PA_ERR_SHAPE, "pa_write_kv: unsupported sizes (tokens %d, blocks %d, bs %d, "
+                "heads %d, dim %d)", num_tokens, num_blocks, block_size, num_kv_heads, head_dim);
+  if (cache_dtype == PA_FP8_E4M3 &&
+      !(std::isfinite(k_scale) && k_scale > 0.f && std::isfinite(v_scale) && v_scale > 0.f))
+    return fail(PA_ERR_SHAPE, "pa_write_kv: e4m3 scales must be finite and positive");
+  if (num_tokens == 0) return ok();
+  if (!k || !v || !slot_mapping || !k_pool || !v_pool)
+    return fail(PA_ERR_NULL, "pa_write_kv: null pointer");
+  int dev;
+  if (current_device(&dev)) return fail(PA_ERR_CUDA, "pa_write_kv: no current device");
+  const int64_t total = 2LL * num_tokens * num_kv_heads * (head_dim / 8);
+  const int64_t grid = std::max<int64_t>(
+      1, std::min<int64_t>(cdiv(total, 256), static_cast<int64_t>(device_sms(dev)) * 8));
+  const int64_t num_slots = static_cast<int64_t>(num_blocks) * block_size;
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  const auto* kk = static_cast<const uint16_t*>(k);
+  const auto* vv = static_cast<const uint16_t*>(v);
+  auto* kp = static_cast<uint8_t*>(k_pool);
+  auto* vp = static_cast<uint8_t*>(v_pool);
+  const unsigned g = static_cast<unsigned>(grid);
+  if (cache_dtype != PA_FP8_E4M3)
+    pa::write_kv_kernel<false, false><<<g, 256, 0, st>>>(kk, vv, slot_mapping, num_tokens, kp, vp,
+                                                         num_slots, num_kv_heads, head_dim, 1.f, 1.f);
+  else if (in_dtype == PA_BF16)
+    pa::write_kv_kernel<true, true><<<g, 256, 0, st>>>(kk, vv, slot_mapping, num_tokens, kp, vp,
+                                                       num_slots, num_kv_heads, head_dim, k_scale, v_scale);
+  else
+    pa::write_kv_kernel<true, false><<<g, 256, 0, st>>>(kk, vv, slot_mapping, num_tokens, kp, vp,
+                                                        num_slots, num_kv_heads, head_dim, k_scale, v_scale);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pa_write_kv launch");
+  return ok();
+}
+
+pa_status pa_copy_blocks(void* k_pool, void* v_pool, pa_dtype cache_dtype, int32_t num_blocks,
+                         int32_t block_size, int32_t num_kv_heads, int32_t head_dim,
+                         const int64_t* src_dst_pairs, int32_t num_pairs, pa_stream_t stream) {
+  if (!valid_dtype(cache_dtype)) return fail(PA_ERR_DTYPE, "pa_copy_blocks: unknown dtype");
+  if (num_pairs < 0 || !cache_shape_ok(num_blocks, block_size, num_kv_heads, head_dim))
+    return fail(PA_ERR_SHAPE, "pa_copy_blocks: unsupported sizes");
+  if (num_pairs == 0) return ok();
+  if (!k_pool || !v_pool || !src_dst_pairs) return fail(PA_ERR_NULL, "pa_copy_blocks: null pointer");
+  const int64_t block_bytes =
+      static_cast<int64_t>(block_size) * num_kv_heads * head_dim * elem_bytes(cache_dtype);
+  const int64_t nvec = block_bytes / 16;
+  const unsigned per_pair = static_cast<unsigned>(std::min<int64_t>(8, cdiv(nvec, 256)));
+  dim3 grid(static_cast<unsigned>(num_pairs), per_pair);
+  pa::copy_blocks_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint8_t*>(k_pool), static_cast<uint8_t*>(v_pool), src_dst_pairs, num_blocks,
+      block_bytes);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pa_copy_blocks launch");
+  return ok();
+}
+
+int32_t pa_decode_split_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t block_size,
+                               int32_t max_context_len, int32_t split_tokens) {
+  if (num_seqs < 0 || num_kv_heads <= 0 || (block_size != 16 && block_size != 32) ||
+      max_context_len < 0 || split_tokens < 0)
+    return 0;
+  return choose_split(num_seqs, num_kv_heads, block_size, max_context_len, split_tokens);
+}
+
+size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                int32_t head_dim, int32_t block_size, int32_t max_context_len,
+                                int32_t split_tokens) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || (head_dim != 64 && head_dim != 128) ||
+      (block_size != 16 && block_size != 32) || max_context_len < 0 || split_tokens < 0)
+    return 0;
+  const int32_t S = choose_split(num_seqs, num_kv_heads, block_size, max_context_len, split_tokens);
+  return ws_layout(num_seqs, num_q_heads, head_dim, max_context_len, S).bytes;
+}
+
+pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_pool,
+                    const void* v_pool, pa_dtype cache_dtype, const int32_t* block_tables,
+                    int32_t max_blocks_per_seq, const int32_t* context_lens,
+                    int32_t max_context_len, int32_t num_seqs, int32_t num_q_heads,
+                    int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                    int32_t num_blocks, float scale, float k_scale, float v_scale,
+                    int32_t split_tokens, void* workspace, size_t workspace_bytes,
+                    pa_stream_t stream) {
+  if (!valid_dtype(q_dtype) || !valid_dtype(cache_dtype))
+    return fail(PA_ERR_DTYPE, "pa_decode: unknown dtype");
+  const bool fp8 = cache_dtype == PA_FP8_E4M3;
+  if (q_dtype == PA_FP8_E4M3 || (!fp8 && q_dtype != cache_dtype))
+    return fail(PA_ERR_DTYPE, "pa_decode: q must be f16/bf16 and match a 16-bit cache");
+  if (num_seqs < 0 || max_blocks_per_seq <= 0 || max_context_len < 0 || split_tokens < 0 ||
+      !cache_shape_ok(num_blocks, block_size, num_kv_heads, head_dim))
+    return fail(PA_ERR_SHAPE, "pa_decode: unsupported sizes (seqs %d, max_blocks %d, max_ctx %d, "
+                "blocks %d, bs %d, kv heads %d, dim %d)", num_seqs, max_blocks_per_seq,
+                max_context_len, num_blocks, block_size, num_kv_heads, head_dim);
+  if (static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * block_size)
+    return fail(PA_ERR_SHAPE, "pa_decode: max_context_len %d exceeds max_blocks_per_seq * bs",
+                max_context_len);
+  if (num_q_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
+      num_q_heads / num_kv_heads > pa::kMaxGroup)
+    return fail(PA_ERR_HEADS, "pa_decode: num_q_heads %d must be a multiple of num_kv_heads %d "
+                "with at most %d query heads per kv head", num_q_heads, num_kv_heads, pa::kMaxGroup);
+  if (!std::isfinite(scale) || (fp8 && !(std::isfinite(k_scale) && k_scale > 0.f &&
+                                         std::isfinite(v_scale) && v_scale > 0.f)))
+    return fail(PA_ERR_SHAPE, "pa_decode: scales must be finite (and positive for e4m3)");
+  if (num_seqs == 0) return ok();
+  if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens)
+    return fail(PA_ERR_NULL, "pa_decode: null pointer");
+  const int32_t S = choose_split(num_seqs, num_kv_heads, block_size, max_context_len, split_tokens);
+  const WsLayout w = ws_layout(num_seqs, num_q_heads, head_dim, max_context_len, S);
+  if (!workspace || workspace_bytes < w.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return fail(PA_ERR_WORKSPACE, "pa_decode: workspace needs %zu bytes, 256-byte aligned (got %zu)",
+                w.bytes, workspace_bytes);
+  int dev;
+  if (current_device(&dev)) return fail(PA_ERR_CUDA, "pa_decode: no current device");
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  auto* ws = static_cast<uint8_t*>(workspace);
+
+  pa::DecodeArgs a;
+  a.out = out;
+  a.q = q;
+  a.k_pool = static_cast<const uint8_t*>(k_pool);
+  a.v_pool = static_cast<const uint8_t*>(v_pool);
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.counter = reinterpret_cast<int32_t*>(ws + w.counter);
+  a.total = reinterpret_cast<const int32_t*>(ws + w.total);
+  a.seq_off = reinterpret_cast<const int32_t*>(ws + w.seq_off);
+  a.lse_part = reinterpret_cast<float*>(ws + w.lse);
+  a.o_part = reinterpret_cast<float*>(ws + w.o);
+  a.num_seqs = num_seqs;
+  a.hq = num_q_heads;
+  a.hkv = num_kv_heads;
+  a.group = num_q_heads / num_kv_heads;
+  a.max_blocks = max_blocks_per_seq;
+  a.num_blocks = num_blocks;
+  a.max_ctx = max_context_len;
+  a.split_tokens = w.split ? S : std::max(S, max_context_len);
+  a.sl2 = scale * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
+  a.out_scale = fp8 ? v_scale : 1.f;
+
+  pa::plan_kernel<<<1, 1024, 0, st>>>(context_lens, num_seqs, max_context_len, max_blocks_per_seq,
+                                      block_size, a.split_tokens, num_kv_heads,
+                                      reinterpret_cast<int32_t*>(ws + w.counter),
+                                      reinterpret_cast<int32_t*>(ws + w.total),
+                                      reinterpret_cast<int32_t*>(ws + w.seq_off));
+  const int64_t ranges_upper =
+      w.split ? static_cast<int64_t>(num_seqs) * cdiv(max_context_len, S) : num_seqs;
+  const int64_t items_upper = ranges_upper * num_kv_heads;
+  const bool qbf = q_dtype == PA_BF16;
+  pa_status s;
+  if (cache_dtype == PA_F16)
+    s = dispatch_shape<pa::kCacheF16, false>(a, head_dim, block_size, items_upper, dev, st);
+  else if (cache_dtype == PA_BF16)
+    s = dispatch_shape<pa::kCacheBF16, true>(a, head_dim, block_size, items_upper, dev, st);
+  else if (qbf)
+    s = dispatch_shape<pa::kCacheE4M3, true>(a, head_dim, block_size, items_upper, dev, st);
+  else
+    s = dispatch_shape<pa::kCacheE4M3, false>(a, head_dim, block_size, items_upper, dev, st);
+  if (s != PA_OK) return s;
+  if (w.split) {
+    const int units = num_q_heads * (head_dim / 4);
+    dim3 grid(static_cast<unsigned>(cdiv(units, 128)), static_cast<unsigned>(num_seqs));
+    if (qbf)
+      pa::merge_kernel<true><<<grid, 128, 0, st>>>(out, a.lse_part, a.o_part, a.seq_off,
+                                                   num_q_heads, head_dim);
+    else
+      pa::merge_kernel<false><<<grid, 128, 0, st>>>(out, a.lse_part, a.o_part, a.seq_off,
+                                                    num_q_heads, head_dim);
+  }
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
+  return ok();
+}
+
+pa_status pa_sync_status(pa_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "pa_sync_status: stream");
+  int v = 0;
+  e = cudaMemcpyFromSymbol(&v, pa::g_device_error, sizeof(int));
+  if (e != cudaSuccess) return cuda_fail(e, "pa_sync_status: read error word");
+  if (v != 0) {
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(pa::g_device_error, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "pa_sync_status: clear error word");
+    if (v == PA_ERR_TIMEOUT)
+      return fail(PA_ERR_TIMEOUT, "a kernel gave up waiting for an asynchronous copy");
+    return fail(static_cast<pa_status>(v), "a kernel met an out-of-range index and skipped it");
+  }
+  return ok();
+}
+
+// ------------------------------------------------------------- debug checks
+pa_status pa_validate_slot_mapping(const int64_t* slot_mapping, int32_t num_tokens,
+                                   int32_t num_blocks, int32_t block_size, pa_stream_t stream) {
+  if (num_tokens < 0 || num_blocks <= 0 || block_size <= 0)
+    return fail(PA_ERR_SHAPE, "pa_validate_slot_mapping: bad sizes");
+  if (num_tokens > 0 && !slot_mapping) return fail(PA_ERR_NULL, "pa_validate_slot_mapping: null");
+  std::vector<int64_t> h;
+  pa_status s = fetch(h, slot_mapping, num_tokens, reinterpret_cast<cudaStream_t>(stream),
+                      "pa_validate_slot_mapping");
+  if (s != PA_OK) return s;
+  const int64_t n = static_cast<int64_t>(num_blocks) * block_size;
+  std::vector<uint8_t> seen(static_cast<size_t>(n), 0);
+  for (int32_t t = 0; t < num_tokens; ++t) {
+    if (h[t] < 0) continue;
+    if (h[t] >= n) return fail(PA_ERR_RANGE, "slot_mapping[%d] = %lld is outside the pool", t, (long long)h[t]);
+    if (seen[h[t]]++) return fail(PA_ERR_ALIAS, "slot %lld is written twice", (long long)h[t]);
+  }
+  return ok();
+}
+
+pa_status pa_validate_copy_pairs(const int64_t* src_dst_pairs, int32_t num_pairs,
+                                 int32_t num_blocks, pa_stream_t stream) {
+  if (num_pairs < 0 || num_blocks <= 0) return fail(PA_ERR_SHAPE, "pa_validate_copy_pairs: bad sizes");
+  if (num_pairs > 0 && !src_dst_pairs) return fail(PA_ERR_NULL, "pa_validate_copy_pairs: null");
+  std::vector<int64_t> h;
+  pa_status s = fetch(h, src_dst_pairs, 2 * static_cast<size_t>(num_pairs),
+                      reinterpret_cast<cudaStream_t>(stream), "pa_validate_copy_pairs");
+  if (s != PA_OK) return s;
+  std::vector<uint8_t> role(static_cast<size_t>(num_blocks), 0);  // 1 src, 2 dst
+  for (int32_t p = 0; p < num_pairs; ++p)
+    for (int k = 0; k < 2; ++k)
+      if (h[2 * p + k] < 0 || h[2 * p + k] >= num_blocks)
+        return fail(PA_ERR_RANGE, "pair %d holds block id %lld outside the pool", p,
+                    (long long)h[2 * p + k]);
+  for (int32_t p = 0; p < num_pairs; ++p) role[h[2 * p]] |= 1;
+  for (int32_t p = 0; p < num_pairs; ++p) {
+    const int64_t d = h[2 * p + 1];
+    if (role[d] & 2) return fail(PA_ERR_ALIAS, "block %lld is a destination twice", (long long)d);
+    if (role[d] & 1) return fail(PA_ERR_ALIAS, "block %lld is both a source and a destination", (long long)d);
+    role[d] |= 2;
+  }
+  return ok();
+}
+
+pa_status pa_validate_block_tables(const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                   const int32_t* context_lens, int32_t num_seqs,
+                                   int32_t max_context_len, int32_t block_size, int32_t num_blocks,
+                                   pa_stream_t stream) {
+  if (num_seqs < 0 || max_blocks_per_seq <= 0 || block_size <= 0 || num_blocks <= 0)
+    return fail(PA_ERR_SHAPE, "pa_validate_block_tables: bad sizes");
+  if (num_seqs > 0 && (!block_tables || !context_lens))
+    return fail(PA_ERR_NULL, "pa_validate_block_tables: null");
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  std::vector<int32_t> t, c;
+  pa_status s = fetch(c, context_lens, num_seqs, st, "pa_validate_block_tables");
+  if (s == PA_OK)
+    s = fetch(t, block_tables, static_cast<size_t>(num_seqs) * max_blocks_per_seq, st,
+              "pa_validate_block_tables");
+  if (s != PA_OK) return s;
+  for (int32_t i = 0; i < num_seqs; ++i) {
+    if (c[i] < 0 || c[i] > max_context_len)
+      return fail(PA_ERR_RANGE, "context_lens[%d] = %d outside [0, %d]", i, c[i], max_context_len);
+    const int64_t nb = cdiv(c[i], block_size);
+    if (nb > max_blocks_per_seq)
+      return fail(PA_ERR_RANGE, "sequence %d needs %lld blocks, table holds %d", i, (long long)nb,
+                  max_blocks_per_seq);
+    for (int64_t j = 0; j < nb; ++j) {
+      const int32_t b = t[static_cast<size_t>(i) * max_blocks_per_seq + j];
+      if (b < 0 || b >= num_blocks)
+        return fail(PA_ERR_RANGE, "block_tables[%d][%lld] = %d outside the pool", i, (long long)j, b);
+    }
+  }
+  return ok();
+}
+
+}  // extern "C"

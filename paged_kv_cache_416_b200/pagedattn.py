@@ -1,0 +1,197 @@
+"""ctypes binding of libpagedattn.so (the C ABI in include/pagedattn.h).
+
+Argument marshalling only: every step of the hot path runs in the library's
+CUDA kernels.  Importing this module loads the library and raises if it is
+missing -- there is no CPU fallback.  torch supplies device memory and
+streams.
+
+Two layers:
+* ``pa_*``: the C entry points themselves, with ctypes signatures (raw
+  pointers, sizes, dtype codes, stream handles);
+* ``write_kv``, ``copy_blocks``, ``decode``, ``decode_workspace_size``,
+  ``sync_status``: the same calls taking torch tensors, which read pointers,
+  sizes and dtypes off the tensors and pass the current torch stream.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedattn.so")
+
+PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
+STATUS_NAMES = {
+    0: "PA_OK", 1: "PA_ERR_NULL", 2: "PA_ERR_DTYPE", 3: "PA_ERR_SHAPE", 4: "PA_ERR_HEADS",
+    5: "PA_ERR_RANGE", 6: "PA_ERR_ALIAS", 7: "PA_ERR_CUDA", 8: "PA_ERR_DEVICE_BOUNDS",
+    9: "PA_ERR_WORKSPACE", 10: "PA_ERR_TIMEOUT",
+}
+_TORCH_TO_PA = {torch.float16: PA_F16, torch.bfloat16: PA_BF16, torch.float8_e4m3fn: PA_FP8_E4M3}
+
+
+class PagedAttnError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {message}")
+        self.status = status
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing; build it with `python -m paged_kv_cache_416_b200.build` "
+            "(there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, F, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "pa_write_kv": (I32, [P, P, I32, P, I32, P, P, I32, I32, I32, I32, I32, F, F, P]),
+        "pa_copy_blocks": (I32, [P, P, I32, I32, I32, I32, I32, P, I32, P]),
+        "pa_decode_split_tokens": (I32, [I32, I32, I32, I32, I32]),
+        "pa_decode_workspace_size": (SZ, [I32, I32, I32, I32, I32, I32, I32]),
+        "pa_decode": (I32, [P, P, I32, P, P, I32, P, I32, P, I32, I32, I32, I32, I32, I32, I32,
+                            F, F, F, I32, P, SZ, P]),
+        "pa_sync_status": (I32, [P]),
+        "pa_last_error": (ctypes.c_char_p, []),
+        "pa_validate_slot_mapping": (I32, [P, I32, I32, I32, P]),
+        "pa_validate_copy_pairs": (I32, [P, I32, I32, P]),
+        "pa_validate_block_tables": (I32, [P, I32, P, I32, I32, I32, I32, P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+# the C entry points, unchanged
+pa_write_kv = _lib.pa_write_kv
+pa_copy_blocks = _lib.pa_copy_blocks
+pa_decode_split_tokens = _lib.pa_decode_split_tokens
+pa_decode_workspace_size = _lib.pa_decode_workspace_size
+pa_decode = _lib.pa_decode
+pa_sync_status = _lib.pa_sync_status
+pa_last_error = _lib.pa_last_error
+pa_validate_slot_mapping = _lib.pa_validate_slot_mapping
+pa_validate_copy_pairs = _lib.pa_validate_copy_pairs
+pa_validate_block_tables = _lib.pa_validate_block_tables
+
+ENTRY_POINTS = [
+    "pa_write_kv", "pa_copy_blocks", "pa_decode_split_tokens", "pa_decode_workspace_size",
+    "pa_decode", "pa_sync_status", "pa_last_error", "pa_validate_slot_mapping",
+    "pa_validate_copy_pairs", "pa_validate_block_tables",
+]
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def check(status: int) -> None:
+    """Raise PagedAttnError for a non-zero status, with pa_last_error()."""
+    if status != 0:
+        msg = _lib.pa_last_error()
+        raise PagedAttnError(status, msg.decode() if msg else "")
+
+
+# ----------------------------------------------------------- tensor helpers
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype(t: torch.Tensor, override: Optional[int] = None) -> int:
+    if override is not None:
+        return override
+    if t.dtype not in _TORCH_TO_PA:
+        raise TypeError(f"unsupported dtype {t.dtype}")
+    return _TORCH_TO_PA[t.dtype]
+
+
+def _contig(*ts):
+    for t in ts:
+        if t is not None and not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+
+
+def write_kv(k, v, slot_mapping, k_pool, v_pool, k_scale: float = 1.0, v_scale: float = 1.0,
+             stream=None) -> None:
+    """pa_write_kv on tensors: k, v [T, Hkv, D] (f16/bf16), slot_mapping int64 [T],
+    pools [N, bs, Hkv, D] (k's dtype, or float8_e4m3fn)."""
+    _contig(k, v, slot_mapping, k_pool, v_pool)
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    N, bs, hkv, d = k_pool.shape
+    check(pa_write_kv(_ptr(k), _ptr(v), _dtype(k), _ptr(slot_mapping), k.shape[0], _ptr(k_pool),
+                      _ptr(v_pool), _dtype(k_pool), N, bs, hkv, d, float(k_scale), float(v_scale),
+                      _stream(stream)))
+
+
+def copy_blocks(k_pool, v_pool, pairs, stream=None) -> None:
+    """pa_copy_blocks on tensors: pairs int64 [P, 2] of (src, dst) block ids."""
+    _contig(k_pool, v_pool, pairs)
+    if pairs.dtype != torch.int64:
+        raise TypeError("pairs must be int64")
+    N, bs, hkv, d = k_pool.shape
+    check(pa_copy_blocks(_ptr(k_pool), _ptr(v_pool), _dtype(k_pool), N, bs, hkv, d, _ptr(pairs),
+                         pairs.shape[0], _stream(stream)))
+
+
+def decode_split_tokens(num_seqs, num_kv_heads, block_size, max_context_len, split_tokens=0) -> int:
+    return int(pa_decode_split_tokens(num_seqs, num_kv_heads, block_size, max_context_len,
+                                      split_tokens))
+
+
+def decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                          max_context_len, split_tokens=0) -> int:
+    return int(pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                                        max_context_len, split_tokens))
+
+
+_ws_cache = {}
+
+
+def workspace_for(device, nbytes: int) -> torch.Tensor:
+    """A cached device byte buffer of at least nbytes (torch-allocated)."""
+    key = torch.device(device)
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=key)
+        _ws_cache[key] = buf
+    return buf
+
+
+def decode(q, k_pool, v_pool, block_tables, context_lens, scale: float, max_context_len: int,
+           k_scale: float = 1.0, v_scale: float = 1.0, split_tokens: int = 0, out=None,
+           workspace=None, stream=None) -> torch.Tensor:
+    """pa_decode on tensors.  q [B, Hq, D]; pools [N, bs, Hkv, D]; block_tables
+    int32 [B, W]; context_lens int32 [B].  Returns out [B, Hq, D] (q's dtype)."""
+    _contig(q, k_pool, v_pool, block_tables, context_lens)
+    if block_tables.dtype != torch.int32 or context_lens.dtype != torch.int32:
+        raise TypeError("block_tables and context_lens must be int32")
+    B, hq, d = q.shape
+    N, bs, hkv, d2 = k_pool.shape
+    if out is None:
+        out = torch.empty_like(q)
+    nbytes = decode_workspace_size(B, hq, hkv, d, bs, max_context_len, split_tokens)
+    if workspace is None:
+        workspace = workspace_for(q.device, nbytes)
+    check(pa_decode(_ptr(out), _ptr(q), _dtype(q), _ptr(k_pool), _ptr(v_pool), _dtype(k_pool),
+                    _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+                    int(max_context_len), B, hq, hkv, d, bs, N, float(scale), float(k_scale),
+                    float(v_scale), int(split_tokens), _ptr(workspace), workspace.numel(),
+                    _stream(stream)))
+    return out
+
+
+def sync_status(stream=None) -> None:
+    """pa_sync_status: synchronise and raise if a kernel reported an error."""
+    check(pa_sync_status(_stream(stream)))

@@ -1,0 +1,108 @@
+"""The C-ABI library loads and exports every entry point its header declares;
+host-side validation rejects bad arguments before any CUDA call (CPU only)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_416_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "pagedattn.h")
+
+
+@pytest.fixture(scope="module")
+def pa():
+    build.build()  # nvcc cross-compiles without a GPU; no-op when up to date
+    from paged_kv_cache_416_b200 import pagedattn
+    return pagedattn
+
+
+def declared_entry_points():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(pa_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_hot_path_calls():
+    names = declared_entry_points()
+    for n in ("pa_decode", "pa_write_kv", "pa_copy_blocks", "pa_decode_workspace_size",
+              "pa_sync_status", "pa_last_error"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(pa):
+    lib = ctypes.CDLL(pa.LIB_PATH)
+    for name in declared_entry_points():
+        assert hasattr(lib, name), name
+    assert set(declared_entry_points()) <= set(pa.ENTRY_POINTS)
+
+
+def test_split_and_workspace_rules(pa):
+    # one item per (sequence, kv head) when that fills the GPU
+    assert pa.pa_decode_split_tokens(256, 8, 16, 4096, 0) == 4096
+    assert pa.pa_decode_workspace_size(256, 64, 8, 128, 16, 4096, 0) == 256 + 1280
+    # long contexts are cut into ranges (multiples of the block size)
+    s = pa.pa_decode_split_tokens(128, 8, 16, 32768, 0)
+    assert s == 1024
+    ranges = 128 * 32
+    assert pa.pa_decode_workspace_size(128, 32, 8, 128, 16, 32768, 0) == \
+        256 + 768 + ranges * 32 * 4 + ranges * 32 * 128 * 4
+    # few sequences: split for parallelism
+    s = pa.pa_decode_split_tokens(1, 8, 32, 16384, 0)
+    assert 256 <= s < 16384 and s % 32 == 0
+    # explicit split rounds up to the block size
+    assert pa.pa_decode_split_tokens(4, 4, 16, 1000, 40) == 48
+    assert pa.pa_decode_split_tokens(4, 4, 24, 1000, 0) == 0  # bad block size
+
+
+def _decode(pa, **kw):
+    args = dict(out=None, q=None, q_dtype=1, k_pool=None, v_pool=None, cache_dtype=1,
+                block_tables=None, max_blocks=4, context_lens=None, max_ctx=64, B=2, hq=8, hkv=2,
+                D=128, bs=16, N=32, scale=0.1, k_scale=1.0, v_scale=1.0, split=0, ws=None,
+                ws_bytes=0, stream=None)
+    args.update(kw)
+    return pa.pa_decode(*args.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q_dtype=0, cache_dtype=1), 2),         # q must match a 16-bit cache
+    (dict(q_dtype=2, cache_dtype=2), 2),         # fp8 queries are not supported
+    (dict(q_dtype=7), 2),
+    (dict(D=96), 3),
+    (dict(bs=8), 3),
+    (dict(max_ctx=65), 3),                       # exceeds max_blocks * bs
+    (dict(hq=7), 4),
+    (dict(hq=32, hkv=2), 4),                     # 16 query heads per kv head
+    (dict(cache_dtype=2, k_scale=0.0), 3),
+    (dict(scale=float("inf")), 3),
+    (dict(), 1),                                 # valid sizes, null pointers
+])
+def test_decode_rejects_bad_arguments_on_the_host(pa, kw, status):
+    assert _decode(pa, **kw) == status
+    assert pa.pa_last_error()
+
+
+def test_decode_with_no_sequences_is_a_no_op(pa):
+    assert _decode(pa, B=0) == 0
+
+
+def test_write_and_copy_validation(pa):
+    W = pa.pa_write_kv
+    assert W(None, None, 1, None, 4, None, None, 0, 8, 16, 2, 128, 1.0, 1.0, None) == 2  # bf16 into f16
+    assert W(None, None, 1, None, 4, None, None, 2, 8, 16, 2, 128, 0.0, 1.0, None) == 3  # bad scale
+    assert W(None, None, 1, None, 4, None, None, 1, 8, 12, 2, 128, 1.0, 1.0, None) == 3  # bad bs
+    assert W(None, None, 1, None, 4, None, None, 1, 8, 16, 2, 128, 1.0, 1.0, None) == 1  # nulls
+    assert W(None, None, 1, None, 0, None, None, 1, 8, 16, 2, 128, 1.0, 1.0, None) == 0  # no tokens
+    C = pa.pa_copy_blocks
+    assert C(None, None, 1, 8, 16, 2, 128, None, 0, None) == 0
+    assert C(None, None, 1, 8, 16, 2, 128, None, 3, None) == 1
+    assert C(None, None, 9, 8, 16, 2, 128, None, 3, None) == 2
+
+
+def test_python_binding_raises_with_the_message(pa):
+    with pytest.raises(pa.PagedAttnError) as e:
+        pa.check(_decode(pa, hq=7))
+    assert "PA_ERR_HEADS" in str(e.value)

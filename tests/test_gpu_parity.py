@@ -1,0 +1,342 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle.
+
+Writes and copies: bit-exact.  Attention: |gpu - ref| <= 2e-3 + 1e-2 |ref|
+element by element (fp16 / bf16 caches with fp32 accumulation; for the e4m3
+cache against the oracle run on the dequantised cache).  Workloads are the
+seeded generators of paged_kv_cache_416_b200.workloads at sizes the oracle
+finishes in seconds (several blocks per warp, ragged last blocks), plus the
+benchmark sizes checked on sampled sequences.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from harness import (as_f64, assert_attention_close, compact_oracle_step, gpu_step,
+                     oracle_step)
+from paged_kv_cache_416_b200 import workloads as W
+from paged_kv_cache_416_b200.workloads import raw
+
+pytestmark = pytest.mark.gpu
+
+SMALL = {
+    "tiny": dict(),
+    "llama13b_mha": dict(num_seqs=6),
+    "llama70b_gqa": dict(num_seqs=3),
+    "llama70b_gqa_ragged": dict(num_seqs=5, context_len=1000),
+    "shared_prefix_fork": dict(prompts=3),
+    "shared_prefix_tails": dict(prompts=3),
+    "fp8_longtail_bs16": dict(num_seqs=10, max_len=6000),
+    "fp8_longtail_bs32": dict(num_seqs=10, max_len=6000),
+}
+
+
+def small(name, seed=None, device="cpu"):
+    base = "llama70b_gqa" if name == "llama70b_gqa_ragged" else name
+    return W.make(base, seed=seed, device=device, **SMALL[name])
+
+
+# ------------------------------------------------------------- cache writes
+
+@pytest.mark.parametrize("in_dt,cache_dt", [("f16", "f16"), ("bf16", "bf16"), ("bf16", "e4m3"),
+                                            ("f16", "e4m3")])
+@pytest.mark.parametrize("bs,hkv,d", [(16, 8, 128), (32, 3, 64)])
+def test_write_kv_bit_exact(pa, in_dt, cache_dt, bs, hkv, d):
+    g = torch.Generator().manual_seed(7)
+    N, T = 40, 300
+    td = W.TORCH_DTYPE
+    k = (torch.randn(T, hkv, d, generator=g) * 3).to(td[in_dt])
+    v = (torch.randn(T, hkv, d, generator=g) * 3).to(td[in_dt])
+    # distinct slots, some padding (-1)
+    slots = torch.randperm(N * bs, generator=g)[:T].to(torch.int64)
+    slots[::7] = -1
+    kp = torch.randint(0, 255, (N, bs, hkv, d), generator=g, dtype=torch.uint8)
+    vp = torch.randint(0, 255, (N, bs, hkv, d), generator=g, dtype=torch.uint8)
+    if cache_dt != "e4m3":
+        kp = torch.randint(-30000, 30000, (N, bs, hkv, d), generator=g, dtype=torch.int16).view(td[cache_dt])
+        vp = torch.randint(-30000, 30000, (N, bs, hkv, d), generator=g, dtype=torch.int16).view(td[cache_dt])
+    else:
+        kp, vp = kp.view(torch.float8_e4m3fn), vp.view(torch.float8_e4m3fn)
+    ks, vs = 0.0123, 0.5
+    ok_, ov_ = raw(kp).copy(), raw(vp).copy()
+    oracle.write_kv(raw(k), raw(v), in_dt, slots.numpy(), ok_, ov_, cache_dt, ks, vs)
+    gk, gv = kp.cuda(), vp.cuda()
+    pa.write_kv(k.cuda(), v.cuda(), slots.cuda(), gk, gv, ks, vs)
+    pa.sync_status()
+    assert np.array_equal(raw(gk), ok_)
+    assert np.array_equal(raw(gv), ov_)
+
+
+def test_write_kv_e4m3_edge_values(pa):
+    """Ties, the saturation boundary, subnormals and infinities quantise as
+    the oracle does (RNE, satfinite)."""
+    vals = oracle.e4m3_finite_values()
+    mids = (vals[:-1] + vals[1:]) / 2
+    x = np.concatenate([vals, -vals, mids, -mids, [448.0, 464.0, 480.0, 1e30, np.inf, -np.inf,
+                                                   2.0 ** -10, 2.0 ** -11, 3 * 2.0 ** -11]])
+    x = x.astype(np.float32)
+    d = 128
+    n = -(-len(x) // d) * d
+    x = np.concatenate([x, np.zeros(n - len(x), np.float32)]).reshape(-1, 1, d)
+    # values must be exact in bf16 for this test: keep those that are
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    T = xb.shape[0]
+    slots = torch.arange(T, dtype=torch.int64)
+    kp = torch.zeros(2, 16, 1, d, dtype=torch.float8_e4m3fn)
+    ok_, ov_ = raw(kp).copy(), raw(kp).copy()
+    oracle.write_kv(raw(xb), raw(xb), "bf16", slots.numpy(), ok_, ov_, "e4m3", 1.0, 1.0)
+    gk, gv = kp.cuda(), kp.clone().cuda()
+    pa.write_kv(xb.cuda(), xb.cuda(), slots.cuda(), gk, gv, 1.0, 1.0)
+    pa.sync_status()
+    assert np.array_equal(raw(gk), ok_) and np.array_equal(raw(gv), ov_)
+
+
+# ------------------------------------------------------------- block copies
+
+@pytest.mark.parametrize("cache_dt,bs,hkv,d", [("bf16", 16, 8, 128), ("e4m3", 32, 4, 64),
+                                               ("f16", 16, 40, 128)])
+def test_copy_blocks_bit_exact(pa, cache_dt, bs, hkv, d):
+    g = torch.Generator().manual_seed(3)
+    N = 200
+    kp = torch.randint(0, 255, (N, bs, hkv, d), generator=g, dtype=torch.uint8)
+    vp = torch.randint(0, 255, (N, bs, hkv, d), generator=g, dtype=torch.uint8)
+    if cache_dt != "e4m3":
+        kp = torch.randint(-30000, 30000, (N, bs, hkv, d), generator=g, dtype=torch.int16).view(W.TORCH_DTYPE[cache_dt])
+        vp = torch.randint(-30000, 30000, (N, bs, hkv, d), generator=g, dtype=torch.int16).view(W.TORCH_DTYPE[cache_dt])
+    else:
+        kp, vp = kp.view(torch.float8_e4m3fn), vp.view(torch.float8_e4m3fn)
+    perm = torch.randperm(N, generator=g)
+    pairs = torch.stack([perm[:60], perm[60:120]], 1).to(torch.int64)  # disjoint src / dst
+    ok_, ov_ = raw(kp).copy(), raw(vp).copy()
+    oracle.copy_blocks(ok_, ov_, pairs.numpy())
+    gk, gv = kp.cuda(), vp.cuda()
+    pa.copy_blocks(gk, gv, pairs.cuda())
+    pa.sync_status()
+    assert np.array_equal(raw(gk), ok_) and np.array_equal(raw(gv), ov_)
+
+
+def test_copy_then_write_leaves_the_source_intact(pa):
+    """After a copy-on-write the two blocks are equal; a write into the copy
+    leaves the source untouched."""
+    kp = torch.randn(8, 16, 2, 64).to(torch.bfloat16).cuda()
+    vp = torch.randn(8, 16, 2, 64).to(torch.bfloat16).cuda()
+    src0k, src0v = kp[3].clone(), vp[3].clone()
+    pa.copy_blocks(kp, vp, torch.tensor([[3, 5]], dtype=torch.int64, device="cuda"))
+    pa.sync_status()
+    assert torch.equal(kp[5], src0k) and torch.equal(vp[5], src0v)
+    new = torch.randn(1, 2, 64).to(torch.bfloat16).cuda()
+    pa.write_kv(new, new, torch.tensor([5 * 16 + 7], dtype=torch.int64, device="cuda"), kp, vp)
+    pa.sync_status()
+    assert torch.equal(kp[5, 7], new[0]) and torch.equal(kp[3], src0k)
+
+
+# ------------------------------------------------------------------ decode
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_decode_step_matches_oracle(pa, name):
+    w = small(name)
+    out, kp, vp = gpu_step(pa, w)
+    ref, okp, ovp = oracle_step(w)
+    # the step's writes and copies are bit-exact
+    assert np.array_equal(raw(kp), okp) and np.array_equal(raw(vp), ovp)
+    assert_attention_close(as_f64(out), ref, name)
+
+
+@pytest.mark.parametrize("name", ["fp8_longtail_bs16", "llama70b_gqa_ragged", "tiny",
+                                  "shared_prefix_tails"])
+def test_decode_split_size_does_not_change_the_result(pa, name):
+    w = small(name)
+    ref, _, _ = oracle_step(w)
+    bs = w.block_size
+    outs = []
+    for split in (bs, 3 * bs, 256, 0, 1 << 20):
+        out, _, _ = gpu_step(pa, w, split_tokens=split)
+        assert_attention_close(as_f64(out), ref, f"{name} split {split}")
+        outs.append(out)
+    # the same call twice gives bit-identical output
+    again, _, _ = gpu_step(pa, w, split_tokens=3 * bs)
+    assert torch.equal(again, outs[1])
+
+
+def test_decode_is_independent_of_physical_placement(pa):
+    """Permuting physical block ids (contents moved along) gives a
+    bit-identical output."""
+    w = small("fp8_longtail_bs16")
+    out1, _, _ = gpu_step(pa, w)
+    g = torch.Generator().manual_seed(99)
+    perm = torch.randperm(w.num_blocks, generator=g)  # old id i -> new id perm[i]
+    kp2 = torch.empty_like(w.k_pool)
+    vp2 = torch.empty_like(w.v_pool)
+    kp2[perm] = w.k_pool
+    vp2[perm] = w.v_pool
+    bt = w.block_tables.copy()
+    m = bt >= 0
+    bt[m] = perm.numpy()[bt[m]]
+    slots = w.slot_mapping.copy()
+    ok_ = slots >= 0
+    slots[ok_] = perm.numpy()[slots[ok_] // w.block_size] * w.block_size + slots[ok_] % w.block_size
+    w2 = W.Workload(**{**w.__dict__, "k_pool": kp2, "v_pool": vp2, "block_tables": bt,
+                       "slot_mapping": slots})
+    out2, _, _ = gpu_step(pa, w2)
+    assert torch.equal(out1, out2)
+
+
+def test_shared_blocks_equal_unshared_copies(pa):
+    """Sequences reading a shared prefix give bit-identical outputs to the
+    same sequences reading private copies of it."""
+    w = small("shared_prefix_tails")
+    out_shared, _, _ = gpu_step(pa, w)
+    # give every sequence private copies of every block it shares
+    bt = w.block_tables.copy()
+    kp, vp = w.k_pool.clone(), w.v_pool.clone()
+    owner = {}
+    extra_k, extra_v = [], []
+    nxt = w.num_blocks
+    for s in range(w.num_seqs):
+        nb = -(-int(w.context_lens[s]) // w.block_size)
+        for j in range(nb):
+            b = int(bt[s, j])
+            if b in owner and owner[b] != s:
+                extra_k.append(kp[b].clone())
+                extra_v.append(vp[b].clone())
+                bt[s, j] = nxt
+                nxt += 1
+            else:
+                owner[b] = s
+    assert extra_k, "the workload shares blocks"
+    kp = torch.cat([kp, torch.stack(extra_k)])
+    vp = torch.cat([vp, torch.stack(extra_v)])
+    w2 = W.Workload(**{**w.__dict__, "k_pool": kp, "v_pool": vp, "block_tables": bt,
+                       "num_blocks": nxt})
+    # the step's new tokens live in private blocks already (no remap needed)
+    out_private, _, _ = gpu_step(pa, w2)
+    assert torch.equal(out_shared, out_private)
+
+
+def test_unused_table_entries_and_slots_are_never_read(pa):
+    w = small("llama70b_gqa_ragged")
+    out1, _, _ = gpu_step(pa, w)
+    bt = w.block_tables.copy()
+    # widen the table with garbage past every sequence's blocks
+    bt = np.concatenate([bt, np.full((bt.shape[0], 5), 10 ** 9, np.int32)], 1)
+    w2 = W.Workload(**{**w.__dict__, "block_tables": bt})
+    out2, _, _ = gpu_step(pa, w2)
+    assert torch.equal(out1, out2)
+
+
+@pytest.mark.parametrize("d,bs,cache", [(64, 16, "f16"), (128, 32, "bf16"), (64, 32, "e4m3"),
+                                         (128, 16, "e4m3")])
+def test_decode_edge_lengths(pa, d, bs, cache):
+    """Lengths 0, 1, bs-1, bs, bs+1, a multiple of bs, and a long one; one
+    token gives that token's value row exactly."""
+    lens = [0, 1, bs - 1, bs, bs + 1, 4 * bs, 777, 2]
+    hq, hkv = 8, 2
+    qd = "bf16" if cache != "f16" else "f16"
+    w = W._generic("edge", lens, hq, hkv, d, bs, qd, cache, seed=17, device="cpu")
+    out, kp, vp = gpu_step(pa, w, split_tokens=2 * bs)
+    ref, _, ovp = oracle_step(w)
+    assert_attention_close(as_f64(out), ref, "edge lengths")
+    o = as_f64(out)
+    assert not o[0].any()  # empty context
+    if cache != "e4m3":
+        # single token: the output is exactly the token's value row
+        v = oracle.decode_cache(ovp, cache)
+        slot = int(w.slot_mapping[1])
+        for h in range(hq):
+            assert np.array_equal(o[1, h], v[slot // bs, slot % bs, h // (hq // hkv)])
+
+
+def test_e4m3_every_code_decodes_exactly(pa):
+    """A one-token context returns v_scale * decode(code) for every one of the
+    256 codes (exact in bf16), NaN codes giving NaN."""
+    d, hkv, bs = 128, 2, 16
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(1, 1, hkv, d)
+    vp = torch.zeros(1, bs, hkv, d, dtype=torch.uint8)
+    vp[0, 0] = codes[0, 0]
+    kp = torch.zeros(1, bs, hkv, d, dtype=torch.uint8)
+    q = torch.randn(1, 4, d).to(torch.bfloat16)
+    out = pa.decode(q.cuda(), kp.view(torch.float8_e4m3fn).cuda(), vp.view(torch.float8_e4m3fn).cuda(),
+                    torch.zeros(1, 1, dtype=torch.int32, device="cuda"),
+                    torch.ones(1, dtype=torch.int32, device="cuda"), 0.1, 1, k_scale=1.0, v_scale=1.0)
+    pa.sync_status()
+    got = as_f64(out)[0]  # [4 heads, D]
+    want = oracle.e4m3_decode(codes.numpy().reshape(hkv, d))
+    for h in range(4):
+        np.testing.assert_array_equal(got[h], want[h // 2])
+
+
+# ------------------------------------------------------ device error word
+
+def test_out_of_range_indices_are_reported_not_faulted(pa):
+    w = small("tiny")
+    bt = w.block_tables.copy()
+    bt[0, 1] = w.num_blocks + 5  # read by sequence 0 (40 tokens, 3 blocks)
+    w2 = W.Workload(**{**w.__dict__, "block_tables": bt})
+    with pytest.raises(pa.PagedAttnError) as e:
+        gpu_step(pa, w2)
+    assert e.value.status == 8
+    pa.sync_status()  # the word was cleared
+    slots = w.slot_mapping.copy()
+    slots[2] = w.num_blocks * w.block_size + 3
+    with pytest.raises(pa.PagedAttnError):
+        gpu_step(pa, W.Workload(**{**w.__dict__, "slot_mapping": slots}))
+    lens = w.context_lens.copy()
+    lens[3] = w.max_context_len + 1  # above the stated maximum
+    kp, vp = w.k_pool.cuda(), w.v_pool.cuda()
+    with pytest.raises(pa.PagedAttnError):
+        pa.decode(w.q.cuda(), kp, vp, torch.from_numpy(w.block_tables).cuda(),
+                  torch.from_numpy(lens).cuda(), w.scale, w.max_context_len)
+        pa.sync_status()
+    with pytest.raises(pa.PagedAttnError):
+        pa.copy_blocks(kp, vp, torch.tensor([[0, 64]], dtype=torch.int64, device="cuda"))
+        pa.sync_status()
+    pa.sync_status()
+
+
+def test_validators_detect_bad_indices(pa):
+    s = pa._stream()
+    slots = torch.tensor([3, 9, -1, 3], dtype=torch.int64, device="cuda")
+    assert pa.pa_validate_slot_mapping(pa._ptr(slots), 4, 4, 16, s) == 6
+    slots = torch.tensor([3, 64], dtype=torch.int64, device="cuda")
+    assert pa.pa_validate_slot_mapping(pa._ptr(slots), 2, 4, 16, s) == 5
+    slots = torch.tensor([3, 63, -5], dtype=torch.int64, device="cuda")
+    assert pa.pa_validate_slot_mapping(pa._ptr(slots), 3, 4, 16, s) == 0
+    pairs = torch.tensor([[1, 2], [3, 2]], dtype=torch.int64, device="cuda")
+    assert pa.pa_validate_copy_pairs(pa._ptr(pairs), 2, 8, s) == 6
+    pairs = torch.tensor([[1, 2], [2, 3]], dtype=torch.int64, device="cuda")
+    assert pa.pa_validate_copy_pairs(pa._ptr(pairs), 2, 8, s) == 6
+    pairs = torch.tensor([[1, 2], [1, 3]], dtype=torch.int64, device="cuda")
+    assert pa.pa_validate_copy_pairs(pa._ptr(pairs), 2, 8, s) == 0
+    w = small("tiny")
+    bt = torch.from_numpy(w.block_tables).cuda()
+    cl = torch.from_numpy(w.context_lens).cuda()
+    assert pa.pa_validate_block_tables(pa._ptr(bt), bt.shape[1], pa._ptr(cl), 4, 63, 16, 64, s) == 0
+    bt[3, 2] = -1
+    assert pa.pa_validate_block_tables(pa._ptr(bt), bt.shape[1], pa._ptr(cl), 4, 63, 16, 64, s) == 5
+
+
+# ---------------------------------------------- benchmark sizes, sampled
+
+def test_benchmark_workload_sampled_against_oracle(pa):
+    """The Llama-3-70B-shaped layer at full size (256 x 4096 tokens, bf16)
+    in the launch configuration the benchmark times; 12 sequences checked."""
+    w = W.make("llama70b_gqa", device="cuda")
+    out, _, _ = gpu_step(pa, w)
+    seqs = [0, 1, 37, 100, 128, 129, 200, 254, 255, 64, 65, 3]
+    ref = compact_oracle_step(w, seqs)
+    assert_attention_close(as_f64(out)[seqs], ref, "llama70b_gqa full size")
+    assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("name", ["fp8_longtail_bs16", "fp8_longtail_bs32", "llama13b_mha"])
+def test_full_size_workloads_against_oracle(pa, name):
+    w = W.make(name, device="cuda")
+    out, _, _ = gpu_step(pa, w)
+    rng = np.random.default_rng(0)
+    seqs = sorted(set(rng.choice(w.num_seqs, size=16, replace=False).tolist()) |
+                  {int(np.argmax(w.context_lens))})
+    ref = compact_oracle_step(w, seqs)
+    assert_attention_close(as_f64(out)[seqs], ref, f"{name} full size")
