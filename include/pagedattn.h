@@ -210,6 +210,45 @@ pa_status pa_validate_block_tables(const int32_t* block_tables, int32_t max_bloc
                                    int32_t max_context_len, int32_t block_size,
                                    int32_t num_blocks, pa_stream_t stream);
 
+/*
+ * pa_decode_noalloc -- pa_decode for callers that cannot allocate device
+ * memory.  (The pages have no counterpart to this call; it exists for
+ * library users.)
+ *
+ * Some callers may not call cudaMalloc at all: a kernel plugin inside a host
+ * framework that owns every device allocation and hands the plugin only its
+ * inputs and outputs, or a serving loop whose memory is budgeted up front and
+ * where an allocation call could block until the device is idle.  Such a
+ * caller still passes q, the pools, the tables and `out`, but no workspace:
+ * this entry point takes pa_decode's scratch (work counter, range offsets,
+ * split partials) from one array of PA_DECODE_NOALLOC_SCRATCH_BYTES bytes
+ * that the library reserves in device memory; every GPU that loads the
+ * library holds that array until the process exits.
+ *
+ * Arguments and results are exactly those of pa_decode without `workspace`
+ * and `workspace_bytes`.  A call whose scratch need
+ * (pa_decode_workspace_size of the same sizes) exceeds
+ * PA_DECODE_NOALLOC_SCRATCH_BYTES is refused with PA_ERR_WORKSPACE before any
+ * launch; a larger split_tokens (fewer context ranges) lowers the need.
+ * The first call on a device looks up the array's device address with
+ * cudaGetSymbolAddress (once per device, with that device current); make
+ * that first call before any stream capture begins.  The call allocates
+ * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ * Every call shares the one array and finds the previous call's contents in
+ * it; the work counter that must start at zero is cleared by the call's own
+ * first kernel.  Calls that overlap on the GPU (other streams, other host
+ * threads) race on the array: order them on one stream.
+ */
+#define PA_DECODE_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+pa_status pa_decode_noalloc(void* out, const void* q, pa_dtype q_dtype,
+                            const void* k_pool, const void* v_pool, pa_dtype cache_dtype,
+                            const int32_t* block_tables, int32_t max_blocks_per_seq,
+                            const int32_t* context_lens, int32_t max_context_len,
+                            int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                            int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                            float scale, float k_scale, float v_scale,
+                            int32_t split_tokens, pa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

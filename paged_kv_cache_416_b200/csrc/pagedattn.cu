@@ -1,5 +1,6 @@
 // Host side of libpagedattn.so: argument validation, kernel selection,
 // workspace layout and the C entry points declared in include/pagedattn.h.
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -428,3 +429,53 @@ pa_status pa_validate_block_tables(const int32_t* block_tables, int32_t max_bloc
 }
 
 }  // extern "C"
+
+// ------------------------------------------------- decode without a workspace
+// Scratch for pa_decode_noalloc: reserved in device memory when the library
+// is loaded (on every GPU that loads it, until the process exits).  Host code
+// must not use this name as a device address: it is a host-side stand-in;
+// the device address comes from cudaGetSymbolAddress below.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[PA_DECODE_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+// Device address of g_noalloc_scratch, looked up once per device.
+std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+
+pa_status noalloc_scratch(int dev, void** ptr) {
+  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
+  if (p == nullptr) {
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return cuda_fail(e, "pa_decode_noalloc: cudaGetSymbolAddress of the built-in scratch");
+    g_noalloc_ptr[dev].store(p, std::memory_order_release);
+  }
+  *ptr = p;
+  return PA_OK;
+}
+}  // namespace
+
+extern "C" pa_status pa_decode_noalloc(
+    void* out, const void* q, pa_dtype q_dtype, const void* k_pool, const void* v_pool,
+    pa_dtype cache_dtype, const int32_t* block_tables, int32_t max_blocks_per_seq,
+    const int32_t* context_lens, int32_t max_context_len, int32_t num_seqs, int32_t num_q_heads,
+    int32_t num_kv_heads, int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
+    float k_scale, float v_scale, int32_t split_tokens, pa_stream_t stream) {
+  const size_t need = pa_decode_workspace_size(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                               block_size, max_context_len, split_tokens);
+  if (need > PA_DECODE_NOALLOC_SCRATCH_BYTES)
+    return fail(PA_ERR_WORKSPACE,
+                "pa_decode_noalloc: these sizes need %zu bytes of scratch but the built-in scratch "
+                "holds %u; pass a larger split_tokens or call pa_decode with your own workspace",
+                need, PA_DECODE_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  if (num_seqs > 0 && need > 0) {  // invalid sizes fall through to pa_decode's checks
+    int dev;
+    if (current_device(&dev)) return fail(PA_ERR_CUDA, "pa_decode_noalloc: no current device");
+    const pa_status s = noalloc_scratch(dev, &scratch);
+    if (s != PA_OK) return s;
+  }
+  return pa_decode(out, q, q_dtype, k_pool, v_pool, cache_dtype, block_tables,
+                   max_blocks_per_seq, context_lens, max_context_len, num_seqs, num_q_heads,
+                   num_kv_heads, head_dim, block_size, num_blocks, scale, k_scale, v_scale,
+                   split_tokens, scratch, PA_DECODE_NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -58,6 +58,8 @@ def _load() -> ctypes.CDLL:
         "pa_validate_slot_mapping": (I32, [P, I32, I32, I32, P]),
         "pa_validate_copy_pairs": (I32, [P, I32, I32, P]),
         "pa_validate_block_tables": (I32, [P, I32, P, I32, I32, I32, I32, P]),
+        "pa_decode_noalloc": (I32, [P, P, I32, P, P, I32, P, I32, P, I32, I32, I32, I32, I32, I32,
+                                    I32, F, F, F, I32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -79,11 +81,15 @@ pa_last_error = _lib.pa_last_error
 pa_validate_slot_mapping = _lib.pa_validate_slot_mapping
 pa_validate_copy_pairs = _lib.pa_validate_copy_pairs
 pa_validate_block_tables = _lib.pa_validate_block_tables
+# pa_decode for callers that cannot allocate device memory: the scratch comes
+# from an array the library reserves when it is loaded (see the header)
+pa_decode_noalloc = _lib.pa_decode_noalloc
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 ENTRY_POINTS = [
     "pa_write_kv", "pa_copy_blocks", "pa_decode_split_tokens", "pa_decode_workspace_size",
     "pa_decode", "pa_sync_status", "pa_last_error", "pa_validate_slot_mapping",
-    "pa_validate_copy_pairs", "pa_validate_block_tables",
+    "pa_validate_copy_pairs", "pa_validate_block_tables", "pa_decode_noalloc",
 ]
 
 
