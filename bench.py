@@ -55,6 +55,8 @@ def parse_args(argv=None):
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--num-seqs", type=int, default=None,
+                    help="override the workload's batch (smaller cases for profiling only)")
     return ap.parse_args(argv)
 
 
@@ -281,7 +283,8 @@ def run_ours(args, rank, local, world):
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    w = W.make(args.workload, seed=args.seed + rank, device=device)
+    kw = {"num_seqs": args.num_seqs} if args.num_seqs else {}
+    w = W.make(args.workload, seed=args.seed + rank, device=device, **kw)
     stream = torch.cuda.current_stream()
     kp, vp = w.k_pool, w.v_pool
     q = w.q.contiguous()

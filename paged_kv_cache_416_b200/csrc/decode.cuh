@@ -13,9 +13,12 @@
 //   item  = (sequence, context range of split_tokens tokens, kv head)
 //   CTA   = 4 warps; a persistent grid pulls items from an atomic counter
 //   warp  = takes every 4th block of the item's range; each warp owns a ring
-//           of kStages shared-memory stages, one stage = the K and V rows of
-//           one block for one kv head, filled by 1-D bulk asynchronous copies
-//           (one per token row, completion counted on an mbarrier)
+//           of kStages shared-memory stages, one stage = the K tile and the V
+//           tile of one block for one kv head, each tile filled by ONE tiled
+//           TMA copy (cp.async.bulk.tensor through a tensor map over the
+//           pool, box = bs token rows of one head, 128B/64B swizzle so that
+//           ldmatrix is free of bank conflicts; completion counted in bytes
+//           on an mbarrier; no multicast)
 // Per block and warp, with the packed heads as the MMA's N = 8 columns:
 //   S^T[t, g] = K[t, :] . Q[g, :]        m16n8k16, A = K rows (ldmatrix)
 //   online softmax over t per column g   (exp2, running max and sum)
@@ -27,6 +30,8 @@
 // workspace and merge_kernel combines the ranges of a sequence.
 #pragma once
 
+#include <cuda.h>  // CUtensorMap
+
 #include "common.cuh"
 
 namespace pa {
@@ -37,18 +42,23 @@ constexpr int kDecodeWarps = 4;
 constexpr int kDecodeThreads = kDecodeWarps * 32;
 constexpr int kMaxGroup = 8;          // packed query heads per kv head (MMA N)
 constexpr int kBarrierBytes = 256;    // mbarrier area at the start of smem
+constexpr int kTileAlign = 1024;      // swizzled tiles start on this boundary
 
 template <int CK, int D, int BS>
 struct DecodeCfg {
+  static constexpr int kBS = BS;
   static constexpr int kElem = (CK == kCacheE4M3) ? 1 : 2;
-  static constexpr int kRowBytes = D * kElem;          // one token row of one head
-  static constexpr int kRowStride = kRowBytes + 16;    // padded: ldmatrix rows hit distinct banks
-  static constexpr int kStageBytes = 2 * BS * kRowStride;  // K rows then V rows
-  static constexpr int kBudget = 110 * 1024;           // per CTA: two CTAs fit one SM
+  static constexpr int kRowBytes = D * kElem;                    // one token row of one head
+  static constexpr int kSwzBytes = kRowBytes >= 128 ? 128 : 64;  // bytes per swizzle row
+  static constexpr int kHalves = kRowBytes / kSwzBytes;          // swizzle rows per token row
+  static constexpr int kSwzMask = kSwzBytes == 128 ? 7 : 3;      // 128B / 64B swizzle
+  static constexpr int kTileBytes = BS * kRowBytes;              // one tensor, one block
+  static constexpr int kStageBytes = 2 * kTileBytes;             // K tile then V tile
+  static constexpr int kBudget = 70 * 1024;                      // per CTA: three fit one SM
   static constexpr int kStagesRaw = kBudget / (kDecodeWarps * kStageBytes);
   static constexpr int kStages = kStagesRaw < 1 ? 1 : (kStagesRaw > 6 ? 6 : kStagesRaw);
   static constexpr int kWarpBytes = kStages * kStageBytes;
-  static constexpr int kSmemBytes = kBarrierBytes + kDecodeWarps * kWarpBytes;
+  static constexpr int kSmemBytes = kBarrierBytes + kTileAlign + kDecodeWarps * kWarpBytes;
   static constexpr int kTokTiles = BS / 16;
   static constexpr int kDimTiles = D / 16;
   static constexpr bool kMmaBF16 = (CK == kCacheBF16);
@@ -56,14 +66,46 @@ struct DecodeCfg {
   static constexpr int kScratchBytes = (kMaxGroup * D + 2 * kMaxGroup) * 4;
   static_assert(kWarpBytes >= kScratchBytes, "warp ring too small for the merge scratch");
   static_assert(kDecodeWarps * kStages <= kBarrierBytes / 8, "too many mbarriers");
-  static_assert(kRowBytes % 16 == 0, "bulk copies move 16-byte multiples");
+  static_assert(kRowBytes == 64 || kRowBytes % 128 == 0, "unsupported row size");
+  static_assert(kTileBytes % (8 * kSwzBytes) == 0, "tiles must hold whole swizzle atoms");
+  static_assert(kWarpBytes % kTileAlign == 0 || kDecodeWarps == 1, "rings keep tiles aligned");
 };
 
+// Byte offset of (token row t, byte b of the row) inside a swizzled tile.
+// The tile holds kHalves groups of BS rows of kSwzBytes bytes; the TMA
+// swizzle XORs the 16-byte chunk index with address bits 7.. (mask 7 for
+// 128B, 3 for 64B), which the tile's kTileAlign alignment makes equal to the
+// offset's bits.
+template <class C>
+__device__ __forceinline__ uint32_t tile_off(int t, int b) {
+  const int row = (b / C::kSwzBytes) * C::kBS + t;
+  const uint32_t o = static_cast<uint32_t>(row * C::kSwzBytes);
+  const uint32_t chunk = static_cast<uint32_t>((b % C::kSwzBytes) >> 4);
+  return o + ((chunk ^ ((o >> 7) & C::kSwzMask)) << 4);
+}
+
+// Tiled TMA load of a 5-D box: tensor map coordinates (x innermost).
+__device__ __forceinline__ void tma_load_5d(uint32_t dst, const CUtensorMap* map, int c0, int c1,
+                                            int c2, int c3, int c4, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
+      ::"r"(dst), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3),
+        "r"(c4), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
 struct DecodeArgs {
+  // Tensor maps over the pools, viewed as 5-D bytes (x, token, half, kv head,
+  // block) = (kSwzBytes, bs, kHalves, Hkv, N); box (kSwzBytes, bs, kHalves, 1, 1).
+  CUtensorMap tmap_k;
+  CUtensorMap tmap_v;
   void* out;
   const void* q;
-  const uint8_t* k_pool;
-  const uint8_t* v_pool;
   const int32_t* block_tables;
   const int32_t* context_lens;
   int32_t* counter;        // workspace: work-queue counter (zeroed by plan_kernel)
@@ -133,10 +175,16 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
   }
 }
 
+// Keep the halves of a 32-bit fragment register whose token is valid:
+// low half <- token t, high half <- token t + 1.
+__device__ __forceinline__ uint32_t pair_mask(bool lo_ok, bool hi_ok) {
+  return (lo_ok ? 0x0000ffffu : 0u) | (hi_ok ? 0xffff0000u : 0u);
+}
+
 // ------------------------------------------------------------ main kernel
 template <int CK, bool kQBF16, int D, int BS>
 __global__ void __launch_bounds__(kDecodeThreads)
-decode_kernel(const DecodeArgs a) {
+decode_kernel(const __grid_constant__ DecodeArgs a) {
   using C = DecodeCfg<CK, D, BS>;
   constexpr bool kMmaBF16 = C::kMmaBF16;
   constexpr int kStages = C::kStages;
@@ -148,19 +196,28 @@ decode_kernel(const DecodeArgs a) {
   const int g = lane >> 2;    // fragment row group
   const int tig = lane & 3;   // thread in group
 
-  uint8_t* const wbase = smem + kBarrierBytes + warp * C::kWarpBytes;
-  const uint32_t wbase_s = smem_addr(wbase);
-  const uint32_t bar0 = smem_addr(smem) + warp * kStages * 8;
+  // stage rings start on a kTileAlign boundary after the mbarriers
+  const uint32_t smem_s = smem_addr(smem);
+  const uint32_t ring_s = (smem_s + kBarrierBytes + kTileAlign - 1) & ~uint32_t(kTileAlign - 1);
+  const uint32_t wbase_s = ring_s + warp * C::kWarpBytes;
+  uint8_t* const ring = smem + (ring_s - smem_s);
+  uint8_t* const wbase = ring + warp * C::kWarpBytes;
+  const uint32_t bar0 = smem_s + warp * kStages * 8;
   if (lane == 0) {
 #pragma unroll
     for (int s = 0; s < kStages; ++s) mbar_init(bar0 + 8 * s, 1);
     mbar_init_fence();
+  }
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&a.tmap_k);
+    prefetch_tensormap(&a.tmap_v);
   }
   __syncthreads();
 
   const int total = *a.total;
   const bool split_mode = a.split_tokens < a.max_ctx;
   uint32_t n_issued = 0, n_consumed = 0;  // warp-uniform ring counters
+  uint32_t skip_stage = 0;                // stages holding a block with a bad table entry
   bool failed = false;                    // a wait timed out: stop issuing / computing
 
   for (;;) {
@@ -197,38 +254,44 @@ decode_kernel(const DecodeArgs a) {
     const int32_t* table = a.block_tables + static_cast<int64_t>(seq) * a.max_blocks;
     const int h0 = kvh * a.group;
 
-    // ---- issue the loads of the warp's i-th block of this item
+    // ---- block-table entries of the warp's blocks, prefetched in registers:
+    // lane l holds the entry of the warp's block (32 * chunk + l); tab_cur is
+    // the chunk the issue cursor is in, tab_nxt the one after it, so the
+    // table read never sits on the path from one block to the next
+    auto load_chunk = [&](int c) -> int {
+      const int i = c * 32 + lane;
+      return i < nb_w ? table[jb0 + warp + i * kDecodeWarps] : -1;
+    };
+    int tab_chunk = 0;
+    int tab_cur = load_chunk(0);
+    int tab_nxt = load_chunk(1);
+
+    // ---- issue the two tile loads of the warp's i-th block of this item
+    // (i increases by at most one chunk between calls)
     auto issue = [&](int i) {
-      const int j = jb0 + warp + i * kDecodeWarps;
       const int st = n_issued % kStages;
       const uint32_t bar = bar0 + 8 * st;
       const uint32_t sK = wbase_s + st * C::kStageBytes;
-      uint8_t* const gK = wbase + st * C::kStageBytes;
-      const int phys = table[j];
+      if ((i >> 5) != tab_chunk) {
+        tab_chunk = i >> 5;
+        tab_cur = tab_nxt;
+        tab_nxt = load_chunk(tab_chunk + 1);
+      }
+      const int phys = __shfl_sync(0xffffffffu, tab_cur, i & 31);
       const bool ok = phys >= 0 && phys < a.num_blocks;
-      if (!ok && lane == 0) record_error(PA_ERR_DEVICE_BOUNDS);
-      const int nv = ok ? min(BS, t1 - j * BS) : 0;  // valid token rows
-      fence_proxy_async_smem();  // earlier generic reads/writes of this stage first
+      skip_stage = ok ? (skip_stage & ~(1u << st)) : (skip_stage | (1u << st));
+      fence_proxy_async_smem();  // this lane's earlier generic accesses of the stage first
       __syncwarp();
-      if (lane == 0) mbar_arrive_expect_tx(bar, 2u * nv * C::kRowBytes);
-      __syncwarp();
-      const int64_t row0 = (static_cast<int64_t>(ok ? phys : 0) * BS * a.hkv + kvh);
-#pragma unroll
-      for (int rr = lane; rr < 2 * BS; rr += 32) {
-        const bool isv = rr >= BS;
-        const int tok = isv ? rr - BS : rr;
-        const uint32_t dst = sK + rr * C::kRowStride;
-        if (tok < nv) {
-          const uint8_t* src = (isv ? a.v_pool : a.k_pool) +
-                               (row0 + static_cast<int64_t>(tok) * a.hkv) * C::kRowBytes;
-          bulk_copy_g2s(dst, src, C::kRowBytes, bar);
-        } else {  // rows past the sequence: zeros, so masked tokens add 0 * 0
-          uint4* z = reinterpret_cast<uint4*>(gK + rr * C::kRowStride);
-#pragma unroll
-          for (int c = 0; c < C::kRowBytes / 16; ++c) z[c] = make_uint4(0, 0, 0, 0);
+      if (lane == 0) {
+        if (ok) {
+          mbar_arrive_expect_tx(bar, 2u * C::kTileBytes);
+          tma_load_5d(sK, &a.tmap_k, 0, 0, 0, kvh, phys, bar);
+          tma_load_5d(sK + C::kTileBytes, &a.tmap_v, 0, 0, 0, kvh, phys, bar);
+        } else {
+          record_error(PA_ERR_DEVICE_BOUNDS);  // the block's tokens are left out
+          mbar_arrive_expect_tx(bar, 0u);
         }
       }
-      __syncwarp();
       ++n_issued;
     };
 
@@ -267,6 +330,7 @@ decode_kernel(const DecodeArgs a) {
       for (int i = 0; i < pro; ++i) issue(i);
     }
 
+    const int li = lane >> 3;  // which 8x8 matrix of an ldmatrix.x4 this lane addresses
     for (int i = 0; i < nb_w; ++i) {
       const int st = n_consumed % kStages;
       const uint32_t par = (n_consumed / kStages) & 1u;
@@ -277,46 +341,54 @@ decode_kernel(const DecodeArgs a) {
           if (lane == 0) record_error(PA_ERR_TIMEOUT);
         }
       }
-      if (!failed) {
+      if (!failed && !((skip_stage >> st) & 1u)) {
         const int j = jb0 + warp + i * kDecodeWarps;
         const int tbase = j * BS;
+        const bool partial = tbase + BS > t1;  // rows past the range hold other data
         const uint32_t sK = wbase_s + st * C::kStageBytes;
-        const uint32_t sV = sK + BS * C::kRowStride;
+        const uint32_t sV = sK + C::kTileBytes;
 
         // ---- S^T = K Q^T  (rows: tokens, cols: packed heads)
         float s[C::kTokTiles][4];
 #pragma unroll
         for (int mt = 0; mt < C::kTokTiles; ++mt) {
           float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+          float s2[4] = {0.f, 0.f, 0.f, 0.f}, s3[4] = {0.f, 0.f, 0.f, 0.f};
           if constexpr (CK == kCacheE4M3) {
-            const int li = lane >> 3;
             const int tok = mt * 16 + (lane & 7) + (li & 1) * 8;
 #pragma unroll
             for (int cp = 0; cp < C::kDimTiles / 2; ++cp) {
               uint32_t r0, r1, r2, r3;
-              ldsm_x4(sK + tok * C::kRowStride + (2 * cp + (li >> 1)) * 16, r0, r1, r2, r3);
+              ldsm_x4(sK + tile_off<C>(tok, (2 * cp + (li >> 1)) * 16), r0, r1, r2, r3);
               const uint32_t a0[4] = {e4m3x2_to_f16x2(r0 & 0xffff), e4m3x2_to_f16x2(r1 & 0xffff),
                                       e4m3x2_to_f16x2(r0 >> 16), e4m3x2_to_f16x2(r1 >> 16)};
               const uint32_t a1[4] = {e4m3x2_to_f16x2(r2 & 0xffff), e4m3x2_to_f16x2(r3 & 0xffff),
                                       e4m3x2_to_f16x2(r2 >> 16), e4m3x2_to_f16x2(r3 >> 16)};
-              mma_16816<false>(s0, a0, qf[2 * cp][0], qf[2 * cp][1]);
-              mma_16816<false>(s1, a1, qf[2 * cp + 1][0], qf[2 * cp + 1][1]);
+              if (cp & 1) {
+                mma_16816<false>(s2, a0, qf[2 * cp][0], qf[2 * cp][1]);
+                mma_16816<false>(s3, a1, qf[2 * cp + 1][0], qf[2 * cp + 1][1]);
+              } else {
+                mma_16816<false>(s0, a0, qf[2 * cp][0], qf[2 * cp][1]);
+                mma_16816<false>(s1, a1, qf[2 * cp + 1][0], qf[2 * cp + 1][1]);
+              }
             }
           } else {
-            const int row = mt * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
-            const uint32_t base = sK + row * C::kRowStride + (lane >> 4) * 16;
+            const int row = mt * 16 + (lane & 7) + (li & 1) * 8;
 #pragma unroll
             for (int ks = 0; ks < C::kDimTiles; ++ks) {
               uint32_t af[4];
-              ldsm_x4(base + ks * 32, af[0], af[1], af[2], af[3]);
-              if (ks & 1) mma_16816<kMmaBF16>(s1, af, qf[ks][0], qf[ks][1]);
-              else mma_16816<kMmaBF16>(s0, af, qf[ks][0], qf[ks][1]);
+              ldsm_x4(sK + tile_off<C>(row, (ks * 16 + (li >> 1) * 8) * 2), af[0], af[1], af[2],
+                      af[3]);
+              if ((ks & 3) == 0) mma_16816<kMmaBF16>(s0, af, qf[ks][0], qf[ks][1]);
+              else if ((ks & 3) == 1) mma_16816<kMmaBF16>(s1, af, qf[ks][0], qf[ks][1]);
+              else if ((ks & 3) == 2) mma_16816<kMmaBF16>(s2, af, qf[ks][0], qf[ks][1]);
+              else mma_16816<kMmaBF16>(s3, af, qf[ks][0], qf[ks][1]);
             }
           }
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int tok = tbase + mt * 16 + g + (e >> 1) * 8;
-            const float x = (s0[e] + s1[e]) * a.sl2;
+            const float x = ((s0[e] + s1[e]) + (s2[e] + s3[e])) * a.sl2;
             s[mt][e] = tok < t1 ? x : -INFINITY;
           }
         }
@@ -358,16 +430,24 @@ decode_kernel(const DecodeArgs a) {
           pb[mt][1] = movmatrix_trans(pack2<kPBF16>(s[mt][2], s[mt][3]));
         }
 
-        // ---- O^T += V^T P^T  (rows: dims, cols: packed heads)
-        if constexpr (CK == kCacheE4M3) {
-          const int li = lane >> 3;
+        // ---- O^T += V^T P^T  (rows: dims, cols: packed heads).  In a partial
+        // block the V rows past the range are zeroed in the fragments (their
+        // P is 0, but the rows may hold anything, NaN included).
 #pragma unroll
-          for (int mt = 0; mt < C::kTokTiles; ++mt) {
+        for (int mt = 0; mt < C::kTokTiles; ++mt) {
+          uint32_t m_lo = 0xffffffffu, m_hi = 0xffffffffu;  // tokens 2tig(+1), 2tig+8(+9)
+          if (partial) {
+            const int tk = tbase + mt * 16 + 2 * tig;
+            m_lo = pair_mask(tk < t1, tk + 1 < t1);
+            m_hi = pair_mask(tk + 8 < t1, tk + 9 < t1);
+          }
+          if constexpr (CK == kCacheE4M3) {
             const int tok = mt * 16 + (lane & 7) + (li & 1) * 8;
 #pragma unroll
             for (int cp = 0; cp < C::kDimTiles / 2; ++cp) {
               uint32_t r0, r1, r2, r3;
-              ldsm_x4_trans(sV + tok * C::kRowStride + (2 * cp + (li >> 1)) * 16, r0, r1, r2, r3);
+              ldsm_x4_trans(sV + tile_off<C>(tok, (2 * cp + (li >> 1)) * 16), r0, r1, r2, r3);
+              r0 &= m_lo; r1 &= m_hi; r2 &= m_lo; r3 &= m_hi;
               // bytes (tok 2tig: dim 2g, 2g+1 | tok 2tig+1: dim 2g, 2g+1) -> pairs per dim
               const uint32_t p0 = __byte_perm(r0, 0, 0x3120), p1 = __byte_perm(r1, 0, 0x3120);
               const uint32_t p2 = __byte_perm(r2, 0, 0x3120), p3 = __byte_perm(r3, 0, 0x3120);
@@ -378,17 +458,14 @@ decode_kernel(const DecodeArgs a) {
               mma_16816<false>(acc[2 * cp], a0, pb[mt][0], pb[mt][1]);
               mma_16816<false>(acc[2 * cp + 1], a1, pb[mt][0], pb[mt][1]);
             }
-          }
-        } else {
-          const int li = lane >> 3;
-#pragma unroll
-          for (int mt = 0; mt < C::kTokTiles; ++mt) {
+          } else {
             const int tok = mt * 16 + (lane & 7) + (li >> 1) * 8;
-            const uint32_t base = sV + tok * C::kRowStride + (li & 1) * 16;
 #pragma unroll
             for (int dt = 0; dt < C::kDimTiles; ++dt) {
               uint32_t af[4];
-              ldsm_x4_trans(base + dt * 32, af[0], af[1], af[2], af[3]);
+              ldsm_x4_trans(sV + tile_off<C>(tok, (dt * 16 + (li & 1) * 8) * 2), af[0], af[1],
+                            af[2], af[3]);
+              af[0] &= m_lo; af[1] &= m_lo; af[2] &= m_hi; af[3] &= m_hi;
               mma_16816<kMmaBF16>(acc[dt], af, pb[mt][0], pb[mt][1]);
             }
           }
@@ -434,7 +511,7 @@ decode_kernel(const DecodeArgs a) {
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kDecodeWarps; ++w) {
-          const float* scr = reinterpret_cast<const float*>(smem + kBarrierBytes + w * C::kWarpBytes);
+          const float* scr = reinterpret_cast<const float*>(ring + w * C::kWarpBytes);
           mw[w] = scr[kMaxGroup * D + h];
           M = fmaxf(M, mw[w]);
         }
@@ -445,7 +522,7 @@ decode_kernel(const DecodeArgs a) {
         if (M != -INFINITY) {
 #pragma unroll
           for (int w = 0; w < kDecodeWarps; ++w) {
-            const float* scr = reinterpret_cast<const float*>(smem + kBarrierBytes + w * C::kWarpBytes);
+            const float* scr = reinterpret_cast<const float*>(ring + w * C::kWarpBytes);
             const float f = fast_exp2(mw[w] - M);
             L += f * scr[kMaxGroup * D + kMaxGroup + h];
             const float4 x0 = *reinterpret_cast<const float4*>(scr + h * D + d0);
@@ -474,7 +551,8 @@ decode_kernel(const DecodeArgs a) {
         }
       }
     }
-    __syncthreads();  // scratch (= stage memory) is free again
+    __syncthreads();           // scratch (= stage memory) is free again ...
+    fence_proxy_async_smem();  // ... and the next item's tile loads come after these accesses
   }
 
   // drain copies still in flight after a timeout (bounded again)

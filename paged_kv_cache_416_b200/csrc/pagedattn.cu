@@ -1,5 +1,6 @@
 // Host side of libpagedattn.so: argument validation, kernel selection,
 // workspace layout and the C entry points declared in include/pagedattn.h.
+#include <cuda.h>
 #include <atomic>
 #include <cmath>
 #include <cstdarg>
@@ -102,6 +103,56 @@ WsLayout ws_layout(int32_t B, int32_t hq, int32_t D, int32_t max_ctx, int32_t S)
   w.o = w.lse + static_cast<size_t>(round_up(ranges * hq * 4, 256));
   w.bytes = w.o + static_cast<size_t>(ranges * hq * D * 4);
   return w;
+}
+
+// --------------------------------------------------------- tensor maps
+// cuTensorMapEncodeTiled is a driver entry point; it is fetched through the
+// runtime so the library needs no link-time dependency on libcuda.
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled_fn() {
+  static std::atomic<EncodeTiledFn> fn{nullptr};
+  EncodeTiledFn f = fn.load(std::memory_order_acquire);
+  if (f == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess && p != nullptr) {
+      f = reinterpret_cast<EncodeTiledFn>(p);
+      fn.store(f, std::memory_order_release);
+    }
+  }
+  return f;
+}
+
+// Tensor map over a pool [N, bs, Hkv, D] viewed as 5-D bytes
+// (x, token, half, kv head, block) = (R, bs, D*e/R, Hkv, N) with R = min(128,
+// D*e) bytes per swizzle row; one box = the bs token rows of one kv head of
+// one block, landing in shared memory as [half][token][R] with the R-byte
+// swizzle (128B or 64B).  Must match DecodeCfg / tile_off in decode.cuh.
+pa_status encode_pool_map(CUtensorMap* map, const void* pool, int32_t num_blocks, int32_t bs,
+                          int32_t hkv, int32_t head_dim, int32_t elem) {
+  EncodeTiledFn fn = encode_tiled_fn();
+  if (fn == nullptr) return fail(PA_ERR_CUDA, "pa_decode: cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t row = static_cast<cuuint64_t>(head_dim) * elem;
+  const cuuint64_t R = row >= 128 ? 128 : 64;
+  const cuuint64_t halves = row / R;
+  const cuuint64_t dims[5] = {R, static_cast<cuuint64_t>(bs), halves, static_cast<cuuint64_t>(hkv),
+                              static_cast<cuuint64_t>(num_blocks)};
+  const cuuint64_t strides[4] = {hkv * row, R, row, static_cast<cuuint64_t>(bs) * hkv * row};
+  const cuuint32_t box[5] = {static_cast<cuuint32_t>(R), static_cast<cuuint32_t>(bs),
+                             static_cast<cuuint32_t>(halves), 1, 1};
+  const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void*>(pool), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        R == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(PA_ERR_CUDA, "pa_decode: cuTensorMapEncodeTiled failed (%d) for the pool", (int)r);
+  return PA_OK;
 }
 
 // ------------------------------------------------------ decode dispatch
@@ -279,11 +330,17 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_po
   auto st = reinterpret_cast<cudaStream_t>(stream);
   auto* ws = static_cast<uint8_t*>(workspace);
 
+  if ((reinterpret_cast<uintptr_t>(k_pool) | reinterpret_cast<uintptr_t>(v_pool)) & 15)
+    return fail(PA_ERR_SHAPE, "pa_decode: the pools must be 16-byte aligned");
   pa::DecodeArgs a;
+  pa_status ms = encode_pool_map(&a.tmap_k, k_pool, num_blocks, block_size, num_kv_heads,
+                                 head_dim, elem_bytes(cache_dtype));
+  if (ms == PA_OK)
+    ms = encode_pool_map(&a.tmap_v, v_pool, num_blocks, block_size, num_kv_heads, head_dim,
+                         elem_bytes(cache_dtype));
+  if (ms != PA_OK) return ms;
   a.out = out;
   a.q = q;
-  a.k_pool = static_cast<const uint8_t*>(k_pool);
-  a.v_pool = static_cast<const uint8_t*>(v_pool);
   a.block_tables = block_tables;
   a.context_lens = context_lens;
   a.counter = reinterpret_cast<int32_t*>(ws + w.counter);

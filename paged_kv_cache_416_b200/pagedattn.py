@@ -39,12 +39,8 @@ class PagedAttnError(RuntimeError):
         self.status = status
 
 
-def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
-        raise ImportError(
-            f"{LIB_PATH} is missing; build it with `python -m paged_kv_cache_416_b200.build` "
-            "(there is no CPU fallback)")
-    lib = ctypes.CDLL(LIB_PATH)
+def declare(lib: ctypes.CDLL) -> ctypes.CDLL:
+    """Set the ctypes signatures of the C entry points on a loaded library."""
     P, I32, I64, F, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
     sig = {
         "pa_write_kv": (I32, [P, P, I32, P, I32, P, P, I32, I32, I32, I32, I32, F, F, P]),
@@ -66,6 +62,14 @@ def _load() -> ctypes.CDLL:
         fn.restype = res
         fn.argtypes = args
     return lib
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing; build it with `python -m paged_kv_cache_416_b200.build` "
+            "(there is no CPU fallback)")
+    return declare(ctypes.CDLL(LIB_PATH))
 
 
 _lib = _load()
