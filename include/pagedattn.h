@@ -120,9 +120,11 @@ pa_status pa_copy_blocks(void* k_pool, void* v_pool, pa_dtype cache_dtype,
 
 /*
  * pa_decode_split_tokens -- the context-split length pa_decode uses for these
- * sizes when split_tokens == 0 (always a multiple of block_size).  A value >=
- * max_context_len means every (sequence, kv head) is one work item and no
- * merge pass runs.  Returns 0 on invalid arguments.
+ * sizes: the automatic choice when split_tokens == 0, else split_tokens
+ * rounded up to a multiple of block_size and raised, if needed, so that no
+ * sequence has more than 1024 ranges.  A value >= max_context_len means every
+ * (sequence, kv head) is one work item and nothing is merged.  Returns 0 on
+ * invalid arguments.
  */
 int32_t pa_decode_split_tokens(int32_t num_seqs, int32_t num_kv_heads,
                                int32_t block_size, int32_t max_context_len,

@@ -27,7 +27,8 @@
 //                                         registers with movmatrix)
 // The warps' partial (max, sum, O) are merged through shared memory at the
 // end of an item; a split item writes (log-sum-exp, O / sum) to the
-// workspace and merge_kernel combines the ranges of a sequence.
+// workspace, and the CTA that finishes the last range of a (sequence, kv
+// head) combines them (log-sum-exp merge) and writes the output.
 #pragma once
 
 #include <cuda.h>  // CUtensorMap
@@ -43,6 +44,7 @@ constexpr int kDecodeThreads = kDecodeWarps * 32;
 constexpr int kMaxGroup = 8;          // packed query heads per kv head (MMA N)
 constexpr int kBarrierBytes = 256;    // mbarrier area at the start of smem
 constexpr int kTileAlign = 1024;      // swizzled tiles start on this boundary
+constexpr int kMaxRanges = 1024;      // context ranges per sequence (fused merge uses smem)
 
 template <int CK, int D, int BS>
 struct DecodeCfg {
@@ -69,6 +71,8 @@ struct DecodeCfg {
   static_assert(kRowBytes == 64 || kRowBytes % 128 == 0, "unsupported row size");
   static_assert(kTileBytes % (8 * kSwzBytes) == 0, "tiles must hold whole swizzle atoms");
   static_assert(kWarpBytes % kTileAlign == 0 || kDecodeWarps == 1, "rings keep tiles aligned");
+  static_assert(kDecodeWarps * kWarpBytes >= (kMaxRanges + 1) * kMaxGroup * 4,
+                "the rings must hold the fused merge's weights");
 };
 
 // Byte offset of (token row t, byte b of the row) inside a swizzled tile.
@@ -111,6 +115,9 @@ struct DecodeArgs {
   int32_t* counter;        // workspace: work-queue counter (zeroed by plan_kernel)
   const int32_t* total;    // workspace: number of items (written by plan_kernel)
   const int32_t* seq_off;  // workspace: [B + 1] first range index of each sequence
+  const int4* order;       // workspace: [ranges] (sequence, range, end token, ranges of
+                           // the sequence), longest range first
+  int32_t* arrived;        // workspace: [B * Hkv] ranges finished per (sequence, kv head)
   float* lse_part;         // workspace: [ranges * Hq]
   float* o_part;           // workspace: [ranges * Hq * D]
   int num_seqs, hq, hkv, group, max_blocks, num_blocks, max_ctx, split_tokens;
@@ -119,31 +126,57 @@ struct DecodeArgs {
 };
 
 // ---------------------------------------------------------------- planning
-// One CTA: validates context lengths, counts each sequence's ranges
-// (max(1, ceil(len / split_tokens))), writes their exclusive prefix sum,
-// the item total (ranges * Hkv) and zeroes the work counter.
+constexpr int kPlanBuckets = 256;  // range-length classes of the longest-first order
+
+// One CTA of 1024 threads, once per decode call:
+//  1. validates the context lengths (an out-of-range length counts as 0 and
+//     is reported), counts each sequence's ranges max(1, ceil(len / S)) and
+//     writes their exclusive prefix sum seq_off (where a sequence's partials
+//     go) and the item total (ranges * Hkv); zeroes the work counter;
+//  2. writes the work order: every (sequence, range) pair with the range's
+//     end token and the sequence's range count, longest range first
+//     (counting sort over kPlanBuckets length classes), so that the
+//     short ranges fill the end of the persistent grid's queue.  The order
+//     inside a class is whatever the atomics give: outputs do not depend on
+//     it, because every item writes its own output or partial slot.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ ctx_lens, int B,
                                                     int max_ctx, int max_blocks, int bs, int S,
                                                     int hkv, int32_t* counter, int32_t* total,
-                                                    int32_t* seq_off) {
+                                                    int32_t* seq_off, int4* order,
+                                                    int32_t* arrived) {
   __shared__ int warp_tot[32];
   __shared__ int carry;
+  __shared__ int hist[kPlanBuckets];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int max_nb = (min(S, max_ctx) + bs - 1) / bs;  // blocks of the longest range
+  auto bucket = [&](int nb) {  // longer ranges -> higher class
+    return max_nb < kPlanBuckets ? nb : static_cast<int>((static_cast<int64_t>(nb) * (kPlanBuckets - 1)) / max_nb);
+  };
+  auto valid_len = [&](int s) {
+    const int c = ctx_lens[s];
+    return (c < 0 || c > max_ctx || c > max_blocks * bs) ? -1 : c;
+  };
   if (tid == 0) {
     carry = 0;
     *counter = 0;
   }
+  if (tid < kPlanBuckets) hist[tid] = 0;
+  if (arrived != nullptr)
+    for (int i = tid; i < B * hkv; i += 1024) arrived[i] = 0;
   __syncthreads();
   for (int base = 0; base < B; base += 1024) {
     const int s = base + tid;
     int n = 0;
     if (s < B) {
-      int c = ctx_lens[s];
-      if (c < 0 || c > max_ctx || c > max_blocks * bs) {
+      int c = valid_len(s);
+      if (c < 0) {
         record_error(PA_ERR_DEVICE_BOUNDS);
         c = 0;
       }
       n = c > 0 ? (c + S - 1) / S : 1;
+      const int last = c - (n - 1) * S;  // tokens of the last range (0 when c == 0)
+      if (n > 1) atomicAdd(&hist[bucket((S + bs - 1) / bs)], n - 1);
+      atomicAdd(&hist[bucket((last + bs - 1) / bs)], 1);
     }
     int x = n;  // inclusive warp scan
 #pragma unroll
@@ -173,6 +206,41 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
     seq_off[B] = carry;
     *total = carry * hkv;
   }
+  // class starts, longest class first: start[b] = sum of hist[b'] for b' > b
+  if (warp == 0) {
+    constexpr int kPer = kPlanBuckets / 32;
+    int v[kPer], sum = 0;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {  // lane owns classes from the top down
+      v[i] = hist[kPlanBuckets - 1 - (lane * kPer + i)];
+      sum += v[i];
+    }
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - sum;
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      hist[kPlanBuckets - 1 - (lane * kPer + i)] = run;  // becomes the class's cursor
+      run += v[i];
+    }
+  }
+  __syncthreads();
+  for (int s = tid; s < B; s += 1024) {
+    int c = valid_len(s);
+    if (c < 0) c = 0;
+    const int n = c > 0 ? (c + S - 1) / S : 1;
+    const int last = c - (n - 1) * S;
+    const int bf = bucket((S + bs - 1) / bs);
+    if (n > 1) {
+      const int p = atomicAdd(&hist[bf], n - 1);
+      for (int r = 0; r < n - 1; ++r) order[p + r] = make_int4(s, r, (r + 1) * S, n);
+    }
+    order[atomicAdd(&hist[bucket((last + bs - 1) / bs)], 1)] = make_int4(s, n - 1, c, n);
+  }
 }
 
 // Keep the halves of a 32-bit fragment register whose token is valid:
@@ -189,7 +257,9 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
   constexpr bool kMmaBF16 = C::kMmaBF16;
   constexpr int kStages = C::kStages;
   extern __shared__ __align__(128) uint8_t smem[];
-  __shared__ int s_item;
+  __shared__ int s_item;   // the CTA's next item ...
+  __shared__ int4 s_desc;  // ... and its descriptor (a.order entry)
+  __shared__ int s_flag;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -215,39 +285,32 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
   __syncthreads();
 
   const int total = *a.total;
-  const bool split_mode = a.split_tokens < a.max_ctx;
   uint32_t n_issued = 0, n_consumed = 0;  // warp-uniform ring counters
   uint32_t skip_stage = 0;                // stages holding a block with a bad table entry
   bool failed = false;                    // a wait timed out: stop issuing / computing
 
+  // the next item and its descriptor, fetched by thread 0
+  auto fetch_next = [&]() {
+    const int it = atomicAdd(a.counter, 1);
+    s_item = it;
+    if (it < total) s_desc = a.order[it / a.hkv];
+  };
+  if (threadIdx.x == 0) fetch_next();
+  __syncthreads();
+
   for (;;) {
-    if (threadIdx.x == 0) s_item = atomicAdd(a.counter, 1);
-    __syncthreads();
     const int item = s_item;
     if (item >= total) break;
 
-    // ---- item -> (sequence, range, kv head)
+    // ---- item -> (sequence, range, kv head); kv heads innermost, so the
+    // heads of one range run side by side and share the table's cache lines
     const int kvh = item % a.hkv;
-    const int r = item / a.hkv;
-    int seq, split, nsplit;
-    if (split_mode) {
-      int lo = 0, hi = a.num_seqs;  // largest seq with seq_off[seq] <= r
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (a.seq_off[mid] <= r) lo = mid; else hi = mid;
-      }
-      seq = lo;
-      split = r - a.seq_off[seq];
-      nsplit = a.seq_off[seq + 1] - a.seq_off[seq];
-    } else {
-      seq = r;
-      split = 0;
-      nsplit = 1;
-    }
-    int ctx = a.context_lens[seq];
-    if (ctx < 0 || ctx > a.max_ctx || ctx > a.max_blocks * BS) ctx = 0;  // recorded by plan_kernel
+    const int4 desc = s_desc;
+    const int seq = desc.x;
+    const int split = desc.y;
+    const int t1 = desc.z;  // end token of the range (validated by plan_kernel)
+    const int nsplit = desc.w;
     const int t0 = split * a.split_tokens;
-    const int t1 = min(ctx, t0 + a.split_tokens);
     const int jb0 = t0 / BS;
     const int nblk = t1 > t0 ? (t1 + BS - 1) / BS - jb0 : 0;
     const int nb_w = nblk > warp ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
@@ -551,6 +614,75 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
         }
       }
     }
+    if (nsplit > 1) {
+      // The CTA that finishes the last range of this (sequence, kv head)
+      // merges all its ranges: out = sum_i w_i o_i / sum_i w_i with
+      // w_i = 2^(lse_i - max lse).  Partials are published with a fence
+      // before the arrival count and read after it through L2.
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        const int prev = atomicAdd(&a.arrived[seq * a.hkv + kvh], 1);
+        s_flag = (prev == nsplit - 1) ? 1 : 0;
+      }
+      __syncthreads();
+      if (s_flag) {
+        __threadfence();
+        // (1) every range's lse of every head into shared memory (the ring is
+        // free: the warps' scratch was consumed above), (2) per head the max
+        // and the weights w_i = 2^(lse_i - max), (3) the weighted sum of the
+        // partial outputs with independent (unrolled) loads
+        float* lse_s = reinterpret_cast<float*>(ring);           // [nsplit][group]
+        float* wsum_s = lse_s + nsplit * a.group;                // [group]
+        const int64_t base = static_cast<int64_t>(a.seq_off[seq]) * a.hq + h0;
+        const int npairs = nsplit * a.group;
+        for (int k = threadIdx.x; k < npairs; k += kDecodeThreads) {
+          const int i = k / a.group, h = k % a.group;
+          lse_s[k] = __ldcg(a.lse_part + base + static_cast<int64_t>(i) * a.hq + h);
+        }
+        __syncthreads();
+        for (int h = warp; h < a.group; h += kDecodeWarps) {
+          float M = -INFINITY;
+          for (int i = lane; i < nsplit; i += 32) M = fmaxf(M, lse_s[i * a.group + h]);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+          float W = 0.f;
+          for (int i = lane; i < nsplit; i += 32) {
+            const float w = (M == -INFINITY) ? 0.f : fast_exp2(lse_s[i * a.group + h] - M);
+            lse_s[i * a.group + h] = w;  // now the weight
+            W += w;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+          if (lane == 0) wsum_s[h] = W;
+        }
+        __syncthreads();
+        constexpr int kVec = 4;
+        const int units = a.group * (D / kVec);
+        for (int u = threadIdx.x; u < units; u += kDecodeThreads) {
+          const int h = u / (D / kVec);
+          const int d0 = (u % (D / kVec)) * kVec;
+          float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+          const float* op = a.o_part + (base + h) * D + d0;
+#pragma unroll 8
+          for (int i = 0; i < nsplit; ++i) {
+            const float w = lse_s[i * a.group + h];
+            const float4 x = __ldcg(reinterpret_cast<const float4*>(op + static_cast<int64_t>(i) * a.hq * D));
+            o0 += w * x.x; o1 += w * x.y; o2 += w * x.z; o3 += w * x.w;
+          }
+          const float W = wsum_s[h];
+          const float inv = W > 0.f ? 1.f / W : 0.f;
+          uint2 pk;
+          pk.x = static_cast<uint32_t>(from_float<kQBF16>(o0 * inv)) | (static_cast<uint32_t>(from_float<kQBF16>(o1 * inv)) << 16);
+          pk.y = static_cast<uint32_t>(from_float<kQBF16>(o2 * inv)) | (static_cast<uint32_t>(from_float<kQBF16>(o3 * inv)) << 16);
+          *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.out) +
+                                    (static_cast<int64_t>(seq) * a.hq + h0 + h) * D + d0) = pk;
+        }
+      }
+    }
+    // the next item is taken only now, when this CTA can start it at once,
+    // so no CTA holds an item it cannot start while others run dry
+    if (threadIdx.x == 0) fetch_next();
     __syncthreads();           // scratch (= stage memory) is free again ...
     fence_proxy_async_smem();  // ... and the next item's tile loads come after these accesses
   }
@@ -563,45 +695,6 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
       ++n_consumed;
     }
   }
-}
-
-// ------------------------------------------------------------ merge kernel
-// out[s, h, :] = sum_i w_i o_i / sum_i w_i with w_i = 2^(lse_i - max lse) over
-// the ranges i of sequence s; sequences with one range were written by the
-// main kernel directly.
-template <bool kOutBF16>
-__global__ void __launch_bounds__(128) merge_kernel(void* __restrict__ out,
-                                                    const float* __restrict__ lse_part,
-                                                    const float* __restrict__ o_part,
-                                                    const int32_t* __restrict__ seq_off, int hq,
-                                                    int D) {
-  const int seq = blockIdx.y;
-  const int base = seq_off[seq];
-  const int n = seq_off[seq + 1] - base;
-  if (n <= 1) return;
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  const int per_head = D / 4;
-  const int h = e / per_head;
-  if (h >= hq) return;
-  const int d0 = (e % per_head) * 4;
-  float M = -INFINITY;
-  for (int i = 0; i < n; ++i) M = fmaxf(M, lse_part[static_cast<int64_t>(base + i) * hq + h]);
-  float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f, W = 0.f;
-  if (M != -INFINITY) {
-    for (int i = 0; i < n; ++i) {
-      const int64_t pi = static_cast<int64_t>(base + i) * hq + h;
-      const float w = fast_exp2(lse_part[pi] - M);
-      const float4 x = *reinterpret_cast<const float4*>(o_part + pi * D + d0);
-      W += w;
-      o0 += w * x.x; o1 += w * x.y; o2 += w * x.z; o3 += w * x.w;
-    }
-    const float inv = 1.f / W;
-    o0 *= inv; o1 *= inv; o2 *= inv; o3 *= inv;
-  }
-  uint2 pk;
-  pk.x = static_cast<uint32_t>(from_float<kOutBF16>(o0)) | (static_cast<uint32_t>(from_float<kOutBF16>(o1)) << 16);
-  pk.y = static_cast<uint32_t>(from_float<kOutBF16>(o2)) | (static_cast<uint32_t>(from_float<kOutBF16>(o3)) << 16);
-  *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(out) + (static_cast<int64_t>(seq) * hq + h) * D + d0) = pk;
 }
 
 }  // namespace pa

@@ -73,7 +73,9 @@ constexpr int64_t kLongContext = 4096;    // above this, cap ranges ...
 constexpr int64_t kLongSplit = 1024;      // ... at this many tokens
 
 int32_t choose_split(int32_t B, int32_t hkv, int32_t bs, int32_t max_ctx, int32_t user) {
-  if (user > 0) return static_cast<int32_t>(round_up(user, bs));
+  // at most kMaxRanges ranges per sequence, whatever was asked for
+  const int64_t floor_s = std::max<int64_t>(bs, cdiv(max_ctx, pa::kMaxRanges));
+  if (user > 0) return static_cast<int32_t>(round_up(std::max<int64_t>(user, floor_s), bs));
   if (max_ctx <= 0) return bs;
   const int64_t units = static_cast<int64_t>(B) * hkv;
   // enough ranges for two waves of persistent CTAs ...
@@ -82,26 +84,33 @@ int32_t choose_split(int32_t B, int32_t hkv, int32_t bs, int32_t max_ctx, int32_
   // ... and no single range much longer than the typical one when lengths
   // can spread far (long contexts): the longest sequence is cut up
   if (max_ctx > kLongContext) s = std::min<int64_t>(s, kLongSplit);
-  return static_cast<int32_t>(round_up(s, bs));
+  return static_cast<int32_t>(round_up(std::max(s, floor_s), bs));
 }
 
+// Workspace of one decode call: work counter and item total, per-sequence
+// range offsets [B + 1], the work order [ranges] of int4, and when contexts
+// are split, arrival counters [B * Hkv], fp32 lse [ranges * Hq] and fp32
+// partial outputs [ranges * Hq * D].
 struct WsLayout {
-  size_t counter = 0, total = 4, seq_off = 256, lse = 0, o = 0, bytes = 0;
+  size_t counter = 0, total = 4, seq_off = 256, order = 0, arrived = 0, lse = 0, o = 0, bytes = 0;
   bool split = false;
+  int64_t ranges = 0;  // upper bound on (sequence, range) pairs
 };
 
-WsLayout ws_layout(int32_t B, int32_t hq, int32_t D, int32_t max_ctx, int32_t S) {
+WsLayout ws_layout(int32_t B, int32_t hq, int32_t hkv, int32_t D, int32_t max_ctx, int32_t S) {
   WsLayout w;
-  w.lse = w.seq_off + static_cast<size_t>(round_up(static_cast<int64_t>(B + 1) * 4, 256));
   w.split = S < max_ctx;
+  w.ranges = w.split ? static_cast<int64_t>(B) * cdiv(max_ctx, S) : B;
+  w.order = w.seq_off + static_cast<size_t>(round_up(static_cast<int64_t>(B + 1) * 4, 256));
+  w.arrived = w.order + static_cast<size_t>(round_up(w.ranges * 16, 256));
   if (!w.split) {
-    w.o = w.lse;
-    w.bytes = w.lse;
+    w.lse = w.o = w.arrived;
+    w.bytes = w.arrived;
     return w;
   }
-  const int64_t ranges = static_cast<int64_t>(B) * cdiv(max_ctx, S);
-  w.o = w.lse + static_cast<size_t>(round_up(ranges * hq * 4, 256));
-  w.bytes = w.o + static_cast<size_t>(ranges * hq * D * 4);
+  w.lse = w.arrived + static_cast<size_t>(round_up(static_cast<int64_t>(B) * hkv * 4, 256));
+  w.o = w.lse + static_cast<size_t>(round_up(w.ranges * hq * 4, 256));
+  w.bytes = w.o + static_cast<size_t>(w.ranges * hq * D * 4);
   return w;
 }
 
@@ -286,7 +295,7 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t n
       (block_size != 16 && block_size != 32) || max_context_len < 0 || split_tokens < 0)
     return 0;
   const int32_t S = choose_split(num_seqs, num_kv_heads, block_size, max_context_len, split_tokens);
-  return ws_layout(num_seqs, num_q_heads, head_dim, max_context_len, S).bytes;
+  return ws_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, S).bytes;
 }
 
 pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_pool,
@@ -321,7 +330,7 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_po
   if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens)
     return fail(PA_ERR_NULL, "pa_decode: null pointer");
   const int32_t S = choose_split(num_seqs, num_kv_heads, block_size, max_context_len, split_tokens);
-  const WsLayout w = ws_layout(num_seqs, num_q_heads, head_dim, max_context_len, S);
+  const WsLayout w = ws_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, S);
   if (!workspace || workspace_bytes < w.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return fail(PA_ERR_WORKSPACE, "pa_decode: workspace needs %zu bytes, 256-byte aligned (got %zu)",
                 w.bytes, workspace_bytes);
@@ -346,6 +355,8 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_po
   a.counter = reinterpret_cast<int32_t*>(ws + w.counter);
   a.total = reinterpret_cast<const int32_t*>(ws + w.total);
   a.seq_off = reinterpret_cast<const int32_t*>(ws + w.seq_off);
+  a.order = reinterpret_cast<const int4*>(ws + w.order);
+  a.arrived = reinterpret_cast<int32_t*>(ws + w.arrived);
   a.lse_part = reinterpret_cast<float*>(ws + w.lse);
   a.o_part = reinterpret_cast<float*>(ws + w.o);
   a.num_seqs = num_seqs;
@@ -363,10 +374,10 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_po
                                       block_size, a.split_tokens, num_kv_heads,
                                       reinterpret_cast<int32_t*>(ws + w.counter),
                                       reinterpret_cast<int32_t*>(ws + w.total),
-                                      reinterpret_cast<int32_t*>(ws + w.seq_off));
-  const int64_t ranges_upper =
-      w.split ? static_cast<int64_t>(num_seqs) * cdiv(max_context_len, S) : num_seqs;
-  const int64_t items_upper = ranges_upper * num_kv_heads;
+                                      reinterpret_cast<int32_t*>(ws + w.seq_off),
+                                      reinterpret_cast<int4*>(ws + w.order),
+                                      w.split ? reinterpret_cast<int32_t*>(ws + w.arrived) : nullptr);
+  const int64_t items_upper = w.ranges * num_kv_heads;
   const bool qbf = q_dtype == PA_BF16;
   pa_status s;
   if (cache_dtype == PA_F16)
@@ -378,16 +389,6 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_po
   else
     s = dispatch_shape<pa::kCacheE4M3, false>(a, head_dim, block_size, items_upper, dev, st);
   if (s != PA_OK) return s;
-  if (w.split) {
-    const int units = num_q_heads * (head_dim / 4);
-    dim3 grid(static_cast<unsigned>(cdiv(units, 128)), static_cast<unsigned>(num_seqs));
-    if (qbf)
-      pa::merge_kernel<true><<<grid, 128, 0, st>>>(out, a.lse_part, a.o_part, a.seq_off,
-                                                   num_q_heads, head_dim);
-    else
-      pa::merge_kernel<false><<<grid, 128, 0, st>>>(out, a.lse_part, a.o_part, a.seq_off,
-                                                    num_q_heads, head_dim);
-  }
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
   return ok();

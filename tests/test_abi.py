@@ -43,13 +43,14 @@ def test_library_exports_every_declared_symbol(pa):
 def test_split_and_workspace_rules(pa):
     # one item per (sequence, kv head) when that fills the GPU
     assert pa.pa_decode_split_tokens(256, 8, 16, 4096, 0) == 4096
-    assert pa.pa_decode_workspace_size(256, 64, 8, 128, 16, 4096, 0) == 256 + 1280
+    # header, range offsets [257] int32, work order [256] int4
+    assert pa.pa_decode_workspace_size(256, 64, 8, 128, 16, 4096, 0) == 256 + 1280 + 4096
     # long contexts are cut into ranges (multiples of the block size)
     s = pa.pa_decode_split_tokens(128, 8, 16, 32768, 0)
     assert s == 1024
     ranges = 128 * 32
     assert pa.pa_decode_workspace_size(128, 32, 8, 128, 16, 32768, 0) == \
-        256 + 768 + ranges * 32 * 4 + ranges * 32 * 128 * 4
+        256 + 768 + ranges * 16 + 128 * 8 * 4 + ranges * 32 * 4 + ranges * 32 * 128 * 4
     # few sequences: split for parallelism
     s = pa.pa_decode_split_tokens(1, 8, 32, 16384, 0)
     assert 256 <= s < 16384 and s % 32 == 0
