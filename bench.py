@@ -4,7 +4,7 @@
 A step is one pass of the whole hot path over one batch: copy-on-write block
 copies (none in the default workload), the cache write of every sequence's
 new token (pa_write_kv), and paged decode attention over all sequences
-(pa_decode: plan + main kernel + merge when contexts are split).
+(pa_decode: plan kernel + decode kernel, which also merges split contexts).
 
 Default workload: the Llama-3-70B-shaped GQA decode layer -- 256 sequences
 x 4096 tokens, 64 query / 8 KV heads, head_dim 128, bf16, block_size 16,
@@ -416,7 +416,7 @@ def run_ours(args, rank, local, world):
         "roofline": {
             "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
             "frac": round(achieved / peak, 4), "traffic": profiled_traffic(),
-            "kernel": "pa_decode (plan + decode_kernel" + (" + merge" if split < w.max_context_len else "") + ")",
+            "kernel": "pa_decode (plan_kernel + decode_kernel)",
             "algorithmic_bytes_per_launch": w.kv_bytes, "peak_kind": peak_kind,
             "mean_launch_us": round(dec_mean_s * 1e6, 2),
         },

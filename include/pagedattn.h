@@ -159,14 +159,16 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
  *
  * Contexts longer than the split length are cut into ranges of split_tokens
  * tokens (0 = automatic, see pa_decode_split_tokens); each range writes a
- * partial (log-sum-exp, normalised vector) into the workspace and a merge
- * pass combines them.  Results depend only on the arguments (not on the grid
- * or on timing): the same call gives bit-identical outputs.
+ * partial (log-sum-exp, normalised vector) into the workspace; the kernel
+ * that finishes a sequence's last range combines them (log-sum-exp merge).
+ * Results depend only on the arguments (not on the grid or on timing): the
+ * same call gives bit-identical outputs.
  *
  * max_context_len must bound every context_lens[s]; a larger length, or one
  * above max_blocks_per_seq * bs, makes that sequence's output zero and
  * reports PA_ERR_DEVICE_BOUNDS.  A table entry outside [0, num_blocks) is
- * skipped (its tokens masked) and reported the same way.
+ * skipped (its tokens left out) and reported the same way.  The pools must be
+ * 16-byte aligned (they are read through TMA tensor maps).
  * workspace: device memory of at least pa_decode_workspace_size(...) bytes,
  * 256-byte aligned, used only during the call (stream-ordered).
  */
