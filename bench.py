@@ -57,6 +57,9 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling only)")
+    ap.add_argument("--op", choices=["decode", "swap", "hash"], default="decode",
+                    help="decode: the decode step (the headline line); the others time "
+                         "one companion operation on one GPU and print its own line")
     return ap.parse_args(argv)
 
 
@@ -482,6 +485,106 @@ def run_reference(args, rank, world):
     }
 
 
+# ------------------------------------------------------- companion operations
+def _events_time(fn, iters, warmup=3):
+    """Mean seconds per call of fn() on the current stream, by CUDA events."""
+    import torch
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(iters):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / 1e3 / iters
+
+
+def run_swap(args):
+    """pa_swap_blocks: move 2048 blocks of the Llama-3-70B-shaped pool (bs 16,
+    8 kv heads, D 128, bf16: 64 KiB of K+V per block) from the device pool to
+    pinned host memory and back, scattered ids.  Roofline: one large pinned
+    cudaMemcpy of the same bytes in the same direction, timed in this run."""
+    import torch
+    from paged_kv_cache_416_b200 import build as _build
+    _build.build()
+    from paged_kv_cache_416_b200 import pagedattn as pa
+    torch.cuda.set_device(0)
+    nb, shape = 2048, (16, 8, 128)
+    g = torch.Generator(device="cuda").manual_seed(args.seed)
+    dev_k = torch.randn((8192,) + shape, generator=g, device="cuda").to(torch.bfloat16)
+    dev_v = torch.randn((8192,) + shape, generator=g, device="cuda").to(torch.bfloat16)
+    host_k = torch.empty((nb,) + shape, dtype=torch.bfloat16).pin_memory()
+    host_v = torch.empty((nb,) + shape, dtype=torch.bfloat16).pin_memory()
+    gc = torch.Generator().manual_seed(args.seed)
+    src = torch.randperm(8192, generator=gc)[:nb]
+    dst = torch.randperm(nb, generator=gc)
+    out_pairs = torch.stack([src, dst], 1).to(torch.int64).cuda()
+    in_pairs = torch.stack([dst, src], 1).to(torch.int64).cuda()
+    moved = 2 * nb * 16 * 8 * 128 * 2
+    iters = max(3, min(args.steps, 50))
+    t_out = _events_time(lambda: pa.swap_blocks(dev_k, dev_v, host_k, host_v, out_pairs), iters)
+    t_in = _events_time(lambda: pa.swap_blocks(host_k, host_v, dev_k, dev_v, in_pairs), iters)
+    pa.sync_status()
+    flat_dev = torch.empty(moved, dtype=torch.uint8, device="cuda")
+    flat_host = torch.empty(moved, dtype=torch.uint8).pin_memory()
+    t_d2h = _events_time(lambda: flat_host.copy_(flat_dev, non_blocking=True), iters)
+    t_h2d = _events_time(lambda: flat_dev.copy_(flat_host, non_blocking=True), iters)
+    out_gbs, in_gbs = moved / t_out / 1e9, moved / t_in / 1e9
+    return {
+        "metric": "block swap GB/s (device pool <-> pinned host)", "op": "swap",
+        "value": round(min(out_gbs, in_gbs), 2), "unit": "GB/s", "n_gpus": 1,
+        "steps": iters, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "2048 scattered blocks of 16x8x128 bf16 (K and V), 256 MiB moved",
+                   "bytes_per_call": moved},
+        "swap_out_gbs": round(out_gbs, 2), "swap_in_gbs": round(in_gbs, 2),
+        "swap_out_us": round(t_out * 1e6, 1), "swap_in_us": round(t_in * 1e6, 1),
+        "roofline": {"bound": "host link", "achieved": round(min(out_gbs, in_gbs), 2),
+                     "peak": round(min(moved / t_d2h, moved / t_h2d) / 1e9, 2), "unit": "GB/s",
+                     "frac": round(min(out_gbs / (moved / t_d2h / 1e9), in_gbs / (moved / t_h2d / 1e9)), 4),
+                     "peak_kind": "one pinned cudaMemcpy of the same bytes, measured in this run",
+                     "memcpy_d2h_gbs": round(moved / t_d2h / 1e9, 2),
+                     "memcpy_h2d_gbs": round(moved / t_h2d / 1e9, 2)},
+        "gpu_launches": 2 * iters,
+    }
+
+
+def run_hash(args):
+    """pa_hash_blocks over 256 sequences x 4096 token ids (bs 16, 65,536
+    full blocks).  Roofline: plain ALU -- about 20 integer instructions per
+    token (FNV-1a: xor + 64-bit multiply per byte of the 4-byte id, plus the
+    per-block chain step) against 148 SMs x 128 lanes x the SM clock; the
+    chain itself is serial along a sequence, which is what bounds the call."""
+    import torch
+    from paged_kv_cache_416_b200 import build as _build
+    _build.build()
+    from paged_kv_cache_416_b200 import pagedattn as pa
+    torch.cuda.set_device(0)
+    B, L, bs = 256, 4096, 16
+    g = torch.Generator(device="cuda").manual_seed(args.seed)
+    toks = torch.randint(0, 128256, (B, L), generator=g, device="cuda", dtype=torch.int32)
+    lens = torch.full((B,), L, dtype=torch.int32, device="cuda")
+    out = torch.empty((B, L // bs), dtype=torch.int64, device="cuda")
+    iters = max(3, min(args.steps, 50))
+    t = _events_time(lambda: pa.hash_blocks(toks, lens, bs, out=out), iters)
+    pa.sync_status()
+    tps = B * L / t
+    clock = ClockSampler(0).max_mhz or 1965.0
+    peak = 148 * 128 * clock * 1e6 / 20
+    return {
+        "metric": "prefix-cache block hashing, token ids hashed per second", "op": "hash",
+        "value": round(tps, 1), "unit": "tokens/s", "n_gpus": 1, "steps": iters,
+        "higher_is_better": True, "dtype": "int32", "data": "synthetic",
+        "config": {"workload": "256 sequences x 4096 token ids, block_size 16", "blocks": B * L // bs},
+        "us_per_call": round(t * 1e6, 2),
+        "roofline": {"bound": "alu", "achieved": round(tps, 1), "peak": round(peak, 1),
+                     "unit": "tokens/s", "frac": round(tps / peak, 4),
+                     "peak_kind": "derived: 148 SMs x 128 int lanes x max SM clock / 20 instructions per token"},
+        "gpu_launches": iters,
+    }
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.warmup < 3:
@@ -495,6 +598,12 @@ def main(argv=None):
         line = run_reference(args, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
+        return 0
+    if args.op != "decode":
+        if rank != 0:
+            return 0
+        line = {"swap": run_swap, "hash": run_hash}[args.op](args)
+        print(json.dumps(line), flush=True)
         return 0
     import torch
     if world > 1:

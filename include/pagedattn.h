@@ -75,8 +75,10 @@ typedef enum pa_status {
   PA_ERR_CUDA = 7,          /* a CUDA runtime call failed; see pa_last_error() */
   PA_ERR_DEVICE_BOUNDS = 8, /* a kernel met an out-of-range index and skipped it */
   PA_ERR_WORKSPACE = 9,     /* workspace missing or smaller than required */
-  PA_ERR_TIMEOUT = 10       /* a kernel gave up waiting for an asynchronous copy
+  PA_ERR_TIMEOUT = 10,      /* a kernel gave up waiting for an asynchronous copy
                                (about one second) and skipped that block */
+  PA_ERR_MEMORY = 11        /* a buffer the device cannot reach (pageable host
+                               memory) */
 } pa_status;
 
 /*
@@ -117,6 +119,54 @@ pa_status pa_copy_blocks(void* k_pool, void* v_pool, pa_dtype cache_dtype,
                          int32_t num_kv_heads, int32_t head_dim,
                          const int64_t* src_dst_pairs, int32_t num_pairs,
                          pa_stream_t stream);
+
+/*
+ * pa_swap_blocks -- move blocks between two pools of the same block shape,
+ * e.g. out of the device pool into pinned host memory when device memory is
+ * full and back in when they are needed again: the pages' fine-grained
+ * eviction, which moves small pages instead of whole sequences to the CPU
+ * (gyaansetu, first article, the fine-grained eviction bullet of how
+ * PagedAttention solves the memory problem).
+ * For each pair p: dst_k[dst] = src_k[src] and dst_v[dst] = src_v[src], all
+ * bs * Hkv * D elements, with (src, dst) = src_dst_pairs[p] (src indexes the
+ * source pool, dst the destination pool).  Each pool pointer is device memory
+ * or host memory the device can address (pinned by cudaHostAlloc /
+ * cudaHostRegister under unified addressing); pageable host memory is
+ * refused with PA_ERR_MEMORY.  src_dst_pairs lives in device memory.  One
+ * launch moves all pairs; bytes cross the host link once.  Ids outside their
+ * pool skip the pair and report PA_ERR_DEVICE_BOUNDS.  Destinations must be
+ * distinct, and the two pools must not overlap.
+ */
+pa_status pa_swap_blocks(const void* src_k, const void* src_v, int32_t src_blocks,
+                         void* dst_k, void* dst_v, int32_t dst_blocks,
+                         pa_dtype cache_dtype, int32_t block_size,
+                         int32_t num_kv_heads, int32_t head_dim,
+                         const int64_t* src_dst_pairs, int32_t num_pairs,
+                         pa_stream_t stream);
+
+/*
+ * pa_hash_blocks -- chained hashes of full blocks of token ids, the key of a
+ * prefix cache: hashing every block carries block sharing across requests
+ * ("PagedAttention", Ultralytics glossary, section "Diziler Arasinda
+ * Bloklari Paylasma": this is how vLLM implements prompt caching).  A block's
+ * hash covers its own tokens and its parent block's hash, so equal hashes
+ * mean equal prefixes (up to 64-bit collisions; a caller may compare tokens
+ * on a hit).
+ * For sequence s (token ids token_ids[s * token_stride ...], num_tokens[s] of
+ * them) and every full block j < num_tokens[s] / block_size:
+ *   inner_j = FNV1a64(the block's block_size ids, 4 little-endian bytes each)
+ *   hash_j  = FNV1a64(hash_{j-1} as 8 LE bytes, inner_j as 8 LE bytes),
+ *   hash_{-1} = 0,
+ * with FNV1a64 the 64-bit FNV-1a hash (offset basis 0xcbf29ce484222325,
+ * prime 0x100000001b3).  block_hashes[s * max_blocks + j] = hash_j; entries
+ * of blocks that are not full are 0.  A length above token_stride, or more
+ * full blocks than max_blocks, is clamped and reported as
+ * PA_ERR_DEVICE_BOUNDS.  All pointers are device pointers.
+ */
+pa_status pa_hash_blocks(const int32_t* token_ids, int64_t token_stride,
+                         const int32_t* num_tokens, int32_t num_seqs,
+                         int32_t block_size, uint64_t* block_hashes,
+                         int32_t max_blocks, pa_stream_t stream);
 
 /*
  * pa_decode_split_tokens -- the context-split length pa_decode uses for these

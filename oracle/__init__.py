@@ -44,6 +44,7 @@ from .paged import (
     slot_of,
     write_kv,
     copy_blocks,
+    swap_blocks,
     gather,
     attention_weights,
     decode,
@@ -60,6 +61,6 @@ from .memory import (
 __all__ = [
     "bf16_bits_to_f64", "f16_bits_to_f64", "e4m3_decode", "e4m3_encode_f32",
     "e4m3_finite_values", "decode_cache", "slot_of", "write_kv", "copy_blocks",
-    "gather", "attention_weights", "decode", "decode_one", "kv_bytes_per_token",
+    "swap_blocks", "gather", "attention_weights", "decode", "decode_one", "kv_bytes_per_token",
     "kv_bytes", "reservation_unused_slots", "paged_unused_slots", "blocks_needed",
 ]

@@ -77,6 +77,18 @@ def copy_blocks(k_pool, v_pool, pairs):
     return k_pool, v_pool
 
 
+def swap_blocks(src_k, src_v, dst_k, dst_v, pairs):
+    """Move blocks between two pools, in place on the destination:
+    ``dst[d] = src[s]`` for every (s, d) pair, for K and V (gyaansetu, first
+    article: fine-grained eviction moves small pages, not whole sequences,
+    to the CPU when memory is full)."""
+    pairs = np.asarray(pairs, dtype=np.int64).reshape(-1, 2)
+    for src, dst in pairs:
+        dst_k[dst] = src_k[src]
+        dst_v[dst] = src_v[src]
+    return dst_k, dst_v
+
+
 def gather(pool_values, block_table_row, context_len: int) -> np.ndarray:
     """A sequence's contiguous cache ``[context_len, H, D]`` from its blocks:
     the blocks named by the first ceil(len / bs) table entries, concatenated

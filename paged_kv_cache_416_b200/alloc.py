@@ -46,6 +46,9 @@ class BlockAllocator:
         self.refcount = np.zeros(self.num_blocks, dtype=np.int64)
         self.tables: Dict[int, List[int]] = {}
         self.lengths: Dict[int, int] = {}
+        # prefix cache: chained block hash -> physical block holding that prefix
+        self.cached: Dict[int, int] = {}
+        self.block_hash: Dict[int, int] = {}
 
     # -- allocation ----------------------------------------------------------
     def _take(self) -> int:
@@ -99,12 +102,52 @@ class BlockAllocator:
             self.refcount[b] += 1
 
     def free_seq(self, seq: int) -> None:
-        """Drop ``seq``; blocks nobody else uses return to the free list tail."""
+        """Drop ``seq``; blocks nobody else uses return to the free list tail
+        (and leave the prefix cache)."""
         for b in self.tables.pop(seq):
             self.refcount[b] -= 1
             if self.refcount[b] == 0:
                 self.free.append(b)
+                h = self.block_hash.pop(b, None)
+                if h is not None and self.cached.get(h) == b:
+                    del self.cached[h]
         del self.lengths[seq]
+
+    # -- prefix cache ("PagedAttention", §Diziler Arasında Blokları Paylaşma:
+    # hashing every block carries sharing across requests) -----------------
+    def register_prefix(self, seq: int, hashes) -> None:
+        """Remember the full blocks of ``seq`` under their chained hashes
+        (``pa_hash_blocks`` of its tokens), so later requests with the same
+        prefix can share them."""
+        t = self.tables[seq]
+        for j, h in enumerate(hashes):
+            h = int(h) & ((1 << 64) - 1)
+            if j >= len(t) or (j + 1) * self.block_size > self.lengths[seq]:
+                break
+            if h not in self.cached:
+                self.cached[h] = t[j]
+                self.block_hash[t[j]] = h
+
+    def allocate_cached(self, seq: int, num_tokens: int, hashes) -> Tuple[List[int], int]:
+        """Like :meth:`allocate`, but the leading full blocks whose chained
+        hash is cached are shared (reference count + 1) instead of taken from
+        the free list.  Returns (table, number of shared blocks)."""
+        if seq in self.tables:
+            raise KeyError(f"sequence {seq} already exists")
+        n = -(-int(num_tokens) // self.block_size)
+        table: List[int] = []
+        for h in hashes:
+            b = self.cached.get(int(h) & ((1 << 64) - 1))
+            if b is None or len(table) >= n:
+                break
+            self.refcount[b] += 1
+            table.append(b)
+        shared = len(table)
+        while len(table) < n:
+            table.append(self._take())
+        self.tables[seq] = table
+        self.lengths[seq] = int(num_tokens)
+        return list(table), shared
 
     # -- views ----------------------------------------------------------------
     def table_array(self, seqs: List[int], width: Optional[int] = None, pad: int = -1) -> np.ndarray:

@@ -1,5 +1,6 @@
-// Cache maintenance kernels: the slot-mapping scatter of new keys/values and
-// the copy-on-write block copy.
+// Cache maintenance kernels: the slot-mapping scatter of new keys/values,
+// the copy-on-write block copy, the block swap between the device pool and
+// host memory, and the chained block hashes used for prefix caching.
 //
 // Both are pure data movement in 16-byte vectors (HBM-bound, and at decode
 // sizes launch-bound).  "PagedAttention" (Ultralytics glossary): token `pos`
@@ -87,6 +88,110 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint8_t* __restrict__ 
     const uint4 b = vs[i];
     kd[i] = a;
     vd[i] = b;
+  }
+}
+
+// Block swap between two pools of the same block shape, either of which may
+// be host memory mapped into the device's address space (pinned, unified
+// addressing): for each pair p, dst[pairs[p][1]] = src[pairs[p][0]] for K and
+// V.  Grid (x: pair, y: CTAs per pair); each thread keeps 4 independent
+// 16-byte loads in flight per tensor, since host memory sits behind the
+// high-latency host link.
+__global__ void __launch_bounds__(256) swap_blocks_kernel(
+    const uint8_t* __restrict__ src_k, const uint8_t* __restrict__ src_v,
+    uint8_t* __restrict__ dst_k, uint8_t* __restrict__ dst_v, const int64_t* __restrict__ pairs,
+    int64_t src_blocks, int64_t dst_blocks, int64_t block_bytes) {
+  const int64_t p = blockIdx.x;
+  const int64_t src = pairs[2 * p], dst = pairs[2 * p + 1];
+  if (src < 0 || src >= src_blocks || dst < 0 || dst >= dst_blocks) {
+    if (blockIdx.y == 0 && threadIdx.x == 0) record_error(PA_ERR_DEVICE_BOUNDS);
+    return;
+  }
+  const int64_t nvec = block_bytes / 16;
+  const uint4* ks = reinterpret_cast<const uint4*>(src_k + src * block_bytes);
+  const uint4* vs = reinterpret_cast<const uint4*>(src_v + src * block_bytes);
+  uint4* kd = reinterpret_cast<uint4*>(dst_k + dst * block_bytes);
+  uint4* vd = reinterpret_cast<uint4*>(dst_v + dst * block_bytes);
+  const int64_t stride = static_cast<int64_t>(gridDim.y) * blockDim.x;
+  constexpr int kUnroll = 4;
+  for (int64_t i0 = blockIdx.y * static_cast<int64_t>(blockDim.x) + threadIdx.x; i0 < nvec;
+       i0 += kUnroll * stride) {
+    uint4 a[kUnroll], b[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i < nvec) {
+        a[u] = ks[i];
+        b[u] = vs[i];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t i = i0 + u * stride;
+      if (i < nvec) {
+        kd[i] = a[u];
+        vd[i] = b[u];
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------ block hashes
+// 64-bit FNV-1a (Fowler / Noll / Vo): per byte, xor then multiply by the
+// prime, mod 2^64, from the offset basis.
+constexpr unsigned long long kFnvOffset = 0xcbf29ce484222325ull;
+constexpr unsigned long long kFnvPrime = 0x100000001b3ull;
+
+__device__ __forceinline__ unsigned long long fnv1a_u32(unsigned long long h, uint32_t w) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {  // the word's 4 bytes, little-endian order
+    h ^= (w >> (8 * i)) & 0xffu;
+    h *= kFnvPrime;
+  }
+  return h;
+}
+
+// One CTA per sequence.  Phase 1 (all threads): inner_j = FNV-1a over the 4
+// little-endian bytes of each of block j's token ids, for every full block
+// j.  Phase 2 (one thread, in order): hash_j = FNV-1a over hash_{j-1} then
+// inner_j (8 little-endian bytes each), hash_{-1} = 0.  Entries of blocks
+// that are not full are 0.
+__global__ void __launch_bounds__(256) hash_blocks_kernel(
+    const int32_t* __restrict__ tokens, int64_t token_stride, const int32_t* __restrict__ num_tokens,
+    int bs, unsigned long long* __restrict__ hashes, int max_blocks) {
+  const int s = blockIdx.x;
+  int n = num_tokens[s];
+  if (n < 0 || n > token_stride) {
+    if (threadIdx.x == 0) record_error(PA_ERR_DEVICE_BOUNDS);
+    n = n < 0 ? 0 : static_cast<int>(token_stride);
+  }
+  int full = n / bs;
+  if (full > max_blocks) {
+    if (threadIdx.x == 0) record_error(PA_ERR_DEVICE_BOUNDS);
+    full = max_blocks;
+  }
+  const int32_t* row = tokens + static_cast<int64_t>(s) * token_stride;
+  unsigned long long* out = hashes + static_cast<int64_t>(s) * max_blocks;
+  for (int j = threadIdx.x; j < max_blocks; j += blockDim.x) {
+    unsigned long long h = 0;
+    if (j < full) {
+      h = kFnvOffset;
+      for (int t = 0; t < bs; ++t) h = fnv1a_u32(h, static_cast<uint32_t>(row[j * bs + t]));
+    }
+    out[j] = h;
+  }
+  __syncthreads();  // the inner hashes are visible to thread 0
+  if (threadIdx.x == 0) {
+    unsigned long long parent = 0;
+    for (int j = 0; j < full; ++j) {
+      const unsigned long long inner = out[j];
+      unsigned long long h = kFnvOffset;
+      h = fnv1a_u32(h, static_cast<uint32_t>(parent));
+      h = fnv1a_u32(h, static_cast<uint32_t>(parent >> 32));
+      h = fnv1a_u32(h, static_cast<uint32_t>(inner));
+      h = fnv1a_u32(h, static_cast<uint32_t>(inner >> 32));
+      out[j] = parent = h;
+    }
   }
 }
 

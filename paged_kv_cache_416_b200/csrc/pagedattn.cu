@@ -280,6 +280,60 @@ pa_status pa_copy_blocks(void* k_pool, void* v_pool, pa_dtype cache_dtype, int32
   return ok();
 }
 
+pa_status pa_swap_blocks(const void* src_k, const void* src_v, int32_t src_blocks, void* dst_k,
+                         void* dst_v, int32_t dst_blocks, pa_dtype cache_dtype, int32_t block_size,
+                         int32_t num_kv_heads, int32_t head_dim, const int64_t* src_dst_pairs,
+                         int32_t num_pairs, pa_stream_t stream) {
+  if (!valid_dtype(cache_dtype)) return fail(PA_ERR_DTYPE, "pa_swap_blocks: unknown dtype");
+  if (num_pairs < 0 || !cache_shape_ok(src_blocks, block_size, num_kv_heads, head_dim) ||
+      dst_blocks <= 0)
+    return fail(PA_ERR_SHAPE, "pa_swap_blocks: unsupported sizes");
+  if (num_pairs == 0) return ok();
+  if (!src_k || !src_v || !dst_k || !dst_v || !src_dst_pairs)
+    return fail(PA_ERR_NULL, "pa_swap_blocks: null pointer");
+  const void* ptrs[5] = {src_k, src_v, dst_k, dst_v, src_dst_pairs};
+  for (const void* p : ptrs) {  // every buffer must be reachable from the device
+    cudaPointerAttributes at;
+    const cudaError_t e = cudaPointerGetAttributes(&at, p);
+    if (e != cudaSuccess) {
+      cudaGetLastError();
+      return fail(PA_ERR_MEMORY, "pa_swap_blocks: a buffer is not known to CUDA");
+    }
+    const bool reachable = at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged ||
+                           (at.type == cudaMemoryTypeHost && at.devicePointer == p);
+    if (!reachable)
+      return fail(PA_ERR_MEMORY, "pa_swap_blocks: a buffer is pageable or not mapped for the device");
+  }
+  const int64_t block_bytes =
+      static_cast<int64_t>(block_size) * num_kv_heads * head_dim * elem_bytes(cache_dtype);
+  const int64_t nvec = block_bytes / 16;
+  const unsigned per_pair = static_cast<unsigned>(std::min<int64_t>(8, cdiv(nvec, 256 * 4)));
+  dim3 grid(static_cast<unsigned>(num_pairs), std::max(1u, per_pair));
+  pa::swap_blocks_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint8_t*>(src_k), static_cast<const uint8_t*>(src_v),
+      static_cast<uint8_t*>(dst_k), static_cast<uint8_t*>(dst_v), src_dst_pairs, src_blocks,
+      dst_blocks, block_bytes);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pa_swap_blocks launch");
+  return ok();
+}
+
+pa_status pa_hash_blocks(const int32_t* token_ids, int64_t token_stride,
+                         const int32_t* num_tokens, int32_t num_seqs, int32_t block_size,
+                         uint64_t* block_hashes, int32_t max_blocks, pa_stream_t stream) {
+  if (num_seqs < 0 || block_size <= 0 || max_blocks <= 0 || token_stride <= 0)
+    return fail(PA_ERR_SHAPE, "pa_hash_blocks: bad sizes");
+  if (num_seqs == 0) return ok();
+  if (!token_ids || !num_tokens || !block_hashes) return fail(PA_ERR_NULL, "pa_hash_blocks: null pointer");
+  pa::hash_blocks_kernel<<<static_cast<unsigned>(num_seqs), 256, 0,
+                           reinterpret_cast<cudaStream_t>(stream)>>>(
+      token_ids, token_stride, num_tokens, block_size,
+      reinterpret_cast<unsigned long long*>(block_hashes), max_blocks);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pa_hash_blocks launch");
+  return ok();
+}
+
 int32_t pa_decode_split_tokens(int32_t num_seqs, int32_t num_kv_heads, int32_t block_size,
                                int32_t max_context_len, int32_t split_tokens) {
   if (num_seqs < 0 || num_kv_heads <= 0 || (block_size != 16 && block_size != 32) ||

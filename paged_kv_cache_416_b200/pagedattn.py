@@ -28,7 +28,7 @@ PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
 STATUS_NAMES = {
     0: "PA_OK", 1: "PA_ERR_NULL", 2: "PA_ERR_DTYPE", 3: "PA_ERR_SHAPE", 4: "PA_ERR_HEADS",
     5: "PA_ERR_RANGE", 6: "PA_ERR_ALIAS", 7: "PA_ERR_CUDA", 8: "PA_ERR_DEVICE_BOUNDS",
-    9: "PA_ERR_WORKSPACE", 10: "PA_ERR_TIMEOUT",
+    9: "PA_ERR_WORKSPACE", 10: "PA_ERR_TIMEOUT", 11: "PA_ERR_MEMORY",
 }
 _TORCH_TO_PA = {torch.float16: PA_F16, torch.bfloat16: PA_BF16, torch.float8_e4m3fn: PA_FP8_E4M3}
 
@@ -45,6 +45,8 @@ def declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     sig = {
         "pa_write_kv": (I32, [P, P, I32, P, I32, P, P, I32, I32, I32, I32, I32, F, F, P]),
         "pa_copy_blocks": (I32, [P, P, I32, I32, I32, I32, I32, P, I32, P]),
+        "pa_swap_blocks": (I32, [P, P, I32, P, P, I32, I32, I32, I32, I32, P, I32, P]),
+        "pa_hash_blocks": (I32, [P, I64, P, I32, I32, P, I32, P]),
         "pa_decode_split_tokens": (I32, [I32, I32, I32, I32, I32]),
         "pa_decode_workspace_size": (SZ, [I32, I32, I32, I32, I32, I32, I32]),
         "pa_decode": (I32, [P, P, I32, P, P, I32, P, I32, P, I32, I32, I32, I32, I32, I32, I32,
@@ -77,6 +79,8 @@ _lib = _load()
 # the C entry points, unchanged
 pa_write_kv = _lib.pa_write_kv
 pa_copy_blocks = _lib.pa_copy_blocks
+pa_swap_blocks = _lib.pa_swap_blocks
+pa_hash_blocks = _lib.pa_hash_blocks
 pa_decode_split_tokens = _lib.pa_decode_split_tokens
 pa_decode_workspace_size = _lib.pa_decode_workspace_size
 pa_decode = _lib.pa_decode
@@ -91,7 +95,7 @@ pa_decode_noalloc = _lib.pa_decode_noalloc
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 ENTRY_POINTS = [
-    "pa_write_kv", "pa_copy_blocks", "pa_decode_split_tokens", "pa_decode_workspace_size",
+    "pa_write_kv", "pa_copy_blocks", "pa_swap_blocks", "pa_hash_blocks", "pa_decode_split_tokens", "pa_decode_workspace_size",
     "pa_decode", "pa_sync_status", "pa_last_error", "pa_validate_slot_mapping",
     "pa_validate_copy_pairs", "pa_validate_block_tables", "pa_decode_noalloc",
 ]
@@ -153,6 +157,36 @@ def copy_blocks(k_pool, v_pool, pairs, stream=None) -> None:
     N, bs, hkv, d = k_pool.shape
     check(pa_copy_blocks(_ptr(k_pool), _ptr(v_pool), _dtype(k_pool), N, bs, hkv, d, _ptr(pairs),
                          pairs.shape[0], _stream(stream)))
+
+
+def swap_blocks(src_k, src_v, dst_k, dst_v, pairs, stream=None) -> None:
+    """pa_swap_blocks on tensors: pools [N, bs, Hkv, D] of one dtype, on the
+    device or in pinned host memory; pairs int64 [P, 2] (src id, dst id) on
+    the device."""
+    _contig(src_k, src_v, dst_k, dst_v, pairs)
+    if pairs.dtype != torch.int64:
+        raise TypeError("pairs must be int64")
+    if src_k.shape[1:] != dst_k.shape[1:] or src_k.dtype != dst_k.dtype:
+        raise ValueError("the pools must share block shape and dtype")
+    N, bs, hkv, d = src_k.shape
+    check(pa_swap_blocks(_ptr(src_k), _ptr(src_v), N, _ptr(dst_k), _ptr(dst_v), dst_k.shape[0],
+                         _dtype(src_k), bs, hkv, d, _ptr(pairs), pairs.shape[0], _stream(stream)))
+
+
+def hash_blocks(token_ids, num_tokens, block_size: int, max_blocks: Optional[int] = None,
+                out=None, stream=None) -> torch.Tensor:
+    """pa_hash_blocks on tensors: token_ids int32 [B, L], num_tokens int32 [B]
+    -> int64 [B, max_blocks] (the uint64 hash bits)."""
+    _contig(token_ids, num_tokens)
+    if token_ids.dtype != torch.int32 or num_tokens.dtype != torch.int32:
+        raise TypeError("token_ids and num_tokens must be int32")
+    B, L = token_ids.shape
+    mb = max(1, L // block_size) if max_blocks is None else int(max_blocks)
+    if out is None:
+        out = torch.empty((B, mb), dtype=torch.int64, device=token_ids.device)
+    check(pa_hash_blocks(_ptr(token_ids), L, _ptr(num_tokens), B, block_size, _ptr(out), mb,
+                         _stream(stream)))
+    return out
 
 
 def decode_split_tokens(num_seqs, num_kv_heads, block_size, max_context_len, split_tokens=0) -> int:

@@ -435,3 +435,21 @@ def test_planted_e4m3_tie_rule_is_caught(monkeypatch):
     monkeypatch.setattr(codecs, "e4m3_encode_f32", ties_away)
     with pytest.raises(AssertionError):
         test_e4m3_encode_matches_library_cast()
+
+
+def test_swap_out_and_back_in_restores_the_blocks():
+    """Evicting blocks to a second pool and bringing them back into other
+    slots leaves their bytes unchanged and touches nothing else."""
+    rng = np.random.default_rng(27)
+    dev_k = rng.integers(0, 1 << 16, size=(10, 4, 2, 8), dtype=np.uint16)
+    dev_v = rng.integers(0, 1 << 16, size=(10, 4, 2, 8), dtype=np.uint16)
+    host_k = np.zeros((6, 4, 2, 8), np.uint16)
+    host_v = np.zeros((6, 4, 2, 8), np.uint16)
+    k0, v0 = dev_k.copy(), dev_v.copy()
+    paged.swap_blocks(dev_k, dev_v, host_k, host_v, [[3, 0], [7, 5]])
+    assert np.array_equal(host_k[0], k0[3]) and np.array_equal(host_v[5], v0[7])
+    assert not host_k[1:5].any()
+    dev_k[[3, 7]] = 0
+    paged.swap_blocks(host_k, host_v, dev_k, dev_v, [[0, 9], [5, 3]])
+    assert np.array_equal(dev_k[9], k0[3]) and np.array_equal(dev_v[3], v0[7])
+    assert np.array_equal(dev_k[:3], k0[:3]) and np.array_equal(dev_k[4:7], k0[4:7])
