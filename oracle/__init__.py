@@ -49,6 +49,7 @@ from .paged import (
     attention_weights,
     decode,
     decode_one,
+    prefill,
 )
 from .memory import (
     kv_bytes_per_token,
@@ -61,6 +62,6 @@ from .memory import (
 __all__ = [
     "bf16_bits_to_f64", "f16_bits_to_f64", "e4m3_decode", "e4m3_encode_f32",
     "e4m3_finite_values", "decode_cache", "slot_of", "write_kv", "copy_blocks",
-    "swap_blocks", "gather", "attention_weights", "decode", "decode_one", "kv_bytes_per_token",
+    "swap_blocks", "gather", "attention_weights", "decode", "decode_one", "prefill", "kv_bytes_per_token",
     "kv_bytes", "reservation_unused_slots", "paged_unused_slots", "blocks_needed",
 ]

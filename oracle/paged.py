@@ -154,3 +154,40 @@ def decode(q_raw, q_dtype: str, k_pool, v_pool, cache_dtype: str, block_tables,
         kv_v = decode_cache(v_pool[ids], cache_dtype, v_scale)
         out[s] = decode_one(q[s], kv_k, kv_v, np.arange(nb), n, scale, num_kv_heads)
     return out
+
+
+def prefill(q_raw, q_dtype: str, k_pool, v_pool, cache_dtype: str, block_tables, context_lens,
+            query_start, scale: float, num_kv_heads: int, k_scale: float = 1.0,
+            v_scale: float = 1.0, seqs=None) -> np.ndarray:
+    """Paged prefill (chunked prefill) attention, fp64.
+
+    Sequence s has ``n = query_start[s+1] - query_start[s]`` new query tokens
+    ``q[query_start[s] + i]`` at positions ``context_lens[s] - n + i`` (their
+    K/V already in the cache).  Token i attends causally to cached tokens
+    0..its position, gathered through the block table ("PagedAttention",
+    §İlgili Teknikler: FlashAttention-style kernels read the paged blocks).
+    Returns ``[total_q, Hq, D]``; rows of sequences not in ``seqs`` are 0.
+    """
+    q = decode_cache(q_raw, q_dtype)
+    total, hq, d = q.shape
+    out = np.zeros((total, hq, d), dtype=np.float64)
+    bs = k_pool.shape[1]
+    group = hq // num_kv_heads
+    qs = np.asarray(query_start, dtype=np.int64)
+    seqs = range(len(qs) - 1) if seqs is None else seqs
+    for s in seqs:
+        n = int(qs[s + 1] - qs[s])
+        ctx = int(context_lens[s])
+        if n <= 0 or ctx <= 0:
+            continue
+        nb = -(-ctx // bs)
+        ids = np.asarray(block_tables[s][:nb], dtype=np.int64)
+        K = gather(decode_cache(k_pool[ids], cache_dtype, k_scale), np.arange(nb), ctx)
+        V = gather(decode_cache(v_pool[ids], cache_dtype, v_scale), np.arange(nb), ctx)
+        for i in range(n):
+            pos = ctx - n + i
+            for h in range(hq):
+                kv = h // group
+                w = attention_weights(q[qs[s] + i, h], K[: pos + 1, kv, :], scale)
+                out[qs[s] + i, h] = w @ V[: pos + 1, kv, :]
+    return out

@@ -453,3 +453,59 @@ def test_swap_out_and_back_in_restores_the_blocks():
     paged.swap_blocks(host_k, host_v, dev_k, dev_v, [[0, 9], [5, 3]])
     assert np.array_equal(dev_k[9], k0[3]) and np.array_equal(dev_v[3], v0[7])
     assert np.array_equal(dev_k[:3], k0[:3]) and np.array_equal(dev_k[4:7], k0[4:7])
+
+
+# --------------------------------------------------------------------------
+# paged prefill (causal, chunked)
+# --------------------------------------------------------------------------
+
+def _prefill_case(rng, hq, hkv, d, bs, ctxs, nqs, dtype="f16"):
+    B = len(ctxs)
+    nbs = [-(-c // bs) for c in ctxs]
+    N = sum(nbs) + 3
+    perm = rng.permutation(N)
+    tables, o = np.full((B, max(nbs)), -1, np.int64), 0
+    for s, nb in enumerate(nbs):
+        tables[s, :nb] = perm[o:o + nb]
+        o += nb
+    to = lambda x: torch.from_numpy(x.astype(np.float32)).to(torch.float16).view(torch.int16).numpy().view(np.uint16)
+    kp = to(rng.standard_normal((N, bs, hkv, d)))
+    vp = to(rng.standard_normal((N, bs, hkv, d)))
+    qs = np.concatenate([[0], np.cumsum(nqs)])
+    q = to(rng.standard_normal((int(qs[-1]), hq, d)))
+    return q, kp, vp, tables, qs
+
+
+def test_prefill_matches_library_sdpa_with_causal_offset():
+    rng = np.random.default_rng(31)
+    hq, hkv, d, bs = 8, 2, 32, 16
+    ctxs, nqs = [50, 17, 33], [50, 5, 1]        # full prefill, a chunk, one token
+    q, kp, vp, tables, qs = _prefill_case(rng, hq, hkv, d, bs, ctxs, nqs)
+    got = paged.prefill(q, "f16", kp, vp, "f16", tables, ctxs, qs, 0.2, hkv)
+    Q = codecs.f16_bits_to_f64(q)
+    for s, (ctx, n) in enumerate(zip(ctxs, nqs)):
+        nb = -(-ctx // bs)
+        K = codecs.f16_bits_to_f64(kp[tables[s, :nb]]).reshape(-1, hkv, d)[:ctx]
+        V = codecs.f16_bits_to_f64(vp[tables[s, :nb]]).reshape(-1, hkv, d)[:ctx]
+        pos = ctx - n + np.arange(n)
+        mask = torch.from_numpy(np.arange(ctx)[None, :] <= pos[:, None])  # [n, ctx]
+        ref = F.scaled_dot_product_attention(
+            torch.from_numpy(Q[qs[s]:qs[s + 1]]).permute(1, 0, 2)[None],
+            torch.from_numpy(K).permute(1, 0, 2)[None], torch.from_numpy(V).permute(1, 0, 2)[None],
+            attn_mask=mask, scale=0.2, enable_gqa=True)[0].permute(1, 0, 2)
+        np.testing.assert_allclose(got[qs[s]:qs[s + 1]], ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_prefill_last_token_equals_decode_and_first_token_sees_itself_only():
+    rng = np.random.default_rng(32)
+    hq, hkv, d, bs = 4, 4, 16, 16
+    ctxs, nqs = [40, 9], [40, 9]
+    q, kp, vp, tables, qs = _prefill_case(rng, hq, hkv, d, bs, ctxs, nqs)
+    pre = paged.prefill(q, "f16", kp, vp, "f16", tables, ctxs, qs, 0.25, hkv)
+    last = q[[qs[1] - 1, qs[2] - 1]]
+    dec = paged.decode(last, "f16", kp, vp, "f16", tables, ctxs, 0.25, hkv)
+    np.testing.assert_allclose(pre[[qs[1] - 1, qs[2] - 1]], dec, rtol=1e-13, atol=1e-13)
+    # a full prefill's first token attends only to itself: its value row
+    v0 = codecs.f16_bits_to_f64(vp[tables[0, 0], 0])
+    for h in range(hq):
+        assert np.array_equal(pre[0, h], v0[h])
