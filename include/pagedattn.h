@@ -233,6 +233,35 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype,
                     void* workspace, size_t workspace_bytes, pa_stream_t stream);
 
 /*
+ * pa_prefill -- paged prefill / chunked-prefill attention on the 5th-
+ * generation tensor cores.  Several new query tokens per sequence attend
+ * causally to the sequence's cached keys and values, gathered block by block
+ * through its block table by FlashAttention-style tiles ("PagedAttention",
+ * Ultralytics glossary, section "Ilgili Teknikler": current engines run
+ * FlashAttention-style kernels that read from paged blocks).
+ * Sequence s has n_s = query_start[s+1] - query_start[s] new tokens, rows
+ * query_start[s] .. +n_s of q and out ([total_q, Hq, D], packed), at positions
+ * context_lens[s] - n_s .. context_lens[s] - 1; their K/V must already be in
+ * the cache (pa_write_kv).  Token i at position p, query head h (kv head
+ * h / (Hq / Hkv)):
+ *   out = sum_{t <= p} softmax_t(scale * <q, K_s[t]>) V_s[t]
+ * accumulated in fp32, rounded to q's dtype.  query_start is int32 [B + 1],
+ * device memory.  Supported: head_dim 128; q and cache both f16 or both
+ * bf16; Hq / Hkv dividing 128; block_size 16 or 32.  max_query_len must
+ * bound every n_s (rows past it are not computed) and max_context_len every
+ * context length; a length below n_s or above the maxima zeroes that
+ * sequence's rows and reports PA_ERR_DEVICE_BOUNDS.  No workspace.
+ */
+pa_status pa_prefill(void* out, const void* q, pa_dtype q_dtype,
+                     const void* k_pool, const void* v_pool, pa_dtype cache_dtype,
+                     const int32_t* block_tables, int32_t max_blocks_per_seq,
+                     const int32_t* context_lens, const int32_t* query_start,
+                     int32_t num_seqs, int32_t max_query_len, int32_t max_context_len,
+                     int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                     int32_t block_size, int32_t num_blocks, float scale,
+                     pa_stream_t stream);
+
+/*
  * pa_sync_status -- synchronise `stream`, then read and clear the device
  * error word of the current device.  Returns PA_OK, PA_ERR_DEVICE_BOUNDS,
  * PA_ERR_TIMEOUT or PA_ERR_CUDA (an asynchronous CUDA error).

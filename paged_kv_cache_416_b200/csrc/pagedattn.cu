@@ -11,6 +11,7 @@
 #include "cache_ops.cuh"
 #include "common.cuh"
 #include "decode.cuh"
+#include "prefill.cuh"
 
 namespace {
 
@@ -142,8 +143,10 @@ EncodeTiledFn encode_tiled_fn() {
 // D*e) bytes per swizzle row; one box = the bs token rows of one kv head of
 // one block, landing in shared memory as [half][token][R] with the R-byte
 // swizzle (128B or 64B).  Must match DecodeCfg / tile_off in decode.cuh.
+// With one_half the box is a single dim half (the prefill kernel places the
+// halves of consecutive blocks in separate K-major tiles).
 pa_status encode_pool_map(CUtensorMap* map, const void* pool, int32_t num_blocks, int32_t bs,
-                          int32_t hkv, int32_t head_dim, int32_t elem) {
+                          int32_t hkv, int32_t head_dim, int32_t elem, bool one_half = false) {
   EncodeTiledFn fn = encode_tiled_fn();
   if (fn == nullptr) return fail(PA_ERR_CUDA, "pa_decode: cuTensorMapEncodeTiled unavailable");
   const cuuint64_t row = static_cast<cuuint64_t>(head_dim) * elem;
@@ -153,7 +156,7 @@ pa_status encode_pool_map(CUtensorMap* map, const void* pool, int32_t num_blocks
                               static_cast<cuuint64_t>(num_blocks)};
   const cuuint64_t strides[4] = {hkv * row, R, row, static_cast<cuuint64_t>(bs) * hkv * row};
   const cuuint32_t box[5] = {static_cast<cuuint32_t>(R), static_cast<cuuint32_t>(bs),
-                             static_cast<cuuint32_t>(halves), 1, 1};
+                             static_cast<cuuint32_t>(one_half ? 1 : halves), 1, 1};
   const cuuint32_t estr[5] = {1, 1, 1, 1, 1};
   const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 5, const_cast<void*>(pool), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -445,6 +448,76 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_po
   if (s != PA_OK) return s;
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
+  return ok();
+}
+
+pa_status pa_prefill(void* out, const void* q, pa_dtype q_dtype, const void* k_pool,
+                     const void* v_pool, pa_dtype cache_dtype, const int32_t* block_tables,
+                     int32_t max_blocks_per_seq, const int32_t* context_lens,
+                     const int32_t* query_start, int32_t num_seqs, int32_t max_query_len,
+                     int32_t max_context_len, int32_t num_q_heads, int32_t num_kv_heads,
+                     int32_t head_dim, int32_t block_size, int32_t num_blocks, float scale,
+                     pa_stream_t stream) {
+  if (!valid_dtype(q_dtype) || !valid_dtype(cache_dtype) || q_dtype == PA_FP8_E4M3 ||
+      cache_dtype != q_dtype)
+    return fail(PA_ERR_DTYPE, "pa_prefill: q and the cache must share a 16-bit dtype");
+  if (head_dim != pa::kPfD || num_seqs < 0 || max_query_len < 0 || max_context_len < 0 ||
+      max_blocks_per_seq <= 0 || !cache_shape_ok(num_blocks, block_size, num_kv_heads, head_dim) ||
+      static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * block_size)
+    return fail(PA_ERR_SHAPE, "pa_prefill: unsupported sizes (head_dim must be %d)", pa::kPfD);
+  if (num_q_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
+      pa::kPfRows % (num_q_heads / num_kv_heads) != 0)
+    return fail(PA_ERR_HEADS, "pa_prefill: num_q_heads / num_kv_heads must divide %d", pa::kPfRows);
+  if (!std::isfinite(scale)) return fail(PA_ERR_SHAPE, "pa_prefill: scale must be finite");
+  if (num_seqs == 0 || max_query_len == 0) return ok();
+  if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens || !query_start)
+    return fail(PA_ERR_NULL, "pa_prefill: null pointer");
+  if ((reinterpret_cast<uintptr_t>(k_pool) | reinterpret_cast<uintptr_t>(v_pool) |
+       reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(out)) & 15)
+    return fail(PA_ERR_SHAPE, "pa_prefill: pools, q and out must be 16-byte aligned");
+  int dev;
+  if (current_device(&dev)) return fail(PA_ERR_CUDA, "pa_prefill: no current device");
+  pa::PrefillArgs a;
+  pa_status ms = encode_pool_map(&a.tmap_k, k_pool, num_blocks, block_size, num_kv_heads,
+                                 head_dim, 2, true);
+  if (ms == PA_OK)
+    ms = encode_pool_map(&a.tmap_v, v_pool, num_blocks, block_size, num_kv_heads, head_dim, 2, true);
+  if (ms != PA_OK) return ms;
+  a.out = out;
+  a.q = q;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.query_start = query_start;
+  a.hq = num_q_heads;
+  a.hkv = num_kv_heads;
+  a.group = num_q_heads / num_kv_heads;
+  a.max_blocks = max_blocks_per_seq;
+  a.num_blocks = num_blocks;
+  a.max_ctx = max_context_len;
+  a.sl2 = scale * 1.4426950408889634f;
+  const int T = pa::kPfRows / a.group;
+  dim3 grid(static_cast<unsigned>(cdiv(max_query_len, T)), static_cast<unsigned>(num_kv_heads),
+            static_cast<unsigned>(num_seqs));
+  if (grid.y > 65535 || grid.z > 65535)
+    return fail(PA_ERR_SHAPE, "pa_prefill: too many kv heads or sequences for one launch");
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  auto launch = [&](auto kern, int smem_bytes) -> pa_status {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill)");
+    kern<<<grid, pa::kPfThreads, smem_bytes, st>>>(a);
+    return PA_OK;
+  };
+  pa_status ls;
+  const bool bf = q_dtype == PA_BF16;
+  if (block_size == 16)
+    ls = bf ? launch(pa::prefill_kernel<true, 16>, pa::PrefillCfg<16>::kSmemBytes)
+            : launch(pa::prefill_kernel<false, 16>, pa::PrefillCfg<16>::kSmemBytes);
+  else
+    ls = bf ? launch(pa::prefill_kernel<true, 32>, pa::PrefillCfg<32>::kSmemBytes)
+            : launch(pa::prefill_kernel<false, 32>, pa::PrefillCfg<32>::kSmemBytes);
+  if (ls != PA_OK) return ls;
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pa_prefill launch");
   return ok();
 }
 

@@ -47,6 +47,8 @@ def declare(lib: ctypes.CDLL) -> ctypes.CDLL:
         "pa_copy_blocks": (I32, [P, P, I32, I32, I32, I32, I32, P, I32, P]),
         "pa_swap_blocks": (I32, [P, P, I32, P, P, I32, I32, I32, I32, I32, P, I32, P]),
         "pa_hash_blocks": (I32, [P, I64, P, I32, I32, P, I32, P]),
+        "pa_prefill": (I32, [P, P, I32, P, P, I32, P, I32, P, P, I32, I32, I32, I32, I32, I32,
+                             I32, I32, F, P]),
         "pa_decode_split_tokens": (I32, [I32, I32, I32, I32, I32]),
         "pa_decode_workspace_size": (SZ, [I32, I32, I32, I32, I32, I32, I32]),
         "pa_decode": (I32, [P, P, I32, P, P, I32, P, I32, P, I32, I32, I32, I32, I32, I32, I32,
@@ -81,6 +83,7 @@ pa_write_kv = _lib.pa_write_kv
 pa_copy_blocks = _lib.pa_copy_blocks
 pa_swap_blocks = _lib.pa_swap_blocks
 pa_hash_blocks = _lib.pa_hash_blocks
+pa_prefill = _lib.pa_prefill
 pa_decode_split_tokens = _lib.pa_decode_split_tokens
 pa_decode_workspace_size = _lib.pa_decode_workspace_size
 pa_decode = _lib.pa_decode
@@ -96,7 +99,7 @@ NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 ENTRY_POINTS = [
     "pa_write_kv", "pa_copy_blocks", "pa_swap_blocks", "pa_hash_blocks", "pa_decode_split_tokens", "pa_decode_workspace_size",
-    "pa_decode", "pa_sync_status", "pa_last_error", "pa_validate_slot_mapping",
+    "pa_decode", "pa_prefill", "pa_sync_status", "pa_last_error", "pa_validate_slot_mapping",
     "pa_validate_copy_pairs", "pa_validate_block_tables", "pa_decode_noalloc",
 ]
 
@@ -233,6 +236,26 @@ def decode(q, k_pool, v_pool, block_tables, context_lens, scale: float, max_cont
                     int(max_context_len), B, hq, hkv, d, bs, N, float(scale), float(k_scale),
                     float(v_scale), int(split_tokens), _ptr(workspace), workspace.numel(),
                     _stream(stream)))
+    return out
+
+
+def prefill(q, k_pool, v_pool, block_tables, context_lens, query_start, scale: float,
+            max_query_len: int, max_context_len: int, out=None, stream=None) -> torch.Tensor:
+    """pa_prefill on tensors.  q [total_q, Hq, D] packed by query_start
+    (int32 [B + 1]); pools [N, bs, Hkv, D]; block_tables int32 [B, W];
+    context_lens int32 [B].  Returns out [total_q, Hq, D]."""
+    _contig(q, k_pool, v_pool, block_tables, context_lens, query_start)
+    for t in (block_tables, context_lens, query_start):
+        if t.dtype != torch.int32:
+            raise TypeError("block_tables, context_lens and query_start must be int32")
+    total, hq, d = q.shape
+    N, bs, hkv, _ = k_pool.shape
+    if out is None:
+        out = torch.empty_like(q)
+    check(pa_prefill(_ptr(out), _ptr(q), _dtype(q), _ptr(k_pool), _ptr(v_pool), _dtype(k_pool),
+                     _ptr(block_tables), block_tables.shape[1], _ptr(context_lens),
+                     _ptr(query_start), context_lens.shape[0], int(max_query_len),
+                     int(max_context_len), hq, hkv, d, bs, N, float(scale), _stream(stream)))
     return out
 
 

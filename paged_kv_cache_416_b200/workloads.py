@@ -334,6 +334,42 @@ def shared_prefix_tails(seed=4, device="cpu", **kw) -> Workload:
     return _shared_prefix("tails", seed, device, **kw)
 
 
+@dataclass
+class PrefillWorkload:
+    """Chunked prefill: sequence s has context_lens[s] cached tokens, of which
+    the last query_start[s+1] - query_start[s] are the new query tokens."""
+    base: Workload                    # pools, tables, lengths (its q/new_k unused)
+    q: torch.Tensor                   # [total_q, Hq, D]
+    query_start: np.ndarray           # int32 [B + 1]
+
+    @property
+    def max_query_len(self) -> int:
+        return int(np.diff(self.query_start).max()) if len(self.query_start) > 1 else 0
+
+    @property
+    def flops(self) -> int:
+        """Causal attention flops: 4 * D * Hq * sum over new tokens of the keys each sees."""
+        b = self.base
+        tot = 0
+        for s in range(b.num_seqs):
+            n = int(self.query_start[s + 1] - self.query_start[s])
+            c = int(b.context_lens[s])
+            tot += n * (c - n) + n * (n + 1) // 2
+        return 4 * b.head_dim * b.num_q_heads * tot
+
+
+def prefill(seed=6, device="cpu", ctxs=(200, 300, 1, 77), nqs=(200, 77, 1, 50), hq=32, hkv=8,
+            d=128, bs=16, dtype="bf16", **kw) -> PrefillWorkload:
+    """Paged prefill inputs: the cache holds every token (the new ones
+    included, as pa_write_kv leaves it); q holds the new tokens, packed."""
+    assert all(n <= c for n, c in zip(nqs, ctxs))
+    base = _generic("prefill", list(ctxs), hq, hkv, d, bs, dtype, dtype, seed, device, **kw)
+    qs = np.concatenate([[0], np.cumsum(nqs)]).astype(np.int32)
+    gen = torch.Generator(device=device).manual_seed(int(seed) + 77)
+    q = _to_storage(_randn((int(qs[-1]), hq, d), gen, device), dtype)
+    return PrefillWorkload(base=base, q=q, query_start=qs)
+
+
 REGISTRY = {
     "tiny": tiny,
     "llama13b_mha": llama13b_mha,
