@@ -57,7 +57,7 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling only)")
-    ap.add_argument("--op", choices=["decode", "swap", "hash"], default="decode",
+    ap.add_argument("--op", choices=["decode", "swap", "hash", "prefill"], default="decode",
                     help="decode: the decode step (the headline line); the others time "
                          "one companion operation on one GPU and print its own line")
     return ap.parse_args(argv)
@@ -585,6 +585,50 @@ def run_hash(args):
     }
 
 
+def run_prefill(args):
+    """pa_prefill: full prefill of 8 sequences x 4096 tokens on the
+    Llama-3-70B-shaped layer (64/8 heads, D 128, bf16, bs 16), causal.
+    Roofline: tensor -- causal attention flops (4 * D * Hq * sum of keys seen
+    per query) against the measured dense bf16 peak."""
+    import torch
+    from paged_kv_cache_416_b200 import build as _build
+    _build.build()
+    from paged_kv_cache_416_b200 import pagedattn as pa
+    from paged_kv_cache_416_b200 import workloads as W
+    torch.cuda.set_device(0)
+    n = 4096
+    pw = W.prefill(seed=args.seed, device="cuda", ctxs=(n,) * 8, nqs=(n,) * 8, hq=64, hkv=8,
+                   bs=16, dtype="bf16")
+    b = pw.base
+    q = pw.q
+    bt = torch.from_numpy(b.block_tables).cuda()
+    cl = torch.from_numpy(b.context_lens).cuda()
+    qs = torch.from_numpy(pw.query_start).cuda()
+    out = torch.empty_like(q)
+    iters = max(3, min(args.steps, 20))
+    t = _events_time(lambda: pa.prefill(q, b.k_pool, b.v_pool, bt, cl, qs, b.scale,
+                                        pw.max_query_len, b.max_context_len, out=out), iters)
+    pa.sync_status()
+    tflops = pw.flops / t / 1e12
+    peak = None
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        peak = float(json.load(open(p))["bf16_tflops"])
+    peak = peak or 1590.0
+    return {
+        "metric": "paged prefill attention TFLOP/s (causal)", "op": "prefill",
+        "value": round(tflops, 2), "unit": "TFLOP/s", "n_gpus": 1, "steps": iters,
+        "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "8 sequences x 4096 new tokens, 64/8 heads, D 128, bf16, bs 16",
+                   "flops_per_call": pw.flops},
+        "ms_per_call": round(t * 1e3, 3),
+        "roofline": {"bound": "tensor", "achieved": round(tflops, 2), "peak": peak,
+                     "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
+                     "peak_kind": "measured dense bf16 (burst)"},
+        "gpu_launches": iters,
+    }
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.warmup < 3:
@@ -602,7 +646,7 @@ def main(argv=None):
     if args.op != "decode":
         if rank != 0:
             return 0
-        line = {"swap": run_swap, "hash": run_hash}[args.op](args)
+        line = {"swap": run_swap, "hash": run_hash, "prefill": run_prefill}[args.op](args)
         print(json.dumps(line), flush=True)
         return 0
     import torch

@@ -485,12 +485,24 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
         }
 
         // ---- P^T as the B operand: transpose the 8x8 (token, head) tiles
+        // With a bf16 cache, P = P_hi + P_lo in bf16: one bf16 value keeps 8
+        // significant bits (error up to 2^-9 of each weight), which outputs
+        // formed by cancellation cannot absorb; fp16 P keeps 11 and stays one.
         uint32_t pb[C::kTokTiles][2];
+        uint32_t pl[C::kTokTiles][2];
         constexpr bool kPBF16 = (CK == kCacheBF16);
 #pragma unroll
         for (int mt = 0; mt < C::kTokTiles; ++mt) {
-          pb[mt][0] = movmatrix_trans(pack2<kPBF16>(s[mt][0], s[mt][1]));
-          pb[mt][1] = movmatrix_trans(pack2<kPBF16>(s[mt][2], s[mt][3]));
+          const uint32_t h0 = pack2<kPBF16>(s[mt][0], s[mt][1]);
+          const uint32_t h1 = pack2<kPBF16>(s[mt][2], s[mt][3]);
+          pb[mt][0] = movmatrix_trans(h0);
+          pb[mt][1] = movmatrix_trans(h1);
+          if constexpr (kPBF16) {
+            pl[mt][0] = movmatrix_trans(pack_bf16x2(s[mt][0] - to_float<true>(h0 & 0xffff),
+                                                    s[mt][1] - to_float<true>(h0 >> 16)));
+            pl[mt][1] = movmatrix_trans(pack_bf16x2(s[mt][2] - to_float<true>(h1 & 0xffff),
+                                                    s[mt][3] - to_float<true>(h1 >> 16)));
+          }
         }
 
         // ---- O^T += V^T P^T  (rows: dims, cols: packed heads).  In a partial
@@ -530,6 +542,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
                             af[2], af[3]);
               af[0] &= m_lo; af[1] &= m_lo; af[2] &= m_hi; af[3] &= m_hi;
               mma_16816<kMmaBF16>(acc[dt], af, pb[mt][0], pb[mt][1]);
+              if constexpr (kPBF16) mma_16816<kMmaBF16>(acc[dt], af, pl[mt][0], pl[mt][1]);
             }
           }
         }

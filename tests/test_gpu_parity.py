@@ -340,3 +340,16 @@ def test_full_size_workloads_against_oracle(pa, name):
                   {int(np.argmax(w.context_lens))})
     ref = compact_oracle_step(w, seqs)
     assert_attention_close(as_f64(out)[seqs], ref, f"{name} full size")
+
+
+@pytest.mark.parametrize("cache", ["bf16", "e4m3"])
+def test_decode_short_contexts_many_sequences(pa, cache):
+    """2-8 keys per sequence concentrate the softmax weights, so outputs are
+    formed by cancellation between O(1) terms and rounding of the weights
+    shows directly; 1024 sequences x 64 heads give many chances to."""
+    rng = np.random.default_rng(41)
+    lens = rng.integers(2, 9, size=1024)
+    w = W._generic("short", lens, 64, 8, 128, 16, "bf16", cache, seed=41, device="cpu")
+    out, _, _ = gpu_step(pa, w)
+    ref, _, _ = oracle_step(w)
+    assert_attention_close(as_f64(out), ref, f"short contexts {cache}")
