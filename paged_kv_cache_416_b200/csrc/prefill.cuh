@@ -14,7 +14,8 @@
 //   CTA   = 4 warps, one (sequence, kv head, 128 query rows) tile; query row
 //           r = (token r / G, head r % G) lives in TMEM lane r and is owned by
 //           thread r for the softmax
-//   per 64-key tile (two TMA stages of K and V, one box per (block, half)):
+//   per 64-key tile (K and V by TMA, one box per (block, dim half); the next
+//   tile's loads are issued as soon as this tile's K and V are consumed):
 //     S[128 x 64]   = Q[128 x 128] K^T          tcgen05.mma M128 N64, K 8 x 16
 //     Vt[128 x 64]  = V^T (warps transpose V in shared memory meanwhile)
 //     softmax       thread r: tcgen05.ld of its S row, causal mask, online
@@ -49,13 +50,13 @@ struct PrefillCfg {
   static constexpr int kPBytes = kPfRows * kPfKeys * 2;   // [128 rows][64 keys = 128 B]
   static constexpr int kBlocksPerTile = kPfKeys / BS;
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kQBytes;           // 2 stages
-  static constexpr int kOffV = kOffK + 2 * kKBytes;       // 2 stages
-  static constexpr int kOffVt = kOffV + 2 * kKBytes;
+  static constexpr int kOffK = kOffQ + kQBytes;
+  static constexpr int kOffV = kOffK + kKBytes;
+  static constexpr int kOffVt = kOffV + kKBytes;
   static constexpr int kOffP = kOffVt + kVtBytes;         // P_hi, then P_lo
-  static constexpr int kTiles = kOffP + 2 * kPBytes;
-  static constexpr int kHead = 256;                       // mbarriers, TMEM slot, masks
-  static constexpr int kSmemBytes = kHead + 1024 + kTiles;
+  static constexpr int kTiles = kOffP + 2 * kPBytes;      // 112 KiB: two CTAs per SM
+  static constexpr int kHead = 256;                       // mbarriers, TMEM slot, mask
+  static constexpr int kSmemBytes = kTiles + kHead;
   static_assert(kPfKeys % BS == 0, "a key tile holds whole blocks");
 };
 
@@ -81,9 +82,9 @@ __device__ __forceinline__ uint32_t swz128(int r, int c) {
 // One CTA per (query tile, kv head, sequence): grid (ceil(max_query_len / T),
 // Hkv, B) with T = 128 / G tokens; CTAs past a sequence's new tokens exit.
 template <bool kBF16, int BS>
-__global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_constant__ PrefillArgs a) {
+__global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_constant__ PrefillArgs a) {
   using C = PrefillCfg<BS>;
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ __align__(1024) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int s = blockIdx.z, kvh = blockIdx.y;
   const int G = a.group;
@@ -110,18 +111,22 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_con
   const int nkt = (ctx - n + i0 + nt - 1) / kPfKeys + 1;  // key tiles up to the last row
   const int32_t* table = a.block_tables + static_cast<int64_t>(s) * a.max_blocks;
 
-  // [mbarriers: full[2], S done, O done | TMEM slot | bad-block masks | pad | tiles]
-  const uint32_t smem_s = smem_addr(smem);
-  const uint32_t full0 = smem_s, bar_s = smem_s + 16, bar_o = smem_s + 24;
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + 32);
-  volatile int* bad_mask = reinterpret_cast<volatile int*>(smem + 64);
-  const uint32_t base_s = (smem_s + C::kHead + 1023) & ~1023u;
-  uint8_t* const base = smem + (base_s - smem_s);
-  const uint32_t sQ = base_s + C::kOffQ, sVt = base_s + C::kOffVt, sP = base_s + C::kOffP;
+  // [tiles (1024-aligned) | mbarriers: full, S done, O done | TMEM slot | bad-block mask]
+  const uint32_t base_s = smem_addr(smem);
+  uint8_t* const base = smem;
+  const uint32_t head_s = base_s + C::kTiles;
+  const uint32_t full = head_s, bar_s = head_s + 8, bar_o = head_s + 16;
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(base + C::kTiles + 32);
+  volatile int* bad_mask = reinterpret_cast<volatile int*>(base + C::kTiles + 64);
+  const uint32_t sQ = base_s + C::kOffQ, sK = base_s + C::kOffK, sV = base_s + C::kOffV;
+  const uint32_t sVt = base_s + C::kOffVt, sP = base_s + C::kOffP;
+  if (base_s & 1023) {  // the swizzled tiles need a 1024-byte aligned start
+    if (tid == 0) record_error(PA_ERR_DEVICE_BOUNDS);
+    return;
+  }
 
   if (tid == 0) {
-    mbar_init(full0, 1);
-    mbar_init(full0 + 8, 1);
+    mbar_init(full, 1);
     mbar_init(bar_s, 1);
     mbar_init(bar_o, 1);
     mbar_init_fence();
@@ -129,7 +134,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_con
     prefetch_tensormap(&a.tmap_v);
   }
   if (warp == 0) {
-    tmem_alloc(smem_s + 32, kPfTmemCols);
+    tmem_alloc(head_s + 32, kPfTmemCols);
     tmem_relinquish();
   }
 
@@ -145,14 +150,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_con
   }
   fence_proxy_async_smem();
 
-  // thread 0: TMA loads of key tile kt into stage kt & 1 (one box per block
-  // and dim half; blocks past the context, or with a bad table entry, are
-  // not loaded and their keys are masked)
+  // thread 0: TMA loads of key tile kt (one box per block and dim half;
+  // blocks past the context, or with a bad table entry, are not loaded and
+  // their keys are masked)
   auto issue_tile = [&](int kt) {
-    const int st = kt & 1;
-    const uint32_t bar = full0 + 8 * st;
-    const uint32_t sK = base_s + C::kOffK + st * C::kKBytes;
-    const uint32_t sV = base_s + C::kOffV + st * C::kKBytes;
     int phys[C::kBlocksPerTile];
     int bad = 0;
     uint32_t bytes = 0;
@@ -171,25 +172,22 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_con
         }
       }
     }
-    bad_mask[st] = bad;
-    mbar_arrive_expect_tx(bar, bytes);
+    *bad_mask = bad;
+    mbar_arrive_expect_tx(full, bytes);
 #pragma unroll
     for (int b = 0; b < C::kBlocksPerTile; ++b) {
       if (phys[b] < 0) continue;
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const uint32_t off = hf * (kPfKeys * 128) + b * BS * 128;
-        tma_load_5d(sK + off, &a.tmap_k, 0, 0, hf, kvh, phys[b], bar);
-        tma_load_5d(sV + off, &a.tmap_v, 0, 0, hf, kvh, phys[b], bar);
+        tma_load_5d(sK + off, &a.tmap_k, 0, 0, hf, kvh, phys[b], full);
+        tma_load_5d(sV + off, &a.tmap_v, 0, 0, hf, kvh, phys[b], full);
       }
     }
   };
-  if (tid == 0) {
-    issue_tile(0);
-    if (nkt > 1) issue_tile(1);
-  }
+  if (tid == 0) issue_tile(0);
   tc_fence_before_sync();
-  __syncthreads();  // Q tile, barriers, TMEM address, masks of tiles 0 and 1
+  __syncthreads();  // Q tile, barriers, TMEM address
   tc_fence_after_sync();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem, tO = tmem + 128;
@@ -204,13 +202,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_con
   bool failed = false;
 
   for (int kt = 0; kt < nkt; ++kt) {
-    const int st = kt & 1;
-    const uint32_t sK = base_s + C::kOffK + st * C::kKBytes;
-    const uint32_t sV = base_s + C::kOffV + st * C::kKBytes;
-    if (!failed && !mbar_wait_bounded(full0 + 8 * st, (kt >> 1) & 1)) {
+    if (!failed && !mbar_wait_bounded(full, kt & 1)) {
       failed = true;
       record_error(PA_ERR_TIMEOUT);
     }
+    const int bad = *bad_mask;
     // ---- S = Q K^T (one thread issues; 8 MMAs of K = 16 along head_dim)
     if (tid == 0 && !failed) {
       tc_fence_after_sync();
@@ -223,7 +219,6 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_con
     }
     // ---- meanwhile Vt = V^T: 8x8 tiles read with ldmatrix, stored transposed;
     // keys the tile must not use (past the context, bad block) are zeroed
-    const int bad = bad_mask[st];
     if (!failed) {
       const int dg = warp * 4 + (lane >> 3);  // 8-dim group this lane addresses
 #pragma unroll
@@ -283,9 +278,9 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_con
     }
     fence_proxy_async_smem();
     tc_fence_before_sync();
-    __syncthreads();  // P and Vt complete, S read
-    // ---- O tile = P Vt^T (4 MMAs of K = 16 along the keys)
+    __syncthreads();  // P and Vt complete; S, K and V no longer read
     if (tid == 0 && !failed) {
+      // ---- O tile = (P_hi + P_lo) Vt^T (2 x 4 MMAs of K = 16 along the keys)
       tc_fence_after_sync();
 #pragma unroll
       for (int k = 0; k < kPfKeys / 16; ++k)
@@ -296,6 +291,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_con
         umma_f16(tO, umma_desc_k128(sP + C::kPBytes + k * 32), umma_desc_k128(sVt + k * 32),
                  kIdescO, 1u);
       umma_commit(bar_o);
+      // the next key tile's loads overlap this product and the O update
+      if (kt + 1 < nkt) issue_tile(kt + 1);
     }
     if (!failed && !mbar_wait_bounded(bar_o, kt & 1)) {
       failed = true;
@@ -311,8 +308,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) prefill_kernel(const __grid_con
       for (int j = 0; j < 32; ++j) o[32 * c + j] = o[32 * c + j] * alpha + __uint_as_float(ot[j]);
     }
     tc_fence_before_sync();
-    __syncthreads();  // stage st, S and the O tile are free
-    if (tid == 0 && !failed && kt + 2 < nkt) issue_tile(kt + 2);
+    __syncthreads();  // S, the O tile, P and Vt are free again
   }
 
   if (row_ok) {
