@@ -11,20 +11,35 @@
 // dense contraction (128 query rows x 64 keys x 128 dims per tile pair), so
 // both products run on tcgen05.mma:
 //
-//   CTA   = 4 warps, one (sequence, kv head, 128 query rows) tile; query row
-//           r = (token r / G, head r % G) lives in TMEM lane r and is owned by
-//           thread r for the softmax
-//   per 64-key tile (K and V by TMA, one box per (block, dim half); the next
-//   tile's loads are issued as soon as this tile's K and V are consumed):
-//     S[128 x 64]   = Q[128 x 128] K^T          tcgen05.mma M128 N64, K 8 x 16
-//     Vt[128 x 64]  = V^T (warps transpose V in shared memory meanwhile)
-//     softmax       thread r: tcgen05.ld of its S row, causal mask, online
-//                   max / sum, P row -> P_hi + P_lo (two 16-bit tiles,
-//                   128B-swizzled) so P keeps ~16 significant bits
-//     Otile[128x128]= (P_hi + P_lo) Vt^T        tcgen05.mma M128 N128, K 2 x 4 x 16
-//     O (registers) = O * alpha + Otile          tcgen05.ld of the O row
+//   CTA   = 5 warps on one (sequence, kv head, 128 query rows) tile.  Warps
+//           0-3 own the rows: query row r = (token r / G, head r % G) lives
+//           in TMEM lane r and thread r runs its softmax.  Warp 4 is the
+//           producer: TMA loads, the MMA issue (one lane), and the zeroing of
+//           values that must not reach O.  The two sides hand over through
+//           mbarriers only (S done, S read, P ready, O done), never a
+//           CTA-wide barrier inside the key loop.
+//   TMEM  = S [0, 64) | P_hi [64, 96) | P_lo [96, 128) | O [128, 256) (fp32
+//           S and O; P two 16-bit values per column)
+//   per 64-key tile kt (K and V by TMA into two stages each, one box per
+//   (block, dim half); K(kt+2) is loaded once S(kt) has been read, V(kt+1)
+//   once O(kt-1) is done):
+//     S            = Q K^T      tcgen05.mma, A = Q and B = K from shared memory
+//                               (K-major), M128 N64, 8 x K16; S(kt+1) is
+//                               issued as soon as the rows have read S(kt),
+//                               so it runs under the softmax of tile kt
+//     softmax      thread r: tcgen05.ld of its S row, causal and block masks
+//                  (only on tiles that need them), online max / sum in packed
+//                  fp32 pairs; P = P_hi + P_lo (two 16-bit parts, so P keeps
+//                  ~16 significant bits) by tcgen05.st into TMEM
+//     O           += P V        tcgen05.mma, A = P from TMEM, B = V from shared
+//                               memory read MN-major (no transpose), M128 N128,
+//                               2 x 4 x K16, accumulated in TMEM across tiles
+//   O is rescaled (tcgen05.ld, multiply, tcgen05.st) only when a row's
+//   running max grows by more than 8 in log2 units; otherwise the weights
+//   keep the stale max (they stay below 2^8) and the sum follows it, so the
+//   normalised result is the same.
 //
-// Every operand tile is K-major with the 128-byte swizzle, rows of 128
+// Every shared-memory operand tile uses the 128-byte swizzle, rows of 128
 // bytes, 8-row groups 1024 bytes apart.  Every wait is bounded.
 #pragma once
 
@@ -36,26 +51,24 @@
 
 namespace pa {
 
-constexpr int kPfThreads = 128;   // 4 warps; thread r owns query row r (TMEM lane r)
+constexpr int kPfRowThreads = 128;  // warps 0-3: thread r owns query row r (TMEM lane r)
+constexpr int kPfThreads = 160;     // + warp 4: loads and MMA issue
 constexpr int kPfRows = 128;      // MMA M: (token, head) rows per CTA
 constexpr int kPfKeys = 64;       // keys per tile
 constexpr int kPfD = 128;         // head_dim
-constexpr int kPfTmemCols = 256;  // S in [0, 64), O tile in [128, 256)
+constexpr int kPfTmemCols = 256;  // S [0, 64), P_hi [64, 96), P_lo [96, 128), O [128, 256)
+constexpr float kPfRescaleLog2 = 8.f;  // rescale O when the max grows by more than this
 
 template <int BS>
 struct PrefillCfg {
   static constexpr int kQBytes = kPfRows * kPfD * 2;      // [2 dim halves][128 rows][128 B]
   static constexpr int kKBytes = kPfKeys * kPfD * 2;      // [2 dim halves][64 keys][128 B]
-  static constexpr int kVtBytes = kPfD * kPfKeys * 2;     // [128 dims][64 keys = 128 B]
-  static constexpr int kPBytes = kPfRows * kPfKeys * 2;   // [128 rows][64 keys = 128 B]
   static constexpr int kBlocksPerTile = kPfKeys / BS;
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + kQBytes;
-  static constexpr int kOffV = kOffK + kKBytes;
-  static constexpr int kOffVt = kOffV + kKBytes;
-  static constexpr int kOffP = kOffVt + kVtBytes;         // P_hi, then P_lo
-  static constexpr int kTiles = kOffP + 2 * kPBytes;      // 112 KiB: two CTAs per SM
-  static constexpr int kHead = 256;                       // mbarriers, TMEM slot, mask
+  static constexpr int kOffK = kOffQ + kQBytes;           // 2 stages
+  static constexpr int kOffV = kOffK + 2 * kKBytes;       // 2 stages
+  static constexpr int kTiles = kOffV + 2 * kKBytes;      // 96 KiB: two CTAs per SM
+  static constexpr int kHead = 256;                       // 8 mbarriers, TMEM slot
   static constexpr int kSmemBytes = kTiles + kHead;
   static_assert(kPfKeys % BS == 0, "a key tile holds whole blocks");
 };
@@ -84,8 +97,9 @@ __device__ __forceinline__ uint32_t swz128(int r, int c) {
 template <bool kBF16, int BS>
 __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_constant__ PrefillArgs a) {
   using C = PrefillCfg<BS>;
-  extern __shared__ __align__(1024) uint8_t smem[];
+  extern __shared__ __align__(1024) uint8_t pf_smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool producer = warp == kPfRowThreads / 32;
   const int s = blockIdx.z, kvh = blockIdx.y;
   const int G = a.group;
   const int T = kPfRows / G;  // query tokens per CTA
@@ -94,233 +108,304 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
   const int i0 = blockIdx.x * T;
   if (n <= 0 || i0 >= n) return;  // the whole CTA, before any TMEM use
   const int nt = min(T, n - i0);
-  const int r = tid;                          // this thread's query row
+  const int r = tid;                          // row of a row thread
   const int tok = r / G;
   const int hr = kvh * G + r % G;             // its query head
-  const bool row_ok = tok < nt;
+  const bool row_ok = !producer && tok < nt;
   const int ctx = a.context_lens[s];
-  uint4* const orow = reinterpret_cast<uint4*>(a.out) +
-                      (static_cast<int64_t>(q0 + i0 + tok) * a.hq + hr) * (kPfD * 2 / 16);
+  const int64_t orow_off = (static_cast<int64_t>(q0 + i0 + tok) * a.hq + hr) * (kPfD * 2 / 16);
   if (ctx < n || ctx > a.max_ctx || ctx > a.max_blocks * BS) {
     if (tid == 0) record_error(PA_ERR_DEVICE_BOUNDS);
     if (row_ok)
-      for (int j = 0; j < kPfD * 2 / 16; ++j) orow[j] = make_uint4(0, 0, 0, 0);
+      for (int j = 0; j < kPfD * 2 / 16; ++j)
+        reinterpret_cast<uint4*>(a.out)[orow_off + j] = make_uint4(0, 0, 0, 0);
     return;
   }
-  const int qpos = ctx - n + i0 + tok;        // this row's position in the sequence
-  const int nkt = (ctx - n + i0 + nt - 1) / kPfKeys + 1;  // key tiles up to the last row
+  const int qfirst = ctx - n + i0;            // position of the CTA's first token
+  const int qpos = qfirst + tok;              // this row's position
+  const int kend = qfirst + nt;               // keys the CTA's rows see: [0, kend)
+  const int nkt = (kend - 1) / kPfKeys + 1;
   const int32_t* table = a.block_tables + static_cast<int64_t>(s) * a.max_blocks;
 
-  // [tiles (1024-aligned) | mbarriers: full, S done, O done | TMEM slot | bad-block mask]
-  const uint32_t base_s = smem_addr(smem);
-  uint8_t* const base = smem;
+  // [tiles (1024-aligned) | mbarriers | TMEM slot]
+  const uint32_t base_s = smem_addr(pf_smem);
+  uint8_t* const base = pf_smem;
   const uint32_t head_s = base_s + C::kTiles;
-  const uint32_t full = head_s, bar_s = head_s + 8, bar_o = head_s + 16;
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(base + C::kTiles + 32);
-  volatile int* bad_mask = reinterpret_cast<volatile int*>(base + C::kTiles + 64);
+  const uint32_t full_k = head_s, full_v = head_s + 16;  // + 8 * stage, TMA
+  const uint32_t bar_s = head_s + 32, bar_o = head_s + 40;  // MMA commits
+  const uint32_t s_free = head_s + 48, p_ready = head_s + 56;  // one arrival per row warp
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(base + C::kTiles + 64);
   const uint32_t sQ = base_s + C::kOffQ, sK = base_s + C::kOffK, sV = base_s + C::kOffV;
-  const uint32_t sVt = base_s + C::kOffVt, sP = base_s + C::kOffP;
   if (base_s & 1023) {  // the swizzled tiles need a 1024-byte aligned start
     if (tid == 0) record_error(PA_ERR_DEVICE_BOUNDS);
     return;
   }
 
-  if (tid == 0) {
-    mbar_init(full, 1);
-    mbar_init(bar_s, 1);
-    mbar_init(bar_o, 1);
+  // physical block of slot b of key tile kt: -1 past the context, -2 for a
+  // bad table entry (its keys are masked and its values zeroed)
+  auto tile_block = [&](int kt, int b) -> int {
+    const int j = kt * C::kBlocksPerTile + b;
+    if (j * BS >= ctx) return -1;
+    const int p = table[j];
+    return (p >= 0 && p < a.num_blocks) ? p : -2;
+  };
+  // producer lane 0: TMA loads of one K or V tile into its stage (one box
+  // per block and dim half); blocks past the context or with a bad entry are
+  // not loaded
+  auto issue_tile = [&](int kt, bool is_v) {
+    const int st = kt & 1;
+    int phys[C::kBlocksPerTile];
+    uint32_t bytes = 0;
+#pragma unroll
+    for (int b = 0; b < C::kBlocksPerTile; ++b) {
+      phys[b] = tile_block(kt, b);
+      if (phys[b] >= 0) bytes += 2u * BS * 128u;
+    }
+    const uint32_t bar = (is_v ? full_v : full_k) + 8 * st;
+    const uint32_t dst = (is_v ? sV : sK) + st * C::kKBytes;
+    const CUtensorMap* map = is_v ? &a.tmap_v : &a.tmap_k;
+    mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+    for (int b = 0; b < C::kBlocksPerTile; ++b) {
+      if (phys[b] < 0) continue;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf)
+        tma_load_5d(dst + hf * (kPfKeys * 128) + b * BS * 128, map, 0, 0, hf, kvh, phys[b], bar);
+    }
+  };
+
+  if (producer && lane == 0) {
+    for (int i = 0; i < 6; ++i) mbar_init(head_s + 8 * i, 1);
+    mbar_init(s_free, kPfRowThreads / 32);
+    mbar_init(p_ready, kPfRowThreads / 32);
     mbar_init_fence();
     prefetch_tensormap(&a.tmap_k);
     prefetch_tensormap(&a.tmap_v);
+    for (int kt = 0; kt < 2 && kt < nkt; ++kt) {
+      issue_tile(kt, false);
+      issue_tile(kt, true);
+    }
   }
   if (warp == 0) {
-    tmem_alloc(head_s + 32, kPfTmemCols);
+    tmem_alloc(head_s + 64, kPfTmemCols);
     tmem_relinquish();
   }
-
-  // Q tile: thread r writes its row (256 B) into the two dim halves
-  {
-    const uint4* src = reinterpret_cast<const uint4*>(a.q) +
-                       (static_cast<int64_t>(q0 + i0 + tok) * a.hq + hr) * (kPfD * 2 / 16);
+  if (!producer) {  // Q tile: thread r writes its row (256 B) into the two dim halves
+    const uint4* src = reinterpret_cast<const uint4*>(a.q) + orow_off;
 #pragma unroll
     for (int j = 0; j < 16; ++j) {
       const uint4 v = row_ok ? src[j] : make_uint4(0, 0, 0, 0);
       *reinterpret_cast<uint4*>(base + C::kOffQ + (j >> 3) * (kPfRows * 128) + swz128(r, j & 7)) = v;
     }
+    fence_proxy_async_smem();
   }
-  fence_proxy_async_smem();
-
-  // thread 0: TMA loads of key tile kt (one box per block and dim half;
-  // blocks past the context, or with a bad table entry, are not loaded and
-  // their keys are masked)
-  auto issue_tile = [&](int kt) {
-    int phys[C::kBlocksPerTile];
-    int bad = 0;
-    uint32_t bytes = 0;
-#pragma unroll
-    for (int b = 0; b < C::kBlocksPerTile; ++b) {
-      const int j = kt * C::kBlocksPerTile + b;
-      phys[b] = -1;
-      if (j * BS < ctx) {
-        const int p = table[j];
-        if (p >= 0 && p < a.num_blocks) {
-          phys[b] = p;
-          bytes += 4u * BS * 128u;  // K and V, two halves each
-        } else {
-          bad |= 1 << b;
-          record_error(PA_ERR_DEVICE_BOUNDS);
-        }
-      }
-    }
-    *bad_mask = bad;
-    mbar_arrive_expect_tx(full, bytes);
-#pragma unroll
-    for (int b = 0; b < C::kBlocksPerTile; ++b) {
-      if (phys[b] < 0) continue;
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const uint32_t off = hf * (kPfKeys * 128) + b * BS * 128;
-        tma_load_5d(sK + off, &a.tmap_k, 0, 0, hf, kvh, phys[b], full);
-        tma_load_5d(sV + off, &a.tmap_v, 0, 0, hf, kvh, phys[b], full);
-      }
-    }
-  };
-  if (tid == 0) issue_tile(0);
+  // any bad table entry among the blocks this CTA reads?  (then every tile
+  // takes the masked path; otherwise only the tiles that cross the diagonal
+  // or the end of the context)
+  int my_bad = 0;
+  for (int j = tid; j * BS < kend; j += kPfThreads) {
+    const int p = table[j];
+    my_bad |= (p < 0 || p >= a.num_blocks);
+  }
   tc_fence_before_sync();
-  __syncthreads();  // Q tile, barriers, TMEM address
+  const bool any_bad = __syncthreads_or(my_bad) != 0;  // + Q tile, barriers, TMEM address
   tc_fence_after_sync();
+  if (any_bad && tid == 0) record_error(PA_ERR_DEVICE_BOUNDS);
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tO = tmem + 128;
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;  // the warp's TMEM lanes
-  constexpr uint32_t kIdescS = umma_idesc_f16(kPfRows, kPfKeys, kBF16);
-  constexpr uint32_t kIdescO = umma_idesc_f16(kPfRows, kPfD, kBF16);
-
-  float o[kPfD];
-#pragma unroll
-  for (int d = 0; d < kPfD; ++d) o[d] = 0.f;
-  float m_run = -INFINITY, l_run = 0.f;
+  const uint32_t tS = tmem, tPh = tmem + 64, tPl = tmem + 96, tO = tmem + 128;
   bool failed = false;
-
-  for (int kt = 0; kt < nkt; ++kt) {
-    if (!failed && !mbar_wait_bounded(full, kt & 1)) {
+  auto wait = [&](uint32_t bar, int parity) {
+    if (!failed && !mbar_wait_bounded(bar, parity)) {
       failed = true;
       record_error(PA_ERR_TIMEOUT);
     }
-    const int bad = *bad_mask;
-    // ---- S = Q K^T (one thread issues; 8 MMAs of K = 16 along head_dim)
-    if (tid == 0 && !failed) {
+  };
+  auto bad_of = [&](int kt) {
+    int m = 0;
+    if (any_bad) {
+#pragma unroll
+      for (int b = 0; b < C::kBlocksPerTile; ++b) m |= (tile_block(kt, b) == -2) << b;
+    }
+    return m;
+  };
+
+  if (producer) {
+    // ======================= producer warp ==============================
+    constexpr uint32_t kIdescS = umma_idesc_f16(kPfRows, kPfKeys, kBF16);
+    constexpr uint32_t kIdescO = umma_idesc_f16(kPfRows, kPfD, kBF16, /*b_mn_major=*/true);
+    auto issue_s = [&](int kt) {  // S(kt) = Q K(kt)^T
+      wait(full_k + 8 * (kt & 1), (kt >> 1) & 1);
+      if (failed || lane != 0) return;
       tc_fence_after_sync();
+      const uint32_t k_st = sK + (kt & 1) * C::kKBytes;
 #pragma unroll
       for (int k = 0; k < kPfD / 16; ++k)
         umma_f16(tS, umma_desc_k128(sQ + (k >> 2) * (kPfRows * 128) + (k & 3) * 32),
-                 umma_desc_k128(sK + (k >> 2) * (kPfKeys * 128) + (k & 3) * 32), kIdescS,
+                 umma_desc_k128(k_st + (k >> 2) * (kPfKeys * 128) + (k & 3) * 32), kIdescS,
                  k > 0 ? 1u : 0u);
       umma_commit(bar_s);
-    }
-    // ---- meanwhile Vt = V^T: 8x8 tiles read with ldmatrix, stored transposed;
-    // keys the tile must not use (past the context, bad block) are zeroed
-    if (!failed) {
-      const int dg = warp * 4 + (lane >> 3);  // 8-dim group this lane addresses
-#pragma unroll
-      for (int kg = 0; kg < kPfKeys / 8; ++kg) {
-        uint32_t r0, r1, r2, r3;
-        ldsm_x4(sV + (dg >> 3) * (kPfKeys * 128) + swz128(kg * 8 + (lane & 7), dg & 7), r0, r1, r2,
-                r3);
-        const int kl = kg * 8 + (lane >> 2);  // the key this thread's fragments hold
-        if (kt * kPfKeys + kl >= ctx || ((bad >> (kl / BS)) & 1)) r0 = r1 = r2 = r3 = 0;
-        stsm_x4_trans(sVt + swz128(dg * 8 + (lane & 7), kg), r0, r1, r2, r3);
+    };
+    issue_s(0);
+    for (int kt = 0; kt < nkt; ++kt) {
+      const int st = kt & 1;
+      if (kt + 1 < nkt) {
+        wait(s_free, kt & 1);  // every row has read S(kt): S(kt) is done, K(kt) free
+        issue_s(kt + 1);
+        if (lane == 0 && !failed && kt + 2 < nkt) issue_tile(kt + 2, false);
       }
-    }
-    fence_proxy_async_smem();
-    // ---- online softmax of this thread's row
-    if (!failed && !mbar_wait_bounded(bar_s, kt & 1)) {
-      failed = true;
-      record_error(PA_ERR_TIMEOUT);
-    }
-    tc_fence_after_sync();
-    uint32_t sa[32], sb[32];
-    tmem_ld32(tS + lane_off, sa);
-    tmem_ld32(tS + lane_off + 32, sb);
-    tmem_wait_ld();
-    float x[kPfKeys];
-    float mx = -INFINITY;
+      wait(p_ready, kt & 1);  // P(kt) in TMEM, O(kt-1) done (the rows waited for it)
+      if (lane == 0 && !failed && kt >= 1 && kt + 1 < nkt) issue_tile(kt + 1, true);
+      wait(full_v + 8 * st, (kt >> 1) & 1);
+      // values of keys past the context or in bad blocks may hold anything
+      // (0 * NaN would reach O): zero their rows of V(kt)
+      const int bad = bad_of(kt);
+      if ((kt + 1) * kPfKeys > ctx || bad) {
 #pragma unroll
-    for (int c = 0; c < kPfKeys; ++c) {
-      const int key = kt * kPfKeys + c;
-      const bool ok = row_ok && !failed && key <= qpos && !((bad >> (c / BS)) & 1);
-      x[c] = ok ? __uint_as_float(c < 32 ? sa[c] : sb[c - 32]) * a.sl2 : -INFINITY;
-      mx = fmaxf(mx, x[c]);
-    }
-    const float m_new = fmaxf(m_run, mx);
-    const float alpha = m_new == -INFINITY ? 1.f : fast_exp2(m_run - m_new);
-    // P = P_hi + P_lo, both in the operands' 16-bit type: rounding P to one
-    // 16-bit value alone (8 significant bits for bf16) errs by up to 2^-9 of
-    // each weight, which outputs formed by cancellation cannot absorb
-    float psum = 0.f;
-    uint32_t pk[kPfKeys / 2], pl[kPfKeys / 2];
+        for (int i = 0; i < 4; ++i) {
+          const int row = lane + 32 * i, key = row & (kPfKeys - 1), hf = row >> 6;
+          if (kt * kPfKeys + key >= ctx || ((bad >> (key / BS)) & 1)) {
+            uint4* dst = reinterpret_cast<uint4*>(base + C::kOffV + st * C::kKBytes +
+                                                  hf * (kPfKeys * 128) + key * 128);
 #pragma unroll
-    for (int c = 0; c < kPfKeys; c += 2) {
-      const float p0 = x[c] == -INFINITY ? 0.f : fast_exp2(x[c] - m_new);
-      const float p1 = x[c + 1] == -INFINITY ? 0.f : fast_exp2(x[c + 1] - m_new);
-      psum += p0 + p1;
-      const uint32_t hi = pack2<kBF16>(p0, p1);
-      pk[c / 2] = hi;
-      pl[c / 2] = pack2<kBF16>(p0 - to_float<kBF16>(hi & 0xffff), p1 - to_float<kBF16>(hi >> 16));
-    }
-    l_run = l_run * alpha + psum;
-    m_run = m_new;
+            for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+      }
+      if (lane == 0 && !failed) {  // O += (P_hi + P_lo) V(kt): 2 x 4 MMAs of K = 16
+        tc_fence_after_sync();
+        const uint32_t v_st = sV + st * C::kKBytes;
 #pragma unroll
-    for (int c = 0; c < 8; ++c) {
-      *reinterpret_cast<uint4*>(base + C::kOffP + swz128(r, c)) =
-          make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      *reinterpret_cast<uint4*>(base + C::kOffP + C::kPBytes + swz128(r, c)) =
-          make_uint4(pl[4 * c], pl[4 * c + 1], pl[4 * c + 2], pl[4 * c + 3]);
+        for (int k = 0; k < kPfKeys / 16; ++k)
+          umma_f16_ts(tO, tPh + 8 * k, umma_desc_mn128(v_st + k * 2048, kPfKeys * 128), kIdescO,
+                      (kt > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+        for (int k = 0; k < kPfKeys / 16; ++k)
+          umma_f16_ts(tO, tPl + 8 * k, umma_desc_mn128(v_st + k * 2048, kPfKeys * 128), kIdescO,
+                      1u);
+        umma_commit(bar_o);
+      }
+      __syncwarp();
     }
-    fence_proxy_async_smem();
-    tc_fence_before_sync();
-    __syncthreads();  // P and Vt complete; S, K and V no longer read
-    if (tid == 0 && !failed) {
-      // ---- O tile = (P_hi + P_lo) Vt^T (2 x 4 MMAs of K = 16 along the keys)
+  } else {
+    // ======================= row warps ==================================
+    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;  // the warp's TMEM lanes
+    const uint64_t sl2x2 = f2(a.sl2, a.sl2);
+    float m_run = -INFINITY;  // running max of the raw scores
+    float l_run = 0.f;        // sum of weights, relative to m_run
+    for (int kt = 0; kt < nkt; ++kt) {
+      wait(bar_s, kt & 1);
       tc_fence_after_sync();
+      uint32_t sv[kPfKeys];
+      {
+        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
+        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
+        tmem_ld32(tS + lane_off, lo);
+        tmem_ld32(tS + lane_off + 32, hi);
+      }
+      tmem_wait_ld();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(s_free);
+      float x[kPfKeys];
 #pragma unroll
-      for (int k = 0; k < kPfKeys / 16; ++k)
-        umma_f16(tO, umma_desc_k128(sP + k * 32), umma_desc_k128(sVt + k * 32), kIdescO,
-                 k > 0 ? 1u : 0u);
+      for (int c = 0; c < kPfKeys; ++c) x[c] = __uint_as_float(sv[c]);
+      // keys past the diagonal, the context, or in a bad block get -inf;
+      // tiles wholly below the CTA's first row need no mask
+      const bool masked = any_bad || kt * kPfKeys + kPfKeys - 1 > qfirst;
+      if (masked) {
+        const int bad = bad_of(kt);
+        const int lim = row_ok ? qpos - kt * kPfKeys : -1;  // keys c <= lim are visible
 #pragma unroll
-      for (int k = 0; k < kPfKeys / 16; ++k)
-        umma_f16(tO, umma_desc_k128(sP + C::kPBytes + k * 32), umma_desc_k128(sVt + k * 32),
-                 kIdescO, 1u);
-      umma_commit(bar_o);
-      // the next key tile's loads overlap this product and the O update
-      if (kt + 1 < nkt) issue_tile(kt + 1);
+        for (int c = 0; c < kPfKeys; ++c)
+          if (c > lim || ((bad >> (c / BS)) & 1)) x[c] = -INFINITY;
+      }
+      float mx = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kPfKeys; c += 2) mx = fmax3(mx, x[c], x[c + 1]);
+      const float m_new = fmaxf(m_run, mx);
+      // rescale only when the max grew by more than 2^8 (in weight terms);
+      // false while the row has seen no key (m_new = -inf)
+      const bool resc = (m_new - m_run) * a.sl2 > kPfRescaleLog2;
+      float alpha = 1.f;
+      if (resc) {
+        alpha = m_run == -INFINITY ? 0.f : fast_exp2((m_run - m_new) * a.sl2);
+        m_run = m_new;
+      }
+      const float nm = m_run == -INFINITY ? 0.f : -m_run * a.sl2;
+      const uint64_t nm2 = f2(nm, nm);
+      // P = P_hi + P_lo, both in the operands' 16-bit type: rounding P to one
+      // 16-bit value alone (8 significant bits for bf16) errs by up to 2^-9 of
+      // each weight, which outputs formed by cancellation cannot absorb
+      uint32_t ph[kPfKeys / 2], pl[kPfKeys / 2];
+      uint64_t sum2 = f2(0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < kPfKeys; c += 2) {
+        const float2 e = f2_split(f2_fma(f2(x[c], x[c + 1]), sl2x2, nm2));
+        const float p0 = fast_exp2(e.x), p1 = fast_exp2(e.y);  // exp2(-inf) = 0
+        const uint64_t pp = f2(p0, p1);
+        sum2 = f2_add(sum2, pp);
+        const uint32_t h = pack2<kBF16>(p0, p1);
+        ph[c / 2] = h;
+        uint64_t hf;
+        if constexpr (kBF16) hf = f2(__uint_as_float(h << 16), __uint_as_float(h & 0xffff0000u));
+        else hf = f2(to_float<false>(h & 0xffff), to_float<false>(h >> 16));
+        const float2 d = f2_split(f2_sub(pp, hf));
+        pl[c / 2] = pack2<kBF16>(d.x, d.y);
+      }
+      const float2 ss = f2_split(sum2);
+      l_run = l_run * alpha + (ss.x + ss.y);
+      if (kt > 0) {
+        wait(bar_o, (kt - 1) & 1);  // O(kt-1) done: P's columns free, O stable
+        tc_fence_after_sync();
+        if (__any_sync(0xffffffffu, resc)) {  // tcgen05.ld / st are warp-wide
+          const uint64_t al2 = f2(alpha, alpha);
+#pragma unroll
+          for (int c = 0; c < kPfD / 32; ++c) {
+            uint32_t ot[32];
+            tmem_ld32(tO + lane_off + 32 * c, ot);
+            tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 32; j += 2) {
+              const float2 v = f2_split(
+                  f2_mul(f2(__uint_as_float(ot[j]), __uint_as_float(ot[j + 1])), al2));
+              ot[j] = __float_as_uint(v.x);
+              ot[j + 1] = __float_as_uint(v.y);
+            }
+            tmem_st32(tO + lane_off + 32 * c, ot);
+          }
+        }
+      }
+      tmem_st32(tPh + lane_off, ph);
+      tmem_st32(tPl + lane_off, pl);
+      tmem_wait_st();
+      tc_fence_before_sync();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_ready);
     }
-    if (!failed && !mbar_wait_bounded(bar_o, kt & 1)) {
-      failed = true;
-      record_error(PA_ERR_TIMEOUT);
-    }
+
+    // ---- epilogue: O / l for this thread's row
+    wait(bar_o, (nkt - 1) & 1);
     tc_fence_after_sync();
+    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+    uint4* const orow = reinterpret_cast<uint4*>(a.out) + orow_off;
 #pragma unroll
     for (int c = 0; c < kPfD / 32; ++c) {
       uint32_t ot[32];
       tmem_ld32(tO + lane_off + 32 * c, ot);
       tmem_wait_ld();
+      if (row_ok) {
 #pragma unroll
-      for (int j = 0; j < 32; ++j) o[32 * c + j] = o[32 * c + j] * alpha + __uint_as_float(ot[j]);
-    }
-    tc_fence_before_sync();
-    __syncthreads();  // S, the O tile, P and Vt are free again
-  }
-
-  if (row_ok) {
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-#pragma unroll
-    for (int j = 0; j < kPfD / 8; ++j) {
-      uint4 v;
-      v.x = pack2<kBF16>(o[8 * j] * inv, o[8 * j + 1] * inv);
-      v.y = pack2<kBF16>(o[8 * j + 2] * inv, o[8 * j + 3] * inv);
-      v.z = pack2<kBF16>(o[8 * j + 4] * inv, o[8 * j + 5] * inv);
-      v.w = pack2<kBF16>(o[8 * j + 6] * inv, o[8 * j + 7] * inv);
-      orow[j] = v;
+        for (int j = 0; j < 4; ++j) {
+          uint4 v;
+          v.x = pack2<kBF16>(__uint_as_float(ot[8 * j]) * inv, __uint_as_float(ot[8 * j + 1]) * inv);
+          v.y = pack2<kBF16>(__uint_as_float(ot[8 * j + 2]) * inv, __uint_as_float(ot[8 * j + 3]) * inv);
+          v.z = pack2<kBF16>(__uint_as_float(ot[8 * j + 4]) * inv, __uint_as_float(ot[8 * j + 5]) * inv);
+          v.w = pack2<kBF16>(__uint_as_float(ot[8 * j + 6]) * inv, __uint_as_float(ot[8 * j + 7]) * inv);
+          orow[4 * c + j] = failed ? make_uint4(0, 0, 0, 0) : v;
+        }
+      }
     }
   }
   tc_fence_before_sync();

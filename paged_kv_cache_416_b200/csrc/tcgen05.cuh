@@ -1,7 +1,8 @@
 // 5th-generation tensor core (tcgen05) helpers for sm_100a: tensor memory
-// (TMEM) allocation, MMA issue and completion, TMEM -> register loads, the
-// ordering fences, and the shared-memory / instruction descriptors of
-// kind::f16 MMAs on K-major, 128-byte-swizzled operand tiles.
+// (TMEM) allocation, MMA issue (operand A from shared or tensor memory) and
+// completion, TMEM <-> register moves, the ordering fences, and the
+// shared-memory / instruction descriptors of kind::f16 MMAs on K-major and
+// MN-major 128-byte-swizzled operand tiles.
 #pragma once
 
 #include "common.cuh"
@@ -40,6 +41,18 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint6
       : "memory");
 }
 
+// ---- D[tmem] (+)= A[tmem] * B[smem]^T: A (M x K, K-major) read from tensor
+// memory, row m in lane m, two 16-bit elements per 32-bit column
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                            uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on `bar` when every MMA this thread issued before has completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
@@ -55,6 +68,16 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 }
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---- registers -> TMEM, same shape as tmem_ld32; complete after tmem_wait_st()
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+               ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // ---- descriptors
@@ -74,12 +97,30 @@ __device__ __forceinline__ uint64_t umma_desc_k128(uint32_t smem_addr) {
   return d;
 }
 
+// Shared-memory matrix descriptor of an MN-major operand in the 128-byte
+// swizzle layout: each 128-byte row holds 64 consecutive MN elements of one K
+// index, 8 rows (8 K values) form a 1024-byte swizzle atom, K groups of 8 are
+// 1024 bytes apart (stride byte offset) and the next 64 MN elements start
+// `mn_stride` bytes further (leading byte offset).  Moving along K by 16
+// adds 2048 bytes to the start address.
+__device__ __forceinline__ uint64_t umma_desc_mn128(uint32_t smem_addr, uint32_t mn_stride) {
+  uint64_t d = static_cast<uint64_t>((smem_addr & 0x3FFFF) >> 4);
+  d |= static_cast<uint64_t>((mn_stride >> 4) & 0x3FFF) << 16;
+  d |= static_cast<uint64_t>(1024 >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  d |= static_cast<uint64_t>(2) << 61;
+  return d;
+}
+
 // Instruction descriptor of kind::f16 with fp32 accumulators, both operands
 // K-major: D format [4,6) = 1 (f32), A / B format [7,10) / [10,13) = 0 f16
 // or 1 bf16, N >> 3 in [17,23), M >> 4 in [24,29).
-__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, bool bf16) {
+// `b_mn_major` sets bit 16: B is read MN-major.
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, bool bf16,
+                                                      bool b_mn_major = false) {
   return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) |
-         (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+         ((b_mn_major ? 1u : 0u) << 16) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
 }
 
 // stmatrix: four 8x8 b16 tiles from the ldmatrix fragment layout, transposed

@@ -57,3 +57,49 @@ def test_prefill_rejects_unsupported_shapes(pa):
     with pytest.raises(pa.PagedAttnError) as e:
         run(pa, pw)
     assert e.value.status == 4
+
+
+def grow_keys(pw, rate):
+    """Scale the key at position p by (1 + p * rate), so the scores, and with
+    them each row's running max, keep growing along the context: the online
+    softmax has to rescale O many times."""
+    b = pw.base
+    kp = b.k_pool.float()
+    flat = kp.view(-1, b.num_kv_heads, kp.shape[-1])
+    bs = kp.shape[1]
+    for s in range(b.num_seqs):
+        for p in range(int(b.context_lens[s])):
+            flat[int(b.block_tables[s, p // bs]) * bs + p % bs] *= 1.0 + p * rate
+    b.k_pool = kp.to(b.k_pool.dtype)
+    return pw
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f16"])
+def test_prefill_long_context_growing_scores(pa, dtype):
+    # a chunk late in a long context (many key tiles, both K/V stages reused
+    # many times) with scores that grow along the keys
+    pw = grow_keys(W.prefill(seed=11, ctxs=(1500, 700), nqs=(96, 700), hq=32, hkv=8, bs=16,
+                             dtype=dtype), 1.0 / 48)
+    assert_attention_close(as_f64(run(pa, pw)), ref(pw), f"prefill growing scores {dtype}")
+
+
+def test_prefill_bad_table_entry_masks_its_block(pa):
+    # a table entry outside the pool: the kernel reports it, masks that
+    # block's keys and zeroes its values; the other outputs equal attention
+    # over the remaining keys
+    pw = W.prefill(seed=12, ctxs=(160,), nqs=(160,), hq=32, hkv=8, bs=16, dtype="bf16")
+    b = pw.base
+    b.block_tables = b.block_tables.copy()
+    b.block_tables[0, 3] = b.k_pool.shape[0] + 5
+    bt = torch.from_numpy(b.block_tables).cuda()
+    out = pa.prefill(pw.q.cuda(), b.k_pool.cuda(), b.v_pool.cuda(), bt,
+                     torch.from_numpy(b.context_lens).cuda(),
+                     torch.from_numpy(pw.query_start).cuda(), b.scale, pw.max_query_len,
+                     b.max_context_len)
+    with pytest.raises(pa.PagedAttnError):
+        pa.sync_status()
+    got = as_f64(out)
+    assert np.isfinite(got).all()
+    # rows before block 3 never see it: they equal the oracle on the intact table
+    good = ref(W.prefill(seed=12, ctxs=(160,), nqs=(160,), hq=32, hkv=8, bs=16, dtype="bf16"))
+    assert_attention_close(got[:48], good[:48], "rows before the bad block")
