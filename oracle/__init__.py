@@ -50,6 +50,10 @@ from .paged import (
     decode,
     decode_one,
     prefill,
+    shared_prefix_blocks,
+    partial_attention,
+    merge_partials,
+    shared_prefix_decode,
 )
 from .memory import (
     kv_bytes_per_token,
@@ -64,4 +68,5 @@ __all__ = [
     "e4m3_finite_values", "decode_cache", "slot_of", "write_kv", "copy_blocks",
     "swap_blocks", "gather", "attention_weights", "decode", "decode_one", "prefill", "kv_bytes_per_token",
     "kv_bytes", "reservation_unused_slots", "paged_unused_slots", "blocks_needed",
+    "shared_prefix_blocks", "partial_attention", "merge_partials", "shared_prefix_decode",
 ]

@@ -191,3 +191,91 @@ def prefill(q_raw, q_dtype: str, k_pool, v_pool, cache_dtype: str, block_tables,
                 w = attention_weights(q[qs[s] + i, h], K[: pos + 1, kv, :], scale)
                 out[qs[s] + i, h] = w @ V[: pos + 1, kv, :]
     return out
+
+
+def shared_prefix_blocks(block_tables, context_lens, members, block_size: int) -> int:
+    """Blocks a group of sequences shares at the head of their tables: the
+    longest run of leading table entries equal in every member's row, cut
+    so that each member keeps at least one token of its own (the prefix
+    lies inside every member's context and ends before its last token).
+    A group of fewer than two members shares nothing.
+
+    ("PagedAttention", §Diziler Arasında Blokları Paylaşma: sequences forked
+    from one prompt -- parallel sampling, beam search, a common prompt --
+    name the same physical blocks in their tables.)"""
+    members = [int(m) for m in members]
+    if len(members) < 2:
+        return 0
+    limit = min((int(context_lens[m]) - 1) // block_size for m in members)
+    lead = block_tables[members[0]]
+    p = 0
+    while p < limit and all(int(block_tables[m][p]) == int(lead[p]) for m in members):
+        p += 1
+    return max(p, 0)
+
+
+def partial_attention(q_vec: np.ndarray, keys: np.ndarray, values: np.ndarray, scale: float):
+    """Attention of one query over one part of its context, kept as the
+    pair (log-sum-exp of the scores, normalised output): ``lse = log sum
+    exp(z)``, ``o = softmax(z) @ values`` with ``z = scale * keys @ q``.
+    An empty part gives (-inf, 0)."""
+    if keys.shape[0] == 0:
+        return -np.inf, np.zeros(values.shape[-1])
+    z = float(scale) * (keys @ q_vec)
+    m = z.max()
+    e = np.exp(z - m)
+    return m + np.log(e.sum()), (e / e.sum()) @ values
+
+
+def merge_partials(parts):
+    """Combine the (lse, o) pairs of disjoint parts of one context into the
+    attention over their union: weights ``exp(lse_i - max lse)``,
+    ``out = sum_i w_i o_i / sum_i w_i``."""
+    lses = np.array([p[0] for p in parts], dtype=np.float64)
+    M = lses.max()
+    if M == -np.inf:
+        return np.zeros_like(parts[0][1])
+    w = np.exp(lses - M)
+    return sum(wi * p[1] for wi, p in zip(w, parts)) / w.sum()
+
+
+def shared_prefix_decode(q_raw, q_dtype: str, k_pool, v_pool, cache_dtype: str, block_tables,
+                         context_lens, group_start, group_seqs, scale: float, num_kv_heads: int,
+                         k_scale: float = 1.0, v_scale: float = 1.0):
+    """Decode attention with shared prefixes taken apart (cascade form), fp64.
+
+    For every group g (sequences ``group_seqs[group_start[g]:group_start[g+1]]``)
+    the shared blocks (``shared_prefix_blocks``) are attended once per member
+    query as one part, the member's remaining tokens as a second part, and
+    the two partial results are merged by log-sum-exp (``merge_partials``).
+    Sequences in no group are one part.  The result is the plain decode
+    attention of every sequence (``decode``), a sum split in two.
+    Returns (out ``[B, Hq, D]``, shared blocks per sequence ``[B]``).
+    """
+    q = decode_cache(q_raw, q_dtype)
+    B, hq, d = q.shape
+    bs = k_pool.shape[1]
+    group = hq // num_kv_heads
+    pre = np.zeros(B, dtype=np.int64)
+    gs = np.asarray(group_start, dtype=np.int64)
+    for g in range(len(gs) - 1):
+        members = list(group_seqs[gs[g]:gs[g + 1]])
+        p = shared_prefix_blocks(block_tables, context_lens, members, bs)
+        for m in members:
+            pre[int(m)] = p
+    out = np.zeros((B, hq, d), dtype=np.float64)
+    for s in range(B):
+        n = int(context_lens[s])
+        if n <= 0:
+            continue
+        nb = -(-n // bs)
+        ids = np.asarray(block_tables[s][:nb], dtype=np.int64)
+        K = gather(decode_cache(k_pool[ids], cache_dtype, k_scale), np.arange(nb), n)
+        V = gather(decode_cache(v_pool[ids], cache_dtype, v_scale), np.arange(nb), n)
+        cut = int(pre[s]) * bs
+        for h in range(hq):
+            kv = h // group
+            head = partial_attention(q[s, h], K[:cut, kv], V[:cut, kv], scale)
+            tail = partial_attention(q[s, h], K[cut:, kv], V[cut:, kv], scale)
+            out[s, h] = merge_partials([head, tail])
+    return out, pre

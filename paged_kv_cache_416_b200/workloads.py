@@ -230,6 +230,13 @@ def fp8_longtail(seed=5, device="cpu", num_seqs=128, block_size=16, max_len=3276
     return w
 
 
+def _sample_groups(prompts: int, samples: int) -> Dict:
+    """The samples of one prompt form a group: group_seqs lists sequences
+    p * samples + i group by group, group_start[g] is where group g starts."""
+    return {"group_start": np.arange(prompts + 1, dtype=np.int32) * samples,
+            "group_seqs": np.arange(prompts * samples, dtype=np.int32)}
+
+
 def _shared_prefix(phase, seed, device, prompts=32, samples=4, prefix=1024,
                    max_tail=512, hq=32, hkv=8, d=128, bs=16) -> Workload:
     """Parallel sampling over a shared prompt (see the module docstring)."""
@@ -279,7 +286,8 @@ def _shared_prefix(phase, seed, device, prompts=32, samples=4, prefix=1024,
             scale=1.0 / math.sqrt(d), k_scale=1.0, v_scale=1.0, context_lens=lens,
             block_tables=tables, q=q, k_pool=k_pool, v_pool=v_pool, new_k=first_k, new_v=first_v,
             slot_mapping=np.asarray(first_slots, dtype=np.int64), cow_pairs=pairs,
-            meta={"seed": int(seed), "allocator": alloc, "prompt_lens": plen, "samples": samples},
+            meta={"seed": int(seed), "allocator": alloc, "prompt_lens": plen, "samples": samples,
+                  **_sample_groups(prompts, samples)},
         )
     # tails phase: lay the state after the fork step and T own tokens down
     # directly (copied prompt rows in the copied blocks, fresh values for the
@@ -322,7 +330,7 @@ def _shared_prefix(phase, seed, device, prompts=32, samples=4, prefix=1024,
         block_tables=tables, q=q, k_pool=k_pool, v_pool=v_pool, new_k=new_k, new_v=new_v,
         slot_mapping=np.asarray(step_slots, dtype=np.int64), cow_pairs=np.zeros((0, 2), np.int64),
         meta={"seed": int(seed), "allocator": alloc, "prompt_lens": plen, "tails": tails,
-              "samples": samples},
+              "samples": samples, **_sample_groups(prompts, samples)},
     )
 
 

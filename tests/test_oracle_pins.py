@@ -21,6 +21,8 @@ import torch.nn.functional as F
 import oracle
 from oracle import codecs, paged, memory
 from paged_kv_cache_416_b200.alloc import BlockAllocator
+from paged_kv_cache_416_b200 import workloads as W
+from paged_kv_cache_416_b200.workloads import raw
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
 
@@ -509,3 +511,56 @@ def test_prefill_last_token_equals_decode_and_first_token_sees_itself_only():
     v0 = codecs.f16_bits_to_f64(vp[tables[0, 0], 0])
     for h in range(hq):
         assert np.array_equal(pre[0, h], v0[h])
+
+
+# ---- shared-prefix (cascade) decode -----------------------------------------
+def test_shared_prefix_blocks_by_hand():
+    # tables agree on their first two entries; bs 16
+    t = np.array([[5, 6, 7, 8], [5, 6, 9, 10], [5, 11, 12, 13]], dtype=np.int32)
+    assert paged.shared_prefix_blocks(t, [60, 60, 60], [0, 1], 16) == 2
+    # the prefix ends before each member's last token: 33 tokens keep 2 blocks, 32 keep 1
+    assert paged.shared_prefix_blocks(t, [33, 60, 60], [0, 1], 16) == 2
+    assert paged.shared_prefix_blocks(t, [32, 60, 60], [0, 1], 16) == 1
+    assert paged.shared_prefix_blocks(t, [60, 60, 60], [0, 1, 2], 16) == 1
+    assert paged.shared_prefix_blocks(t, [60, 60, 60], [1], 16) == 0  # one member
+    t2 = t.copy()
+    t2[1, 0] = 99
+    assert paged.shared_prefix_blocks(t2, [60, 60, 60], [0, 1], 16) == 0
+
+
+def test_partial_attention_and_merge_by_brute_force():
+    rng = np.random.default_rng(21)
+    q = rng.standard_normal(4)
+    K = rng.standard_normal((7, 4))
+    V = rng.standard_normal((7, 3))
+    z = [0.5 * sum(K[t, i] * q[i] for i in range(4)) for t in range(7)]
+    lse = math.log(math.fsum(math.exp(x) for x in z))
+    w = [math.exp(x - lse) for x in z]
+    full = [math.fsum(w[t] * V[t, j] for t in range(7)) for j in range(3)]
+    l, o = paged.partial_attention(q, K, V, 0.5)
+    assert abs(l - lse) < 1e-12
+    np.testing.assert_allclose(o, full, rtol=0, atol=1e-12)
+    for cut in range(8):  # any split point, the empty parts included
+        parts = [paged.partial_attention(q, K[:cut], V[:cut], 0.5),
+                 paged.partial_attention(q, K[cut:], V[cut:], 0.5)]
+        np.testing.assert_allclose(paged.merge_partials(parts), full, rtol=0, atol=1e-12)
+    # an empty part carries no weight
+    e = paged.partial_attention(q, K[:0], V[:0], 0.5)
+    assert e[0] == -np.inf and not e[1].any()
+
+
+@pytest.mark.parametrize("phase", ["fork", "tails"])
+def test_shared_prefix_decode_equals_plain_decode(phase):
+    w = W._shared_prefix(phase, 4, "cpu", prompts=3, samples=3, prefix=64, max_tail=40,
+                         hq=8, hkv=2, d=32, bs=16)
+    kp, vp = raw(w.k_pool), raw(w.v_pool)
+    paged.copy_blocks(kp, vp, w.cow_pairs)  # the decode step: copy-on-write, then the write
+    paged.write_kv(raw(w.new_k), raw(w.new_v), "bf16", w.slot_mapping, kp, vp, "bf16")
+    args = (raw(w.q), "bf16", kp, vp, "bf16", w.block_tables, w.context_lens)
+    got, pre = paged.shared_prefix_decode(*args, w.meta["group_start"], w.meta["group_seqs"],
+                                          w.scale, w.num_kv_heads)
+    ref = paged.decode(*args, w.scale, w.num_kv_heads)
+    assert np.isfinite(ref).all()
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+    # every sample shares its prompt's full blocks: 64 + r tokens -> 4 blocks at bs 16
+    assert (pre == 4).all()
