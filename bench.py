@@ -57,7 +57,8 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling only)")
-    ap.add_argument("--op", choices=["decode", "swap", "hash", "prefill"], default="decode",
+    ap.add_argument("--op", choices=["decode", "swap", "hash", "prefill", "shared_prefix"],
+                    default="decode",
                     help="decode: the decode step (the headline line); the others time "
                          "one companion operation on one GPU and print its own line")
     return ap.parse_args(argv)
@@ -629,6 +630,71 @@ def run_prefill(args):
     }
 
 
+def unique_kv_bytes(w) -> int:
+    """K+V bytes of the distinct physical blocks the step reads (each block
+    counted up to the furthest token any sequence reads in it)."""
+    import numpy as np
+    bs = w.block_size
+    used = {}
+    for s in range(w.num_seqs):
+        n = int(w.context_lens[s])
+        for j in range(-(-n // bs)):
+            b = int(w.block_tables[s, j])
+            used[b] = max(used.get(b, 0), min(bs, n - j * bs))
+    tokens = int(np.sum(list(used.values())))
+    return tokens * w.num_kv_heads * w.head_dim * 2 * {"e4m3": 1}.get(w.cache_dtype, 2)
+
+
+def run_shared_prefix(args):
+    """pa_decode_shared_prefix on the shared-prefix workload (32 prompts x 4
+    samples, 32/8 heads, D 128, bf16, bs 16, 1024 + r shared tokens, tails
+    U{0..512}): every prompt's blocks are read once for its four samples.
+    Timed beside pa_decode on the same inputs.  Roofline: HBM, on the unique
+    bytes (the distinct blocks read), against the measured copy bandwidth."""
+    import torch
+    from paged_kv_cache_416_b200 import build as _build
+    _build.build()
+    from paged_kv_cache_416_b200 import pagedattn as pa
+    from paged_kv_cache_416_b200 import workloads as W
+    torch.cuda.set_device(0)
+    w = W.make("shared_prefix_tails", seed=args.seed, device="cuda")
+    kp, vp = w.k_pool, w.v_pool
+    pa.write_kv(w.new_k, w.new_v, torch.from_numpy(w.slot_mapping).cuda(), kp, vp)
+    q = w.q.contiguous()
+    bt = torch.from_numpy(w.block_tables).cuda()
+    cl = torch.from_numpy(w.context_lens).cuda()
+    gs = torch.from_numpy(w.meta["group_start"]).cuda()
+    gq = torch.from_numpy(w.meta["group_seqs"]).cuda()
+    out = torch.empty_like(q)
+    ws = pa.workspace_for(q.device, pa.shared_prefix_workspace_size(
+        w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size, w.max_context_len))
+    iters = max(20, min(args.steps, 200))
+    t_shared = _events_time(lambda: pa.decode_shared_prefix(
+        q, kp, vp, bt, cl, gs, gq, w.scale, w.max_context_len, out=out, workspace=ws), iters)
+    t_plain = _events_time(lambda: pa.decode(q, kp, vp, bt, cl, w.scale, w.max_context_len,
+                                             out=out), iters)
+    pa.sync_status()
+    logical = w.kv_bytes
+    unique = unique_kv_bytes(w)
+    peak, peak_kind = measured_peaks()
+    ach = unique / t_shared / 1e9
+    return {
+        "metric": "shared-prefix decode: KV-read GB/s (logical bytes)", "op": "shared_prefix",
+        "value": round(logical / t_shared / 1e9, 1), "unit": "GB/s", "n_gpus": 1,
+        "steps": iters, "higher_is_better": True, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "shared_prefix_tails: 32 prompts x 4 samples, 32/8 heads, D 128, "
+                               "bf16, bs 16, 1024 + r shared tokens, tails U{0..512}",
+                   "logical_kv_bytes": logical, "unique_kv_bytes": unique},
+        "us_per_call": round(t_shared * 1e6, 2),
+        "plain_decode_us_per_call": round(t_plain * 1e6, 2),
+        "speedup_vs_plain_decode": round(t_plain / t_shared, 3),
+        "roofline": {"bound": "hbm", "achieved": round(ach, 1), "peak": peak, "unit": "GB/s",
+                     "frac": round(ach / peak, 4), "bytes": "unique",
+                     "peak_kind": peak_kind},
+        "gpu_launches": 4 * iters,
+    }
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.warmup < 3:
@@ -646,7 +712,8 @@ def main(argv=None):
     if args.op != "decode":
         if rank != 0:
             return 0
-        line = {"swap": run_swap, "hash": run_hash, "prefill": run_prefill}[args.op](args)
+        line = {"swap": run_swap, "hash": run_hash, "prefill": run_prefill,
+                "shared_prefix": run_shared_prefix}[args.op](args)
         print(json.dumps(line), flush=True)
         return 0
     import torch

@@ -233,6 +233,55 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype,
                     void* workspace, size_t workspace_bytes, pa_stream_t stream);
 
 /*
+ * pa_decode_shared_prefix_workspace_size -- bytes of device workspace
+ * pa_decode_shared_prefix needs for these sizes (planning arrays, the work
+ * list and the per-range partials).  Returns 0 on invalid arguments.
+ */
+size_t pa_decode_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                              int32_t num_kv_heads, int32_t head_dim,
+                                              int32_t block_size, int32_t max_context_len,
+                                              int32_t split_tokens);
+
+/*
+ * pa_decode_shared_prefix -- decode attention for sequences whose block
+ * tables share leading blocks (samples forked from one prompt, beams, a
+ * common system prompt: "PagedAttention", Ultralytics glossary, section
+ * "Diziler Arasinda Bloklari Paylasma", where several tables name the same
+ * physical blocks).  The result is pa_decode's (same formula, same
+ * arguments; up to fp32 rounding order, within the attention tolerance),
+ * but the shared blocks are read from memory once per group instead of
+ * once per member:
+ *   - group g lists its sequences in group_seqs[group_start[g] ..
+ *     group_start[g+1]) (device int32 arrays; group_start has num_groups + 1
+ *     entries, non-decreasing from 0, group_seqs group_start[num_groups]).
+ *     Sequences in no group are decoded on their own.  A sequence listed
+ *     twice, or outside [0, num_seqs), makes its group(s) decode unshared
+ *     and is reported as PA_ERR_RANGE at the next pa_sync_status.
+ *   - the shared part of a group is found on the device: the longest run of
+ *     leading table entries equal in every member's row, cut so that each
+ *     member keeps at least one token of its own.  Groups of one member, or
+ *     with a length outside [1, max_context_len], share nothing.
+ *   - up to 16 / (Hq/Hkv) members form a chunk whose query heads are the
+ *     rows of one tile: the shared blocks are attended once by all rows,
+ *     each member's own blocks by its rows only, in one pass over the
+ *     chunk's blocks, cut into ranges merged by log-sum-exp.
+ * Supported: q and cache both f16 or both bf16 (no e4m3), head_dim 64 or
+ * 128, block_size 16 or 32, Hq / Hkv <= 8.  split_tokens: 0 = automatic,
+ * else the shortest range in tokens.  workspace: at least
+ * pa_decode_shared_prefix_workspace_size(...) bytes, 256-byte aligned,
+ * stream-ordered use only.  Other errors as pa_decode.
+ */
+pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype q_dtype,
+                                  const void* k_pool, const void* v_pool, pa_dtype cache_dtype,
+                                  const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                  const int32_t* context_lens, int32_t max_context_len,
+                                  const int32_t* group_start, const int32_t* group_seqs,
+                                  int32_t num_groups, int32_t num_seqs, int32_t num_q_heads,
+                                  int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                  int32_t num_blocks, float scale, int32_t split_tokens,
+                                  void* workspace, size_t workspace_bytes, pa_stream_t stream);
+
+/*
  * pa_prefill -- paged prefill / chunked-prefill attention on the 5th-
  * generation tensor cores.  Several new query tokens per sequence attend
  * causally to the sequence's cached keys and values, gathered block by block

@@ -1,0 +1,654 @@
+// Shared-prefix-aware (cascade) decode attention, sm_100a.
+//
+// Method: sequences forked from one prompt (parallel sampling, beam search, a
+// common system prompt) name the same physical blocks at the head of their
+// block tables ("PagedAttention", Ultralytics glossary, section "Diziler
+// Arasinda Bloklari Paylasma").  Plain decode reads those blocks once per
+// sequence; here they are read once per group.
+//
+// Work decomposition
+//   chunk = up to 16 / G members of one group that share P leading blocks
+//           (or one sequence on its own, P = 0).  Its rows are the members'
+//           query heads of one kv head, at most 16 (the MMA's M).
+//   virtual block list of a chunk = the P shared blocks, then each member's
+//           own blocks (its table from entry P on), member after member.
+//           A shared block is attended by every row, an own block by its
+//           member's G rows only (the others see -inf scores for it).
+//   item  = (chunk, range of its virtual blocks, kv head); a chunk's blocks
+//           are cut into ranges of equal length; CTA = 4 warps, persistent,
+//           items from an atomic counter
+//   warp  = every 4th block of the range, through a ring of stages filled by
+//           one tiled TMA copy per K or V tile (the decode kernel's tensor
+//           maps, swizzle and shared-memory layout); the table entries of
+//           the warp's next 32 blocks are resolved ahead in registers
+// Per 16 keys and warp (m16n8k16, rows = the chunk's query rows):
+//   S = Q K^T        A = Q (registers), B = K rows (ldmatrix)
+//   online softmax   per row, masked by block owner and valid keys
+//   O += P V         A = P from the S accumulators (hi + lo 16-bit parts for
+//                    bf16), B = V (ldmatrix.trans; values of keys past a
+//                    member's length are zeroed in the fragments)
+// The warps' states are merged through shared memory.  A chunk of one range
+// writes the output; otherwise each range writes (log-sum-exp, normalised
+// output) per row and the CTA that finishes the chunk's last range merges
+// them (log-sum-exp merge).
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "decode.cuh"
+
+namespace pa {
+
+constexpr int kCascadeRows = 16;        // query rows per chunk (members x heads)
+constexpr int kCascadeMaxRanges = 512;  // ranges per chunk (their weights sit in smem)
+// work items (x Hkv) the range length aims at: ~1.5 waves of 444 persistent
+// CTAs (on the shared-prefix workload 666 ran 80.1 us, 444: 84.3, 888: 81.7,
+// 1332: 87.4 -- shorter ranges pay the per-range start and merge more often)
+constexpr int kCascadeTargetItems = 666;
+
+struct CascadeArgs {
+  CUtensorMap tmap_k;          // decode tensor maps over the pools
+  CUtensorMap tmap_v;
+  void* out;                   // [B, Hq, D]
+  const void* q;               // [B, Hq, D]
+  const int32_t* block_tables;
+  const int32_t* context_lens;
+  const int32_t* chunk_seqs;   // members, chunk by chunk
+  const int4* chunks;          // [2 * chunks]: (member offset, members, shared blocks, first
+                               // slot), (virtual blocks, ranges, blocks per range, -)
+  const int2* items;           // (chunk, range)
+  const int32_t* total;        // number of (chunk, range) items
+  int32_t* counter;            // work counter (zeroed by the planning kernel)
+  int32_t* arrived;            // [chunks * Hkv] ranges finished
+  float* lse_part;             // [slots * Hkv * 16]
+  float* o_part;               // [slots * Hkv * 16 * D]
+  int hq, hkv, group, max_blocks, num_blocks;
+  float sl2;                   // scale * log2(e)
+};
+
+template <bool kBF16, int D, int BS>
+__global__ void __launch_bounds__(kDecodeThreads)
+cascade_kernel(const __grid_constant__ CascadeArgs a) {
+  using C = DecodeCfg<kBF16 ? kCacheBF16 : kCacheF16, D, BS>;
+  constexpr int kStages = C::kStages;
+  constexpr int kNT = D / 8;  // output n-tiles (8 dims each)
+  constexpr int kRows = kCascadeRows;
+  static_assert(C::kWarpBytes >= (kRows * D + 2 * kRows) * 4, "warp ring too small for the merge");
+  static_assert(kDecodeWarps * C::kWarpBytes >= (kCascadeMaxRanges + 1) * kRows * 4,
+                "rings too small for the range weights");
+  static_assert(kStages <= 8, "stage info array");
+  extern __shared__ __align__(128) uint8_t smem[];
+  __shared__ int s_item;
+  __shared__ int s_flag;
+  __shared__ int s_seq[kRows];           // the chunk's members
+  __shared__ int s_tail[kRows];          // their own blocks (after the shared ones)
+  __shared__ int s_ctx[kRows];
+  __shared__ int s_binfo[kDecodeWarps][8];  // per warp and stage: owner + 1 | valid keys << 8
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int g = lane >> 2;   // fragment row (and row + 8)
+  const int tig = lane & 3;  // thread in group
+  const int li = lane >> 3;  // which 8x8 matrix of an ldmatrix.x4 this lane addresses
+
+  const uint32_t smem_s = smem_addr(smem);
+  const uint32_t ring_s = (smem_s + kBarrierBytes + kTileAlign - 1) & ~uint32_t(kTileAlign - 1);
+  const uint32_t wbase_s = ring_s + warp * C::kWarpBytes;
+  uint8_t* const ring = smem + (ring_s - smem_s);
+  const uint32_t bar0 = smem_s + warp * kStages * 8;
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < kStages; ++s) mbar_init(bar0 + 8 * s, 1);
+    mbar_init_fence();
+  }
+  if (threadIdx.x == 0) {
+    prefetch_tensormap(&a.tmap_k);
+    prefetch_tensormap(&a.tmap_v);
+    s_item = atomicAdd(a.counter, 1);
+  }
+  __syncthreads();
+
+  const int total = *a.total * a.hkv;
+  uint32_t n_issued = 0, n_consumed = 0;
+  uint32_t skip_stage = 0;
+  bool failed = false;
+
+  for (;;) {
+    const int item = s_item;
+    if (item >= total) break;
+    const int kvh = item % a.hkv;
+    const int2 cr = a.items[item / a.hkv];
+    const int chunk = cr.x, range = cr.y;
+    const int4 c0 = a.chunks[2 * chunk], c1 = a.chunks[2 * chunk + 1];
+    const int members = c0.y, P = c0.z, slot0 = c0.w;
+    const int vblocks = c1.x, nranges = c1.y, R = c1.z;
+    const int rows = members * a.group;
+    if (threadIdx.x < members) {
+      const int seq = a.chunk_seqs[c0.x + threadIdx.x];
+      const int c = a.context_lens[seq];  // validated by the planning kernel
+      s_seq[threadIdx.x] = seq;
+      s_ctx[threadIdx.x] = c;
+      s_tail[threadIdx.x] = (c + BS - 1) / BS - P;
+    }
+    __syncthreads();
+    const int vb0 = range * R;
+    const int nblk = max(0, min(vblocks, vb0 + R) - vb0);
+    const int nb_w = nblk > warp ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
+
+    // ---- virtual block -> (physical block, owner + 1 | valid keys << 8)
+    auto resolve = [&](int v, int& phys) -> int {
+      int seq, j, info;
+      if (v < P) {
+        seq = s_seq[0];
+        j = v;
+        info = BS << 8;  // every row, every key
+      } else {
+        int u = v - P, i = 0;
+        while (i < members - 1 && u >= s_tail[i]) u -= s_tail[i++];
+        seq = s_seq[i];
+        j = P + u;
+        info = (i + 1) | (min(BS, s_ctx[i] - j * BS) << 8);
+      }
+      phys = a.block_tables[static_cast<int64_t>(seq) * a.max_blocks + j];
+      return info;
+    };
+    // lane l holds the warp's block 32 * chunk + l; cur / nxt as in decode
+    int tab_chunk = 0, phys_cur = -1, info_cur = 0, phys_nxt = -1, info_nxt = 0;
+    auto load_chunk = [&](int ch, int& phys, int& info) {
+      const int i = ch * 32 + lane;
+      if (i < nb_w) {
+        info = resolve(vb0 + warp + i * kDecodeWarps, phys);
+      } else {
+        phys = -1;
+        info = 0;
+      }
+    };
+    load_chunk(0, phys_cur, info_cur);
+    load_chunk(1, phys_nxt, info_nxt);
+
+    auto issue = [&](int i) {
+      const int st = n_issued % kStages;
+      const uint32_t bar = bar0 + 8 * st;
+      const uint32_t sK = wbase_s + st * C::kStageBytes;
+      if ((i >> 5) != tab_chunk) {
+        tab_chunk = i >> 5;
+        phys_cur = phys_nxt;
+        info_cur = info_nxt;
+        load_chunk(tab_chunk + 1, phys_nxt, info_nxt);
+      }
+      const int phys = __shfl_sync(0xffffffffu, phys_cur, i & 31);
+      const int info = __shfl_sync(0xffffffffu, info_cur, i & 31);
+      const bool ok = phys >= 0 && phys < a.num_blocks;
+      skip_stage = ok ? (skip_stage & ~(1u << st)) : (skip_stage | (1u << st));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        s_binfo[warp][st] = info;
+        if (ok) {
+          mbar_arrive_expect_tx(bar, 2u * C::kTileBytes);
+          tma_load_5d(sK, &a.tmap_k, 0, 0, 0, kvh, phys, bar);
+          tma_load_5d(sK + C::kTileBytes, &a.tmap_v, 0, 0, 0, kvh, phys, bar);
+        } else {
+          record_error(PA_ERR_DEVICE_BOUNDS);  // the block's tokens are left out
+          mbar_arrive_expect_tx(bar, 0u);
+        }
+      }
+      ++n_issued;
+    };
+    if (!failed) {
+      const int pro = min(kStages, nb_w);
+      for (int i = 0; i < pro; ++i) issue(i);
+    }
+
+    // ---- query rows as the A operand: rows g and g + 8 of each 16-dim step
+    uint32_t qa[D / 16][4];
+    {
+      const uint16_t* qrow[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = g + 8 * h;
+        const int rr = r < rows ? r : 0;
+        qrow[h] = reinterpret_cast<const uint16_t*>(a.q) +
+                  (static_cast<int64_t>(s_seq[rr / a.group]) * a.hq + kvh * a.group +
+                   rr % a.group) * D;
+      }
+      const bool ok0 = g < rows, ok1 = g + 8 < rows;
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        const int d0 = ks * 16 + 2 * tig;
+        qa[ks][0] = ok0 ? *reinterpret_cast<const uint32_t*>(qrow[0] + d0) : 0u;
+        qa[ks][1] = ok1 ? *reinterpret_cast<const uint32_t*>(qrow[1] + d0) : 0u;
+        qa[ks][2] = ok0 ? *reinterpret_cast<const uint32_t*>(qrow[0] + d0 + 8) : 0u;
+        qa[ks][3] = ok1 ? *reinterpret_cast<const uint32_t*>(qrow[1] + d0 + 8) : 0u;
+      }
+    }
+    const int own0 = g / a.group, own1 = (g + 8) / a.group;  // member of rows g, g + 8
+
+    float acc[kNT][4];
+#pragma unroll
+    for (int n = 0; n < kNT; ++n)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
+    float m_run[2] = {-INFINITY, -INFINITY};  // rows g, g + 8 (log2 units)
+    float l_run[2] = {0.f, 0.f};              // this thread's share of the row sums
+
+    for (int i = 0; i < nb_w; ++i) {
+      const int st = n_consumed % kStages;
+      const uint32_t par = (n_consumed / kStages) & 1u;
+      if (!failed) {
+        const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar0 + 8 * st, par));
+        if (!ok) {
+          failed = true;
+          if (lane == 0) record_error(PA_ERR_TIMEOUT);
+        }
+      }
+      __syncwarp();  // lane 0's s_binfo write of this stage is visible
+      if (!failed && !((skip_stage >> st) & 1u)) {
+        const uint32_t sK = wbase_s + st * C::kStageBytes;
+        const uint32_t sV = sK + C::kTileBytes;
+        const int info = s_binfo[warp][st];
+        const int owner = (info & 0xff) - 1;  // -1: a shared block
+        const int valid = info >> 8;           // keys of the block inside the context
+        // rows that attend this block: every member's for a shared block,
+        // the owner's G rows for an own block
+        const bool act0 = owner < 0 || own0 == owner;
+        const bool act1 = owner < 0 || own1 == owner;
+        const bool full = owner < 0;           // shared blocks are whole and seen by all
+#pragma unroll
+        for (int kt = 0; kt < BS / 16; ++kt) {
+          // ---- S = Q K^T for 16 keys: two n-tiles of 8 keys, even / odd
+          // dim steps in separate accumulators (four independent chains)
+          float s[2][4], so[2][4];
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) s[nt][e] = so[nt][e] = 0.f;
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) {
+            const int key = kt * 16 + nt * 8 + (lane & 7);
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ks += 2) {
+              uint32_t b0, b1, b2, b3;
+              ldsm_x4(sK + tile_off<C>(key, ((ks + (li >> 1)) * 16 + (li & 1) * 8) * 2), b0, b1,
+                      b2, b3);
+              mma_16816<kBF16>(s[nt], qa[ks], b0, b1);
+              mma_16816<kBF16>(so[nt], qa[ks + 1], b2, b3);
+            }
+          }
+          // ---- online softmax of rows g (elements 0, 1) and g + 8 (2, 3)
+          float alpha[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const bool act = h == 0 ? act0 : act1;
+            float x[4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+              for (int e = 0; e < 2; ++e) {
+                const int key = kt * 16 + nt * 8 + 2 * tig + e;
+                const float v = (s[nt][2 * h + e] + so[nt][2 * h + e]) * a.sl2;
+                x[2 * nt + e] = (full || (act && key < valid)) ? v : -INFINITY;
+              }
+            float bm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+            const float mn = fmaxf(m_run[h], bm);
+            alpha[h] = mn == -INFINITY ? 1.f : fast_exp2(m_run[h] - mn);
+            m_run[h] = mn;
+            float ps = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              x[e] = x[e] == -INFINITY ? 0.f : fast_exp2(x[e] - mn);
+              ps += x[e];
+            }
+            l_run[h] = l_run[h] * alpha[h] + ps;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+              s[nt][2 * h] = x[2 * nt];
+              s[nt][2 * h + 1] = x[2 * nt + 1];
+            }
+          }
+#pragma unroll
+          for (int n = 0; n < kNT; ++n) {
+            acc[n][0] *= alpha[0];
+            acc[n][1] *= alpha[0];
+            acc[n][2] *= alpha[1];
+            acc[n][3] *= alpha[1];
+          }
+          // ---- P as the A operand (16 rows x 16 keys): the S accumulator
+          // layout of two n-tiles is the A fragment layout.  bf16 keeps P as
+          // hi + lo parts: one bf16 value (8 significant bits) errs by up to
+          // 2^-9 of a weight, which outputs formed by cancellation cannot
+          // absorb; fp16 P keeps 11 bits and stays one part.
+          uint32_t pa[4], pl[4];
+          pa[0] = pack2<kBF16>(s[0][0], s[0][1]);
+          pa[1] = pack2<kBF16>(s[0][2], s[0][3]);
+          pa[2] = pack2<kBF16>(s[1][0], s[1][1]);
+          pa[3] = pack2<kBF16>(s[1][2], s[1][3]);
+          if constexpr (kBF16) {
+            pl[0] = pack_bf16x2(s[0][0] - to_float<true>(pa[0] & 0xffff), s[0][1] - to_float<true>(pa[0] >> 16));
+            pl[1] = pack_bf16x2(s[0][2] - to_float<true>(pa[1] & 0xffff), s[0][3] - to_float<true>(pa[1] >> 16));
+            pl[2] = pack_bf16x2(s[1][0] - to_float<true>(pa[2] & 0xffff), s[1][1] - to_float<true>(pa[2] >> 16));
+            pl[3] = pack_bf16x2(s[1][2] - to_float<true>(pa[3] & 0xffff), s[1][3] - to_float<true>(pa[3] >> 16));
+          }
+          // ---- O += P V: B = V (keys x dims) through ldmatrix.trans.  Keys
+          // past the member's length (the end of its last block) may hold
+          // anything, NaN included: their values are zeroed here.
+          uint32_t m_lo = 0xffffffffu, m_hi = 0xffffffffu;  // keys 2tig(+1), 2tig+8(+9)
+          if (valid < BS) {
+            const int tk = kt * 16 + 2 * tig;
+            m_lo = pair_mask(tk < valid, tk + 1 < valid);
+            m_hi = pair_mask(tk + 8 < valid, tk + 9 < valid);
+          }
+          const int vkey = kt * 16 + (li & 1) * 8 + (lane & 7);
+#pragma unroll
+          for (int n2 = 0; n2 < D / 16; ++n2) {
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_trans(sV + tile_off<C>(vkey, (n2 * 16 + (li >> 1) * 8) * 2), b0, b1, b2, b3);
+            b0 &= m_lo; b1 &= m_hi; b2 &= m_lo; b3 &= m_hi;
+            mma_16816<kBF16>(acc[2 * n2], pa, b0, b1);
+            mma_16816<kBF16>(acc[2 * n2 + 1], pa, b2, b3);
+            if constexpr (kBF16) {
+              mma_16816<kBF16>(acc[2 * n2], pl, b0, b1);
+              mma_16816<kBF16>(acc[2 * n2 + 1], pl, b2, b3);
+            }
+          }
+        }
+      }
+      __syncwarp();
+      ++n_consumed;
+      if (!failed && i + kStages < nb_w) issue(i + kStages);
+    }
+
+    // ---- merge the warps' states through shared memory (the rings are
+    // idle: every load of this item has been consumed)
+    {
+      float* scr = reinterpret_cast<float*>(ring + warp * C::kWarpBytes);
+      float lsum[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        float v = l_run[h];
+        v += __shfl_xor_sync(0xffffffffu, v, 1);
+        v += __shfl_xor_sync(0xffffffffu, v, 2);
+        lsum[h] = v;
+      }
+#pragma unroll
+      for (int n = 0; n < kNT; ++n) {
+        const int d = n * 8 + 2 * tig;
+        *reinterpret_cast<float2*>(scr + g * D + d) = make_float2(acc[n][0], acc[n][1]);
+        *reinterpret_cast<float2*>(scr + (g + 8) * D + d) = make_float2(acc[n][2], acc[n][3]);
+      }
+      if (tig == 0) {
+        scr[kRows * D + g] = m_run[0];
+        scr[kRows * D + g + 8] = m_run[1];
+        scr[kRows * D + kRows + g] = lsum[0];
+        scr[kRows * D + kRows + g + 8] = lsum[1];
+      }
+    }
+    __syncthreads();
+    {
+      constexpr int kVec = 8;
+      const int units = rows * (D / kVec);
+      for (int u = threadIdx.x; u < units; u += kDecodeThreads) {
+        const int r = u / (D / kVec);
+        const int d0 = (u % (D / kVec)) * kVec;
+        float mw[kDecodeWarps];
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kDecodeWarps; ++w) {
+          const float* scr = reinterpret_cast<const float*>(ring + w * C::kWarpBytes);
+          mw[w] = scr[kRows * D + r];
+          M = fmaxf(M, mw[w]);
+        }
+        float o[kVec];
+#pragma unroll
+        for (int v = 0; v < kVec; ++v) o[v] = 0.f;
+        float L = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+          for (int w = 0; w < kDecodeWarps; ++w) {
+            const float* scr = reinterpret_cast<const float*>(ring + w * C::kWarpBytes);
+            const float f = fast_exp2(mw[w] - M);
+            L += f * scr[kRows * D + kRows + r];
+            const float4 x0 = *reinterpret_cast<const float4*>(scr + r * D + d0);
+            const float4 x1 = *reinterpret_cast<const float4*>(scr + r * D + d0 + 4);
+            o[0] += f * x0.x; o[1] += f * x0.y; o[2] += f * x0.z; o[3] += f * x0.w;
+            o[4] += f * x1.x; o[5] += f * x1.y; o[6] += f * x1.z; o[7] += f * x1.w;
+          }
+          const float inv = 1.f / L;
+#pragma unroll
+          for (int v = 0; v < kVec; ++v) o[v] *= inv;
+        }
+        if (nranges == 1) {
+          const int64_t qh = static_cast<int64_t>(s_seq[r / a.group]) * a.hq + kvh * a.group +
+                             r % a.group;
+          uint4 pk;
+          pk.x = pack2<kBF16>(o[0], o[1]);
+          pk.y = pack2<kBF16>(o[2], o[3]);
+          pk.z = pack2<kBF16>(o[4], o[5]);
+          pk.w = pack2<kBF16>(o[6], o[7]);
+          *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.out) + qh * D + d0) = pk;
+        } else {
+          const int64_t pi = (static_cast<int64_t>(slot0 + range) * a.hkv + kvh) * kRows + r;
+          float* op = a.o_part + pi * D + d0;
+          *reinterpret_cast<float4*>(op) = make_float4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<float4*>(op + 4) = make_float4(o[4], o[5], o[6], o[7]);
+          if (d0 == 0) a.lse_part[pi] = (M == -INFINITY) ? -INFINITY : M + log2f(L);
+        }
+      }
+    }
+    if (nranges > 1) {
+      // the CTA that finishes the chunk's last range merges every range:
+      // out = sum_i w_i o_i / sum_i w_i, w_i = 2^(lse_i - max lse); partials
+      // are published with a fence before the arrival count, read through L2
+      __threadfence();
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        const int prev = atomicAdd(&a.arrived[chunk * a.hkv + kvh], 1);
+        s_flag = (prev == nranges - 1) ? 1 : 0;
+      }
+      __syncthreads();
+      if (s_flag) {
+        __threadfence();
+        float* w_s = reinterpret_cast<float*>(ring);   // [nranges][16] weights
+        float* wsum_s = w_s + nranges * kRows;         // [16]
+        const int64_t base = (static_cast<int64_t>(slot0) * a.hkv + kvh) * kRows;
+        const int64_t rstride = static_cast<int64_t>(a.hkv) * kRows;  // between ranges
+        for (int k2 = threadIdx.x; k2 < nranges * rows; k2 += kDecodeThreads) {
+          const int i = k2 / rows, r = k2 % rows;
+          w_s[i * kRows + r] = __ldcg(a.lse_part + base + i * rstride + r);
+        }
+        __syncthreads();
+        for (int r = warp; r < rows; r += kDecodeWarps) {
+          float M = -INFINITY;
+          for (int i = lane; i < nranges; i += 32) M = fmaxf(M, w_s[i * kRows + r]);
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+          float W = 0.f;
+          for (int i = lane; i < nranges; i += 32) {
+            const float w = (M == -INFINITY) ? 0.f : fast_exp2(w_s[i * kRows + r] - M);
+            w_s[i * kRows + r] = w;
+            W += w;
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) W += __shfl_xor_sync(0xffffffffu, W, o);
+          if (lane == 0) wsum_s[r] = W;
+        }
+        __syncthreads();
+        constexpr int kVec = 4;
+        const int units = rows * (D / kVec);
+        for (int u = threadIdx.x; u < units; u += kDecodeThreads) {
+          const int r = u / (D / kVec);
+          const int d0 = (u % (D / kVec)) * kVec;
+          float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+          const float* op = a.o_part + (base + r) * D + d0;
+#pragma unroll 8
+          for (int i = 0; i < nranges; ++i) {
+            const float w = w_s[i * kRows + r];
+            const float4 x = __ldcg(reinterpret_cast<const float4*>(op + i * rstride * D));
+            o0 += w * x.x; o1 += w * x.y; o2 += w * x.z; o3 += w * x.w;
+          }
+          const float W = wsum_s[r];
+          const float inv = W > 0.f ? 1.f / W : 0.f;
+          const int64_t qh = static_cast<int64_t>(s_seq[r / a.group]) * a.hq + kvh * a.group +
+                             r % a.group;
+          uint2 pk;
+          pk.x = pack2<kBF16>(o0 * inv, o1 * inv);
+          pk.y = pack2<kBF16>(o2 * inv, o3 * inv);
+          *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.out) + qh * D + d0) = pk;
+        }
+      }
+    }
+    if (threadIdx.x == 0) s_item = atomicAdd(a.counter, 1);
+    __syncthreads();           // scratch (= stage memory) and s_seq free again ...
+    fence_proxy_async_smem();  // ... before the next item's tile loads
+  }
+
+  if (failed) {  // drain copies still in flight after a timeout (bounded again)
+    while (n_consumed < n_issued) {
+      const int st = n_consumed % kStages;
+      mbar_wait_bounded(bar0 + 8 * st, (n_consumed / kStages) & 1u);
+      ++n_consumed;
+    }
+  }
+}
+
+
+// ------------------------------------------------------------- planning
+// One CTA of 1024 threads, once per call:
+//  1. members are counted; a sequence listed twice, or outside [0, B),
+//     invalidates every group holding it (those decode plainly; reported);
+//  2. one warp per group: the shared blocks P = the longest run of leading
+//     table entries equal in every member's row, cut so that every member
+//     keeps at least one token of its own (P * bs <= len - 1).  Groups of
+//     one member, or with a length outside [1, max_ctx], share nothing.  A
+//     group with P > 0 becomes chunks of up to 16 / G members;
+//  3. every other sequence is a chunk of its own (P = 0); a length outside
+//     [0, min(max_ctx, max_blocks * bs)] counts as 0 and is reported;
+//  4. virtual lengths V (blocks), then the range length R = the largest of
+//     r_floor, T * Hkv / kCascadeTargetItems (T = all chunks' blocks) and
+//     max V / kCascadeMaxRanges; a chunk is cut into ceil(V / R) ranges of
+//     equal length, each with its partial slot;
+//  5. the (chunk, range) work list, the item count, arrival counters and the
+//     work counter.
+// Chunk and slot numbers come from atomics (their order varies), but every
+// output depends only on its chunk's ranges, merged in range order: results
+// are the same from call to call.
+__global__ void __launch_bounds__(1024) cascade_plan_kernel(
+    const int32_t* __restrict__ ctx_lens, const int32_t* __restrict__ block_tables,
+    const int32_t* __restrict__ group_start, const int32_t* __restrict__ group_seqs,
+    int num_groups, int B, int max_ctx, int max_blocks, int bs, int group, int hkv, int r_floor,
+    int32_t* seen, int32_t* chunk_seqs, int4* chunks, int2* items, int32_t* total,
+    int32_t* counter, int32_t* arrived) {
+  __shared__ int n_chunks, n_used, tv_sum, v_max, n_items;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) {
+    n_chunks = n_used = tv_sum = v_max = n_items = 0;
+    *counter = 0;
+  }
+  for (int s = tid; s < B; s += 1024) seen[s] = 0;
+  __syncthreads();
+  const int n_members = num_groups > 0 ? group_start[num_groups] : 0;
+  for (int i = tid; i < n_members; i += 1024) {
+    const int m = group_seqs[i];
+    if (m >= 0 && m < B) atomicAdd(&seen[m], 1);
+  }
+  __syncthreads();
+  const int per_chunk = max(1, kCascadeRows / group);
+  for (int gi = warp; gi < num_groups; gi += 32) {
+    const int m0 = group_start[gi], m1 = group_start[gi + 1];
+    const int k = m1 - m0;
+    const bool listed = k >= 2 && m0 >= 0 && m1 <= n_members;  // a well-formed range
+    int limit = 1 << 30;
+    int bad = 0;
+    for (int i = m0 + lane; listed && i < m1; i += 32) {
+      const int m = group_seqs[i];
+      if (m < 0 || m >= B || seen[m] != 1) {
+        bad = 1;
+        continue;
+      }
+      const int c = ctx_lens[m];
+      if (c < 1 || c > max_ctx || c > max_blocks * bs) bad = 1;
+      else limit = min(limit, (c - 1) / bs);
+    }
+    const bool any_bad = __any_sync(0xffffffffu, bad);
+    if (lane == 0 && k >= 2 && (!listed || any_bad)) record_error(PA_ERR_RANGE);
+    if (!listed || any_bad) continue;
+    limit = __reduce_min_sync(0xffffffffu, limit);
+    // first table index below limit where some member differs from the first
+    const int32_t* lead = block_tables + static_cast<int64_t>(group_seqs[m0]) * max_blocks;
+    int first_diff = limit;
+    for (int j = lane; j < limit; j += 32) {
+      const int e = lead[j];
+      bool same = true;
+      for (int i = m0 + 1; i < m1; ++i)
+        same &= block_tables[static_cast<int64_t>(group_seqs[i]) * max_blocks + j] == e;
+      if (!same) {
+        first_diff = j;
+        break;
+      }
+    }
+    const int P = __reduce_min_sync(0xffffffffu, first_diff);
+    if (P <= 0) continue;
+    const int nch = (k + per_chunk - 1) / per_chunk;
+    int cbase = 0, mbase = 0;
+    if (lane == 0) {
+      cbase = atomicAdd(&n_chunks, nch);
+      mbase = atomicAdd(&n_used, k);
+    }
+    cbase = __shfl_sync(0xffffffffu, cbase, 0);
+    mbase = __shfl_sync(0xffffffffu, mbase, 0);
+    for (int i = lane; i < k; i += 32) {
+      const int m = group_seqs[m0 + i];
+      chunk_seqs[mbase + i] = m;
+      seen[m] = -1;  // claimed
+    }
+    for (int c = lane; c < nch; c += 32)
+      chunks[2 * (cbase + c)] = make_int4(mbase + c * per_chunk, min(per_chunk, k - c * per_chunk), P, 0);
+  }
+  __syncthreads();
+  for (int s = tid; s < B; s += 1024) {
+    if (seen[s] == -1) continue;
+    const int c = atomicAdd(&n_chunks, 1);
+    const int m = atomicAdd(&n_used, 1);
+    chunk_seqs[m] = s;
+    chunks[2 * c] = make_int4(m, 1, 0, 0);
+  }
+  __syncthreads();
+  const int nc = n_chunks;
+  for (int c = tid; c < nc; c += 1024) {
+    const int4 d = chunks[2 * c];
+    int V = d.z;
+    for (int i = 0; i < d.y; ++i) {
+      int len = ctx_lens[chunk_seqs[d.x + i]];
+      if (len < 0 || len > max_ctx || len > max_blocks * bs) {  // only unshared ones get here
+        record_error(PA_ERR_DEVICE_BOUNDS);
+        len = 0;
+      }
+      V += (len + bs - 1) / bs - d.z;
+    }
+    chunks[2 * c + 1] = make_int4(V, 0, 0, 0);
+    atomicAdd(&tv_sum, V);
+    atomicMax(&v_max, V);
+  }
+  __syncthreads();
+  const int R = max(max(r_floor, 1),
+                    max(static_cast<int>((static_cast<int64_t>(tv_sum) * hkv + kCascadeTargetItems - 1) /
+                                         kCascadeTargetItems),
+                        (v_max + kCascadeMaxRanges - 1) / kCascadeMaxRanges));
+  for (int c = tid; c < nc; c += 1024) {
+    const int V = chunks[2 * c + 1].x;
+    const int nr = max(1, (V + R - 1) / R);
+    const int rc = V > 0 ? (V + nr - 1) / nr : 1;  // equal ranges of at most R blocks
+    const int slot0 = atomicAdd(&n_items, nr);    // one slot per range
+    chunks[2 * c].w = slot0;
+    chunks[2 * c + 1] = make_int4(V, nr, rc, 0);
+    for (int r = 0; r < nr; ++r) items[slot0 + r] = make_int2(c, r);
+    for (int h = 0; h < hkv; ++h) arrived[c * hkv + h] = 0;
+  }
+  __syncthreads();
+  if (tid == 0) *total = n_items;
+}
+
+}  // namespace pa

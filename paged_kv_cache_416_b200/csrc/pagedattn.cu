@@ -12,6 +12,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "prefill.cuh"
+#include "cascade.cuh"
 
 namespace {
 
@@ -115,6 +116,38 @@ WsLayout ws_layout(int32_t B, int32_t hq, int32_t hkv, int32_t D, int32_t max_ct
   return w;
 }
 
+// Shared-prefix (cascade) decode workspace: work counter and item count,
+// then seen [B], chunk members [B], chunk descriptors [2B] int4, the work
+// list [slots] int2, arrival counters [B * Hkv], and the partials: fp32 lse
+// [slots * Hkv * 16] and fp32 outputs [slots * Hkv * 16 * D].  Slots are
+// bounded through the shortest range r_floor: at most B * max_blocks /
+// r_floor + B (a chunk of V blocks takes max(1, ceil(V / R)) <= V / R + 1).
+struct CascadeWs {
+  size_t counter = 0, total = 4, seen = 256, chunk_seqs = 0, chunks = 0, items = 0, arrived = 0,
+         lse = 0, o = 0, bytes = 0;
+  int32_t r_floor = 1;
+  int64_t slots = 0;
+};
+
+CascadeWs cascade_ws_layout(int32_t B, int32_t hkv, int32_t D, int32_t bs, int32_t max_ctx,
+                            int32_t split_tokens) {
+  CascadeWs w;
+  const int64_t max_nb = std::max<int64_t>(1, cdiv(max_ctx, bs));
+  const int64_t auto_floor = cdiv(static_cast<int64_t>(B) * max_nb * hkv, 4 * pa::kCascadeTargetItems);
+  const int64_t user_floor = split_tokens > 0 ? cdiv(split_tokens, bs) : 1;
+  w.r_floor = static_cast<int32_t>(std::max<int64_t>(std::max<int64_t>(4, auto_floor), user_floor));
+  w.slots = cdiv(static_cast<int64_t>(B) * max_nb, w.r_floor) + B;
+  const size_t arr = static_cast<size_t>(round_up(static_cast<int64_t>(B) * 4, 256));
+  w.chunk_seqs = w.seen + arr;
+  w.chunks = w.chunk_seqs + arr;
+  w.items = w.chunks + static_cast<size_t>(round_up(static_cast<int64_t>(B) * 32, 256));
+  w.arrived = w.items + static_cast<size_t>(round_up(w.slots * 8, 256));
+  w.lse = w.arrived + static_cast<size_t>(round_up(static_cast<int64_t>(B) * hkv * 4, 256));
+  w.o = w.lse + static_cast<size_t>(round_up(w.slots * hkv * pa::kCascadeRows * 4, 256));
+  w.bytes = w.o + static_cast<size_t>(w.slots * hkv * pa::kCascadeRows * D * 4);
+  return w;
+}
+
 // --------------------------------------------------------- tensor maps
 // cuTensorMapEncodeTiled is a driver entry point; it is fetched through the
 // runtime so the library needs no link-time dependency on libcuda.
@@ -196,6 +229,37 @@ pa_status dispatch_shape(const pa::DecodeArgs& a, int D, int BS, int64_t items, 
   if (D == 128 && BS == 32) return launch_decode_main<CK, kQBF16, 128, 32>(a, items, dev, st);
   if (D == 64 && BS == 16) return launch_decode_main<CK, kQBF16, 64, 16>(a, items, dev, st);
   if (D == 64 && BS == 32) return launch_decode_main<CK, kQBF16, 64, 32>(a, items, dev, st);
+  return fail(PA_ERR_SHAPE, "head_dim %d / block_size %d not supported", D, BS);
+}
+
+template <bool kBF16, int D, int BS>
+pa_status launch_cascade(const pa::CascadeArgs& args, int64_t items_upper, int dev,
+                         cudaStream_t stream) {
+  using C = pa::DecodeCfg<kBF16 ? pa::kCacheBF16 : pa::kCacheF16, D, BS>;
+  auto kern = pa::cascade_kernel<kBF16, D, BS>;
+  static int occ[kMaxDevices] = {0};
+  if (occ[dev] == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(cascade)");
+    int n = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, pa::kDecodeThreads, C::kSmemBytes);
+    if (e != cudaSuccess) return cuda_fail(e, "occupancy(cascade)");
+    occ[dev] = n > 0 ? n : 1;
+  }
+  const int64_t grid = std::max<int64_t>(
+      1, std::min<int64_t>(items_upper, static_cast<int64_t>(device_sms(dev)) * occ[dev]));
+  kern<<<static_cast<unsigned>(grid), pa::kDecodeThreads, C::kSmemBytes, stream>>>(args);
+  return PA_OK;
+}
+
+template <bool kBF16>
+pa_status dispatch_cascade(const pa::CascadeArgs& a, int D, int BS, int64_t items, int dev,
+                           cudaStream_t st) {
+  if (D == 128 && BS == 16) return launch_cascade<kBF16, 128, 16>(a, items, dev, st);
+  if (D == 128 && BS == 32) return launch_cascade<kBF16, 128, 32>(a, items, dev, st);
+  if (D == 64 && BS == 16) return launch_cascade<kBF16, 64, 16>(a, items, dev, st);
+  if (D == 64 && BS == 32) return launch_cascade<kBF16, 64, 32>(a, items, dev, st);
   return fail(PA_ERR_SHAPE, "head_dim %d / block_size %d not supported", D, BS);
 }
 
@@ -448,6 +512,103 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_po
   if (s != PA_OK) return s;
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
+  return ok();
+}
+
+size_t pa_decode_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_heads,
+                                              int32_t num_kv_heads, int32_t head_dim,
+                                              int32_t block_size, int32_t max_context_len,
+                                              int32_t split_tokens) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || (head_dim != 64 && head_dim != 128) ||
+      (block_size != 16 && block_size != 32) || max_context_len < 0 || split_tokens < 0)
+    return 0;
+  return cascade_ws_layout(num_seqs, num_kv_heads, head_dim, block_size, max_context_len,
+                           split_tokens).bytes;
+}
+
+pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype q_dtype, const void* k_pool,
+                                  const void* v_pool, pa_dtype cache_dtype,
+                                  const int32_t* block_tables, int32_t max_blocks_per_seq,
+                                  const int32_t* context_lens, int32_t max_context_len,
+                                  const int32_t* group_start, const int32_t* group_seqs,
+                                  int32_t num_groups, int32_t num_seqs, int32_t num_q_heads,
+                                  int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                                  int32_t num_blocks, float scale, int32_t split_tokens,
+                                  void* workspace, size_t workspace_bytes, pa_stream_t stream) {
+  if (!valid_dtype(q_dtype) || !valid_dtype(cache_dtype))
+    return fail(PA_ERR_DTYPE, "pa_decode_shared_prefix: unknown dtype");
+  if (cache_dtype == PA_FP8_E4M3 || q_dtype != cache_dtype)
+    return fail(PA_ERR_DTYPE, "pa_decode_shared_prefix: q and cache must both be f16 or both bf16");
+  if (num_seqs < 0 || num_groups < 0 || max_blocks_per_seq <= 0 || max_context_len < 0 ||
+      split_tokens < 0 || !cache_shape_ok(num_blocks, block_size, num_kv_heads, head_dim))
+    return fail(PA_ERR_SHAPE, "pa_decode_shared_prefix: unsupported sizes (seqs %d, groups %d, "
+                "max_blocks %d, max_ctx %d, blocks %d, bs %d, kv heads %d, dim %d)", num_seqs,
+                num_groups, max_blocks_per_seq, max_context_len, num_blocks, block_size,
+                num_kv_heads, head_dim);
+  if (static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * block_size)
+    return fail(PA_ERR_SHAPE, "pa_decode_shared_prefix: max_context_len %d exceeds "
+                "max_blocks_per_seq * bs", max_context_len);
+  if (num_q_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
+      num_q_heads / num_kv_heads > pa::kMaxGroup)
+    return fail(PA_ERR_HEADS, "pa_decode_shared_prefix: num_q_heads %d must be a multiple of "
+                "num_kv_heads %d with at most %d query heads per kv head", num_q_heads,
+                num_kv_heads, pa::kMaxGroup);
+  if (!std::isfinite(scale)) return fail(PA_ERR_SHAPE, "pa_decode_shared_prefix: scale must be finite");
+  if (num_seqs == 0) return ok();
+  if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens ||
+      (num_groups > 0 && (!group_start || !group_seqs)))
+    return fail(PA_ERR_NULL, "pa_decode_shared_prefix: null pointer");
+  const CascadeWs w = cascade_ws_layout(num_seqs, num_kv_heads, head_dim, block_size,
+                                        max_context_len, split_tokens);
+  if (!workspace || workspace_bytes < w.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return fail(PA_ERR_WORKSPACE, "pa_decode_shared_prefix: workspace needs %zu bytes, 256-byte "
+                "aligned (got %zu)", w.bytes, workspace_bytes);
+  if ((reinterpret_cast<uintptr_t>(k_pool) | reinterpret_cast<uintptr_t>(v_pool)) & 15)
+    return fail(PA_ERR_SHAPE, "pa_decode_shared_prefix: the pools must be 16-byte aligned");
+  int dev;
+  if (current_device(&dev)) return fail(PA_ERR_CUDA, "pa_decode_shared_prefix: no current device");
+  auto st = reinterpret_cast<cudaStream_t>(stream);
+  auto* ws = static_cast<uint8_t*>(workspace);
+
+  pa::CascadeArgs a;
+  pa_status ms = encode_pool_map(&a.tmap_k, k_pool, num_blocks, block_size, num_kv_heads,
+                                 head_dim, elem_bytes(cache_dtype));
+  if (ms == PA_OK)
+    ms = encode_pool_map(&a.tmap_v, v_pool, num_blocks, block_size, num_kv_heads, head_dim,
+                         elem_bytes(cache_dtype));
+  if (ms != PA_OK) return ms;
+  a.out = out;
+  a.q = q;
+  a.block_tables = block_tables;
+  a.context_lens = context_lens;
+  a.chunk_seqs = reinterpret_cast<const int32_t*>(ws + w.chunk_seqs);
+  a.chunks = reinterpret_cast<const int4*>(ws + w.chunks);
+  a.items = reinterpret_cast<const int2*>(ws + w.items);
+  a.total = reinterpret_cast<const int32_t*>(ws + w.total);
+  a.counter = reinterpret_cast<int32_t*>(ws + w.counter);
+  a.arrived = reinterpret_cast<int32_t*>(ws + w.arrived);
+  a.lse_part = reinterpret_cast<float*>(ws + w.lse);
+  a.o_part = reinterpret_cast<float*>(ws + w.o);
+  a.hq = num_q_heads;
+  a.hkv = num_kv_heads;
+  a.group = num_q_heads / num_kv_heads;
+  a.max_blocks = max_blocks_per_seq;
+  a.num_blocks = num_blocks;
+  a.sl2 = scale * 1.4426950408889634f;
+
+  pa::cascade_plan_kernel<<<1, 1024, 0, st>>>(
+      context_lens, block_tables, group_start, group_seqs, num_groups, num_seqs, max_context_len,
+      max_blocks_per_seq, block_size, a.group, num_kv_heads, w.r_floor,
+      reinterpret_cast<int32_t*>(ws + w.seen), reinterpret_cast<int32_t*>(ws + w.chunk_seqs),
+      reinterpret_cast<int4*>(ws + w.chunks), reinterpret_cast<int2*>(ws + w.items),
+      reinterpret_cast<int32_t*>(ws + w.total), a.counter, a.arrived);
+  const int64_t items_upper = w.slots * num_kv_heads;
+  const pa_status s = cache_dtype == PA_BF16
+                          ? dispatch_cascade<true>(a, head_dim, block_size, items_upper, dev, st)
+                          : dispatch_cascade<false>(a, head_dim, block_size, items_upper, dev, st);
+  if (s != PA_OK) return s;
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "pa_decode_shared_prefix launch");
   return ok();
 }
 

@@ -53,6 +53,9 @@ def declare(lib: ctypes.CDLL) -> ctypes.CDLL:
         "pa_decode_workspace_size": (SZ, [I32, I32, I32, I32, I32, I32, I32]),
         "pa_decode": (I32, [P, P, I32, P, P, I32, P, I32, P, I32, I32, I32, I32, I32, I32, I32,
                             F, F, F, I32, P, SZ, P]),
+        "pa_decode_shared_prefix_workspace_size": (SZ, [I32, I32, I32, I32, I32, I32, I32]),
+        "pa_decode_shared_prefix": (I32, [P, P, I32, P, P, I32, P, I32, P, I32, P, P, I32, I32,
+                                          I32, I32, I32, I32, I32, F, I32, P, SZ, P]),
         "pa_sync_status": (I32, [P]),
         "pa_last_error": (ctypes.c_char_p, []),
         "pa_validate_slot_mapping": (I32, [P, I32, I32, I32, P]),
@@ -87,6 +90,8 @@ pa_prefill = _lib.pa_prefill
 pa_decode_split_tokens = _lib.pa_decode_split_tokens
 pa_decode_workspace_size = _lib.pa_decode_workspace_size
 pa_decode = _lib.pa_decode
+pa_decode_shared_prefix_workspace_size = _lib.pa_decode_shared_prefix_workspace_size
+pa_decode_shared_prefix = _lib.pa_decode_shared_prefix
 pa_sync_status = _lib.pa_sync_status
 pa_last_error = _lib.pa_last_error
 pa_validate_slot_mapping = _lib.pa_validate_slot_mapping
@@ -101,6 +106,7 @@ ENTRY_POINTS = [
     "pa_write_kv", "pa_copy_blocks", "pa_swap_blocks", "pa_hash_blocks", "pa_decode_split_tokens", "pa_decode_workspace_size",
     "pa_decode", "pa_prefill", "pa_sync_status", "pa_last_error", "pa_validate_slot_mapping",
     "pa_validate_copy_pairs", "pa_validate_block_tables", "pa_decode_noalloc",
+    "pa_decode_shared_prefix_workspace_size", "pa_decode_shared_prefix",
 ]
 
 
@@ -236,6 +242,37 @@ def decode(q, k_pool, v_pool, block_tables, context_lens, scale: float, max_cont
                     int(max_context_len), B, hq, hkv, d, bs, N, float(scale), float(k_scale),
                     float(v_scale), int(split_tokens), _ptr(workspace), workspace.numel(),
                     _stream(stream)))
+    return out
+
+
+def shared_prefix_workspace_size(num_seqs, hq, hkv, head_dim, bs, max_context_len,
+                                 split_tokens=0) -> int:
+    return int(pa_decode_shared_prefix_workspace_size(num_seqs, hq, hkv, head_dim, bs,
+                                                      int(max_context_len), int(split_tokens)))
+
+
+def decode_shared_prefix(q, k_pool, v_pool, block_tables, context_lens, group_start, group_seqs,
+                         scale: float, max_context_len: int, split_tokens: int = 0, out=None,
+                         workspace=None, stream=None) -> torch.Tensor:
+    """pa_decode_shared_prefix on tensors: pa_decode's arguments plus the
+    groups (group_start int32 [G + 1], group_seqs int32 [group_start[G]]),
+    16-bit caches.  Returns out [B, Hq, D]."""
+    _contig(q, k_pool, v_pool, block_tables, context_lens, group_start, group_seqs)
+    for t in (block_tables, context_lens, group_start, group_seqs):
+        if t.dtype != torch.int32:
+            raise TypeError("block_tables, context_lens and the group arrays must be int32")
+    B, hq, d = q.shape
+    N, bs, hkv, _ = k_pool.shape
+    if out is None:
+        out = torch.empty_like(q)
+    nbytes = shared_prefix_workspace_size(B, hq, hkv, d, bs, max_context_len, split_tokens)
+    if workspace is None:
+        workspace = workspace_for(q.device, nbytes)
+    check(pa_decode_shared_prefix(
+        _ptr(out), _ptr(q), _dtype(q), _ptr(k_pool), _ptr(v_pool), _dtype(k_pool),
+        _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), int(max_context_len),
+        _ptr(group_start), _ptr(group_seqs), group_start.shape[0] - 1, B, hq, hkv, d, bs, N,
+        float(scale), int(split_tokens), _ptr(workspace), workspace.numel(), _stream(stream)))
     return out
 
 
