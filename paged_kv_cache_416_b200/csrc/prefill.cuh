@@ -52,7 +52,7 @@
 namespace pa {
 
 constexpr int kPfRowThreads = 128;  // warps 0-3: thread r owns query row r (TMEM lane r)
-constexpr int kPfThreads = 160;     // + warp 4: loads and MMA issue
+constexpr int kPfThreads = 192;     // + warp 4: MMA issue, warp 5: TMA loads
 constexpr int kPfRows = 128;      // MMA M: (token, head) rows per CTA
 constexpr int kPfKeys = 64;       // keys per tile
 constexpr int kPfD = 128;         // head_dim
@@ -68,7 +68,7 @@ struct PrefillCfg {
   static constexpr int kOffK = kOffQ + kQBytes;           // 2 stages
   static constexpr int kOffV = kOffK + 2 * kKBytes;       // 2 stages
   static constexpr int kTiles = kOffV + 2 * kKBytes;      // 96 KiB: two CTAs per SM
-  static constexpr int kHead = 256;                       // 8 mbarriers, TMEM slot
+  static constexpr int kHead = 256;                       // 12 mbarriers, TMEM slot, block ids
   static constexpr int kSmemBytes = kTiles + kHead;
   static_assert(kPfKeys % BS == 0, "a key tile holds whole blocks");
 };
@@ -99,7 +99,8 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
   using C = PrefillCfg<BS>;
   extern __shared__ __align__(1024) uint8_t pf_smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool producer = warp == kPfRowThreads / 32;
+  const bool producer = warp >= kPfRowThreads / 32;     // warps 4 (MMA) and 5 (loads)
+  const bool mma_warp = warp == kPfRowThreads / 32;
   const int s = blockIdx.z, kvh = blockIdx.y;
   const int G = a.group;
   const int T = kPfRows / G;  // query tokens per CTA
@@ -127,14 +128,18 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
   const int nkt = (kend - 1) / kPfKeys + 1;
   const int32_t* table = a.block_tables + static_cast<int64_t>(s) * a.max_blocks;
 
-  // [tiles (1024-aligned) | mbarriers | TMEM slot]
+  // [tiles (1024-aligned) | mbarriers | TMEM slot | block ids of 4 key tiles]
   const uint32_t base_s = smem_addr(pf_smem);
   uint8_t* const base = pf_smem;
   const uint32_t head_s = base_s + C::kTiles;
   const uint32_t full_k = head_s, full_v = head_s + 16;  // + 8 * stage, TMA
   const uint32_t bar_s = head_s + 32, bar_o = head_s + 40;  // MMA commits
   const uint32_t s_free = head_s + 48, p_ready = head_s + 56;  // one arrival per row warp
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(base + C::kTiles + 64);
+  const uint32_t k_empty = head_s + 64, v_empty = head_s + 80;  // + 8 * stage, MMA commits
+  const uint32_t tmem_slot_s = head_s + 96;  // tcgen05.alloc writes the TMEM address here
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(base + C::kTiles + 96);
+  // the loader's block ids of key tile kt (K issue writes, V issue reads)
+  int* const s_phys = reinterpret_cast<int*>(base + C::kTiles + 128);  // [4][kBlocksPerTile]
   const uint32_t sQ = base_s + C::kOffQ, sK = base_s + C::kOffK, sV = base_s + C::kOffV;
   if (base_s & 1023) {  // the swizzled tiles need a 1024-byte aligned start
     if (tid == 0) record_error(PA_ERR_DEVICE_BOUNDS);
@@ -149,18 +154,15 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     const int p = table[j];
     return (p >= 0 && p < a.num_blocks) ? p : -2;
   };
-  // producer lane 0: TMA loads of one K or V tile into its stage (one box
-  // per block and dim half); blocks past the context or with a bad entry are
-  // not loaded
-  auto issue_tile = [&](int kt, bool is_v) {
+  // loader lane 0: TMA loads of one K or V tile into its stage (one box per
+  // block and dim half); blocks past the context or with a bad entry
+  // (phys < 0) are not loaded
+  auto issue_tile = [&](int kt, bool is_v, const int* phys) {
     const int st = kt & 1;
-    int phys[C::kBlocksPerTile];
     uint32_t bytes = 0;
 #pragma unroll
-    for (int b = 0; b < C::kBlocksPerTile; ++b) {
-      phys[b] = tile_block(kt, b);
+    for (int b = 0; b < C::kBlocksPerTile; ++b)
       if (phys[b] >= 0) bytes += 2u * BS * 128u;
-    }
     const uint32_t bar = (is_v ? full_v : full_k) + 8 * st;
     const uint32_t dst = (is_v ? sV : sK) + st * C::kKBytes;
     const CUtensorMap* map = is_v ? &a.tmap_v : &a.tmap_k;
@@ -174,20 +176,27 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     }
   };
 
-  if (producer && lane == 0) {
+  if (producer && !mma_warp && lane == 0) {
     for (int i = 0; i < 6; ++i) mbar_init(head_s + 8 * i, 1);
     mbar_init(s_free, kPfRowThreads / 32);
     mbar_init(p_ready, kPfRowThreads / 32);
+    for (int i = 0; i < 4; ++i) mbar_init(k_empty + 8 * i, 1);  // k_empty[2], v_empty[2]
     mbar_init_fence();
     prefetch_tensormap(&a.tmap_k);
     prefetch_tensormap(&a.tmap_v);
     for (int kt = 0; kt < 2 && kt < nkt; ++kt) {
-      issue_tile(kt, false);
-      issue_tile(kt, true);
+      int phys[C::kBlocksPerTile];
+#pragma unroll
+      for (int b = 0; b < C::kBlocksPerTile; ++b) {
+        phys[b] = tile_block(kt, b);
+        s_phys[(kt & 3) * C::kBlocksPerTile + b] = phys[b];
+      }
+      issue_tile(kt, false, phys);
+      issue_tile(kt, true, phys);
     }
   }
   if (warp == 0) {
-    tmem_alloc(head_s + 64, kPfTmemCols);
+    tmem_alloc(tmem_slot_s, kPfTmemCols);
     tmem_relinquish();
   }
   if (!producer) {  // Q tile: thread r writes its row (256 B) into the two dim halves
@@ -229,11 +238,11 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     return m;
   };
 
-  if (producer) {
-    // ======================= producer warp ==============================
+  if (mma_warp) {
+    // ======================= MMA warp (lane 0 issues) ====================
     constexpr uint32_t kIdescS = umma_idesc_f16(kPfRows, kPfKeys, kBF16);
     constexpr uint32_t kIdescO = umma_idesc_f16(kPfRows, kPfD, kBF16, /*b_mn_major=*/true);
-    auto issue_s = [&](int kt) {  // S(kt) = Q K(kt)^T
+    auto issue_s = [&](int kt) {  // S(kt) = Q K(kt)^T; then K(kt)'s stage is free
       wait(full_k + 8 * (kt & 1), (kt >> 1) & 1);
       if (failed || lane != 0) return;
       tc_fence_after_sync();
@@ -244,17 +253,16 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
                  umma_desc_k128(k_st + (k >> 2) * (kPfKeys * 128) + (k & 3) * 32), kIdescS,
                  k > 0 ? 1u : 0u);
       umma_commit(bar_s);
+      umma_commit(k_empty + 8 * (kt & 1));
     };
     issue_s(0);
     for (int kt = 0; kt < nkt; ++kt) {
       const int st = kt & 1;
       if (kt + 1 < nkt) {
-        wait(s_free, kt & 1);  // every row has read S(kt): S(kt) is done, K(kt) free
+        wait(s_free, kt & 1);  // every row has read S(kt): S's columns are free
         issue_s(kt + 1);
-        if (lane == 0 && !failed && kt + 2 < nkt) issue_tile(kt + 2, false);
       }
       wait(p_ready, kt & 1);  // P(kt) in TMEM, O(kt-1) done (the rows waited for it)
-      if (lane == 0 && !failed && kt >= 1 && kt + 1 < nkt) issue_tile(kt + 1, true);
       wait(full_v + 8 * st, (kt >> 1) & 1);
       // values of keys past the context or in bad blocks may hold anything
       // (0 * NaN would reach O): zero their rows of V(kt)
@@ -285,8 +293,54 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
           umma_f16_ts(tO, tPl + 8 * k, umma_desc_mn128(v_st + k * 2048, kPfKeys * 128), kIdescO,
                       1u);
         umma_commit(bar_o);
+        umma_commit(v_empty + 8 * st);
       }
       __syncwarp();
+    }
+  } else if (producer) {
+    // ======================= load warp (lane 0 issues) ===================
+    // K(kt) waits for its stage (S(kt-2) done), V(kt) for its own (O(kt-2)
+    // done); whichever is ready goes first.  The block ids of the next K
+    // tile are read ahead, while the loader waits.
+    int nk = min(2, nkt), nv = min(2, nkt);  // tiles 0 and 1 went out above
+    int nphys[C::kBlocksPerTile];
+#pragma unroll
+    for (int b = 0; b < C::kBlocksPerTile; ++b) nphys[b] = nk < nkt ? tile_block(nk, b) : -1;
+    unsigned long long t_idle = global_timer_ns();
+    while ((nk < nkt || nv < nkt) && !failed) {
+      bool did = false;
+      if (nv < nk && nv < nkt) {
+        const int ready = __shfl_sync(
+            0xffffffffu, lane == 0 ? (int)mbar_try_wait(v_empty + 8 * (nv & 1), ((nv >> 1) - 1) & 1) : 0, 0);
+        if (ready) {
+          if (lane == 0) issue_tile(nv, true, s_phys + (nv & 3) * C::kBlocksPerTile);
+          ++nv;
+          did = true;
+        }
+      }
+      if (nk < nkt) {
+        const int ready = __shfl_sync(
+            0xffffffffu, lane == 0 ? (int)mbar_try_wait(k_empty + 8 * (nk & 1), ((nk >> 1) - 1) & 1) : 0, 0);
+        if (ready) {
+          if (lane == 0) {
+#pragma unroll
+            for (int b = 0; b < C::kBlocksPerTile; ++b)
+              s_phys[(nk & 3) * C::kBlocksPerTile + b] = nphys[b];
+            issue_tile(nk, false, nphys);
+          }
+          ++nk;
+#pragma unroll
+          for (int b = 0; b < C::kBlocksPerTile; ++b) nphys[b] = nk < nkt ? tile_block(nk, b) : -1;
+          did = true;
+        }
+      }
+      const unsigned long long now = global_timer_ns();
+      if (did) {
+        t_idle = now;
+      } else if (now - t_idle > kWaitLimitNs) {
+        failed = true;
+        if (lane == 0) record_error(PA_ERR_TIMEOUT);
+      }
     }
   } else {
     // ======================= row warps ==================================
