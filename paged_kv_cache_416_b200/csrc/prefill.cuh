@@ -18,8 +18,9 @@
 //           values that must not reach O.  The two sides hand over through
 //           mbarriers only (S done, S read, P ready, O done), never a
 //           CTA-wide barrier inside the key loop.
-//   TMEM  = S [0, 64) | P_hi [64, 96) | P_lo [96, 128) | O [128, 256) (fp32
-//           S and O; P two 16-bit values per column)
+//   TMEM  = two S/P buffers [0, 64) and [64, 128) | O [128, 256): S(kt) in
+//           buffer kt & 1 (fp32), then P(kt) over it (P_hi in its first 32
+//           columns, P_lo in the next 32, two 16-bit values per column)
 //   per 64-key tile kt (K and V by TMA into two stages each, one box per
 //   (block, dim half); K(kt+2) is loaded once S(kt) has been read, V(kt+1)
 //   once O(kt-1) is done):
@@ -56,7 +57,7 @@ constexpr int kPfThreads = 192;     // + warp 4: MMA issue, warp 5: TMA loads
 constexpr int kPfRows = 128;      // MMA M: (token, head) rows per CTA
 constexpr int kPfKeys = 64;       // keys per tile
 constexpr int kPfD = 128;         // head_dim
-constexpr int kPfTmemCols = 256;  // S [0, 64), P_hi [64, 96), P_lo [96, 128), O [128, 256)
+constexpr int kPfTmemCols = 256;  // S/P buffers [0, 64) and [64, 128), O [128, 256)
 constexpr float kPfRescaleLog2 = 8.f;  // rescale O when the max grows by more than this
 
 template <int BS>
@@ -136,8 +137,9 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
   const uint32_t bar_s = head_s + 32, bar_o = head_s + 40;  // MMA commits
   const uint32_t s_free = head_s + 48, p_ready = head_s + 56;  // one arrival per row warp
   const uint32_t k_empty = head_s + 64, v_empty = head_s + 80;  // + 8 * stage, MMA commits
-  const uint32_t tmem_slot_s = head_s + 96;  // tcgen05.alloc writes the TMEM address here
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(base + C::kTiles + 96);
+  const uint32_t bar_done = head_s + 96;                           // the last O product
+  const uint32_t tmem_slot_s = head_s + 104;  // tcgen05.alloc writes the TMEM address here
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(base + C::kTiles + 104);
   // the loader's block ids of key tile kt (K issue writes, V issue reads)
   int* const s_phys = reinterpret_cast<int*>(base + C::kTiles + 128);  // [4][kBlocksPerTile]
   const uint32_t sQ = base_s + C::kOffQ, sK = base_s + C::kOffK, sV = base_s + C::kOffV;
@@ -180,7 +182,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     for (int i = 0; i < 6; ++i) mbar_init(head_s + 8 * i, 1);
     mbar_init(s_free, kPfRowThreads / 32);
     mbar_init(p_ready, kPfRowThreads / 32);
-    for (int i = 0; i < 4; ++i) mbar_init(k_empty + 8 * i, 1);  // k_empty[2], v_empty[2]
+    for (int i = 0; i < 5; ++i) mbar_init(k_empty + 8 * i, 1);  // k/v_empty[2], done
     mbar_init_fence();
     prefetch_tensormap(&a.tmap_k);
     prefetch_tensormap(&a.tmap_v);
@@ -221,7 +223,10 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
   tc_fence_after_sync();
   if (any_bad && tid == 0) record_error(PA_ERR_DEVICE_BOUNDS);
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tPh = tmem + 64, tPl = tmem + 96, tO = tmem + 128;
+  // S(kt) and then P(kt) (hi in the first 32 columns, lo in the next 32) live
+  // in buffer kt & 1; O in [128, 256)
+  const uint32_t tO = tmem + 128;
+  auto tbuf = [&](int kt) { return tmem + 64u * static_cast<uint32_t>(kt & 1); };
   bool failed = false;
   auto wait = [&](uint32_t bar, int parity) {
     if (!failed && !mbar_wait_bounded(bar, parity)) {
@@ -249,7 +254,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
       const uint32_t k_st = sK + (kt & 1) * C::kKBytes;
 #pragma unroll
       for (int k = 0; k < kPfD / 16; ++k)
-        umma_f16(tS, umma_desc_k128(sQ + (k >> 2) * (kPfRows * 128) + (k & 3) * 32),
+        umma_f16(tbuf(kt), umma_desc_k128(sQ + (k >> 2) * (kPfRows * 128) + (k & 3) * 32),
                  umma_desc_k128(k_st + (k >> 2) * (kPfKeys * 128) + (k & 3) * 32), kIdescS,
                  k > 0 ? 1u : 0u);
       umma_commit(bar_s);
@@ -259,7 +264,10 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     for (int kt = 0; kt < nkt; ++kt) {
       const int st = kt & 1;
       if (kt + 1 < nkt) {
-        wait(s_free, kt & 1);  // every row has read S(kt): S's columns are free
+        wait(s_free, kt & 1);  // every row has read S(kt)
+        // S(kt+1) overwrites buffer (kt+1) & 1, whose P(kt-1) O(kt-1) reads:
+        // wait for O(kt-1) (these waits go in order, one per product)
+        if (kt >= 1) wait(bar_o, (kt - 1) & 1);
         issue_s(kt + 1);
       }
       wait(p_ready, kt & 1);  // P(kt) in TMEM, O(kt-1) done (the rows waited for it)
@@ -284,19 +292,21 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
       if (lane == 0 && !failed) {  // O += (P_hi + P_lo) V(kt): 2 x 4 MMAs of K = 16
         tc_fence_after_sync();
         const uint32_t v_st = sV + st * C::kKBytes;
+        const uint32_t tP = tbuf(kt);
 #pragma unroll
         for (int k = 0; k < kPfKeys / 16; ++k)
-          umma_f16_ts(tO, tPh + 8 * k, umma_desc_mn128(v_st + k * 2048, kPfKeys * 128), kIdescO,
+          umma_f16_ts(tO, tP + 8 * k, umma_desc_mn128(v_st + k * 2048, kPfKeys * 128), kIdescO,
                       (kt > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
         for (int k = 0; k < kPfKeys / 16; ++k)
-          umma_f16_ts(tO, tPl + 8 * k, umma_desc_mn128(v_st + k * 2048, kPfKeys * 128), kIdescO,
-                      1u);
+          umma_f16_ts(tO, tP + 32 + 8 * k, umma_desc_mn128(v_st + k * 2048, kPfKeys * 128),
+                      kIdescO, 1u);
         umma_commit(bar_o);
         umma_commit(v_empty + 8 * st);
       }
       __syncwarp();
     }
+    if (lane == 0 && !failed) umma_commit(bar_done);
   } else if (producer) {
     // ======================= load warp (lane 0 issues) ===================
     // K(kt) waits for its stage (S(kt-2) done), V(kt) for its own (O(kt-2)
@@ -352,11 +362,12 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
       wait(bar_s, kt & 1);
       tc_fence_after_sync();
       uint32_t sv[kPfKeys];
+      const uint32_t tb = tbuf(kt) + lane_off;
       {
         uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
         uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
-        tmem_ld32(tS + lane_off, lo);
-        tmem_ld32(tS + lane_off + 32, hi);
+        tmem_ld32(tb, lo);
+        tmem_ld32(tb + 32, hi);
       }
       tmem_wait_ld();
       tc_fence_before_sync();
@@ -410,10 +421,12 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
       }
       const float2 ss = f2_split(sum2);
       l_run = l_run * alpha + (ss.x + ss.y);
-      if (kt > 0) {
-        wait(bar_o, (kt - 1) & 1);  // O(kt-1) done: P's columns free, O stable
+      // O is touched only to rescale it: then wait for O(kt-1) (S(kt) done
+      // means O(kt-2) is, so this wait cannot fall two phases behind)
+      if (kt > 0 && __any_sync(0xffffffffu, resc)) {
+        wait(bar_o, (kt - 1) & 1);
         tc_fence_after_sync();
-        if (__any_sync(0xffffffffu, resc)) {  // tcgen05.ld / st are warp-wide
+        {  // tcgen05.ld / st are warp-wide
           const uint64_t al2 = f2(alpha, alpha);
 #pragma unroll
           for (int c = 0; c < kPfD / 32; ++c) {
@@ -431,8 +444,10 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
           }
         }
       }
-      tmem_st32(tPh + lane_off, ph);
-      tmem_st32(tPl + lane_off, pl);
+      // P(kt) over S(kt) in its buffer: the buffer's previous reader O(kt-2)
+      // finished before S(kt) did
+      tmem_st32(tb, ph);
+      tmem_st32(tb + 32, pl);
       tmem_wait_st();
       tc_fence_before_sync();
       __syncwarp();
@@ -440,7 +455,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     }
 
     // ---- epilogue: O / l for this thread's row
-    wait(bar_o, (nkt - 1) & 1);
+    wait(bar_done, 0);
     tc_fence_after_sync();
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
     uint4* const orow = reinterpret_cast<uint4*>(a.out) + orow_off;
