@@ -107,3 +107,57 @@ def test_python_binding_raises_with_the_message(pa):
     with pytest.raises(pa.PagedAttnError) as e:
         pa.check(_decode(pa, hq=7))
     assert "PA_ERR_HEADS" in str(e.value)
+
+
+def _shared(pa, **kw):
+    args = dict(out=None, q=None, q_dtype=1, k_pool=None, v_pool=None, cache_dtype=1,
+                block_tables=None, max_blocks=4, context_lens=None, max_ctx=64, group_start=None,
+                group_seqs=None, num_groups=1, B=2, hq=8, hkv=2, D=128, bs=16, N=32, scale=0.1,
+                split=0, ws=None, ws_bytes=0, stream=None)
+    args.update(kw)
+    return pa.pa_decode_shared_prefix(*args.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(q_dtype=2, cache_dtype=2), 2),         # no e4m3 cache on this path
+    (dict(q_dtype=0, cache_dtype=1), 2),
+    (dict(D=96), 3),
+    (dict(num_groups=-1), 3),
+    (dict(max_ctx=65), 3),
+    (dict(hq=7), 4),
+    (dict(scale=float("nan")), 3),
+    (dict(), 1),                                 # valid sizes, null pointers
+])
+def test_shared_prefix_decode_rejects_bad_arguments_on_the_host(pa, kw, status):
+    assert _shared(pa, **kw) == status
+    assert pa.pa_last_error()
+
+
+def test_shared_prefix_workspace_is_bounded(pa):
+    # the partial slots are bounded through the shortest range the host
+    # fixes, so the workspace stays a few tens of MB at the bench's sizes
+    n = pa.pa_decode_shared_prefix_workspace_size(128, 32, 8, 128, 16, 1568, 0)
+    assert 0 < n < 64 << 20
+    n_big = pa.pa_decode_shared_prefix_workspace_size(256, 64, 8, 128, 16, 32768, 0)
+    assert 0 < n_big < 96 << 20
+    assert pa.pa_decode_shared_prefix_workspace_size(4, 8, 2, 96, 16, 64, 0) == 0
+    assert _shared(pa, B=0) == 0
+
+
+def _prefill(pa, **kw):
+    args = dict(out=None, q=None, q_dtype=1, k_pool=None, v_pool=None, cache_dtype=1,
+                block_tables=None, max_blocks=4, context_lens=None, query_start=None, B=2,
+                max_q=16, max_ctx=64, hq=32, hkv=8, D=128, bs=16, N=32, scale=0.1, stream=None)
+    args.update(kw)
+    return pa.pa_prefill(*args.values())
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(cache_dtype=2), 2),                    # tensor-core path: 16-bit caches only
+    (dict(q_dtype=0), 2),
+    (dict(D=64), 3),
+    (dict(hq=24, hkv=8), 4),                     # G = 3 does not divide 128 rows
+    (dict(), 1),
+])
+def test_prefill_rejects_bad_arguments_on_the_host(pa, kw, status):
+    assert _prefill(pa, **kw) == status
