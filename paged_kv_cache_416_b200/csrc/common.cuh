@@ -49,11 +49,6 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                ::"r"(bar), "r"(bytes) : "memory");
 }
 
-// Barrier `id` (1..15) among `count` threads (whole warps) of the CTA.
-__device__ __forceinline__ void named_barrier(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 // Plain arrival (count 1, no transaction bytes), release semantics.
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
