@@ -8,29 +8,26 @@
 //
 // Work decomposition
 //   chunk = up to 16 / G members of one group that share P leading blocks
-//           (or one sequence on its own, P = 0).  Its rows are the members'
-//           query heads of one kv head, at most 16 (the MMA's M).
-//   virtual block list of a chunk = the P shared blocks, then each member's
-//           own blocks (its table from entry P on), member after member.
-//           A shared block is attended by every row, an own block by its
-//           member's G rows only (the others see -inf scores for it).
-//   item  = (chunk, range of its virtual blocks, kv head); a chunk's blocks
-//           are cut into ranges of equal length; CTA = 4 warps, persistent,
-//           items from an atomic counter
-//   warp  = every 4th block of the range, through a ring of stages filled by
-//           one tiled TMA copy per K or V tile (the decode kernel's tensor
-//           maps, swizzle and shared-memory layout); the table entries of
-//           the warp's next 32 blocks are resolved ahead in registers
-// Per 16 keys and warp (m16n8k16, rows = the chunk's query rows):
-//   S = Q K^T        A = Q (registers), B = K rows (ldmatrix)
-//   online softmax   per row, masked by block owner and valid keys
-//   O += P V         A = P from the S accumulators (hi + lo 16-bit parts for
-//                    bf16), B = V (ldmatrix.trans; values of keys past a
-//                    member's length are zeroed in the fragments)
-// The warps' states are merged through shared memory.  A chunk of one range
-// writes the output; otherwise each range writes (log-sum-exp, normalised
-// output) per row and the CTA that finishes the chunk's last range merges
-// them (log-sum-exp merge).
+//           (or one sequence on its own, P = 0)
+//   range = a run of at most R blocks that is either shared (the first P
+//           blocks, attended by every member's G query heads: up to 16 rows)
+//           or one member's own (its blocks from P on, attended by its G
+//           heads only); the planning kernel cuts every chunk into such
+//           ranges of about equal length, each with its partial slot
+//   item  = (range, kv head); CTA = 4 warps, persistent, items from an atomic
+//           counter; warp = every 4th block of the range through a ring of
+//           stages, each K or V tile one tiled TMA copy (the decode kernel's
+//           tensor maps, swizzle and layout), table entries read ahead
+// A shared range runs m16n8k16 tiles whose 16 rows are the chunk's query
+// heads: S = Q K^T (A = Q in registers, B = K rows), online softmax per row,
+// O += P V (A = P straight from the S accumulators, B = V by ldmatrix.trans).
+// An own range runs the decode kernel's form with the member's heads as the
+// MMA's N = 8 columns: S^T = K Q^T, P^T by movmatrix, O^T += V^T P^T, half the
+// MMAs of a 16-row tile.  bf16 keeps P as hi + lo parts in both.
+// The warps' states merge through shared memory; a chunk of one range writes
+// the output, otherwise every range writes (log-sum-exp, normalised output)
+// per row (-inf for rows it does not attend) and the CTA that finishes the
+// chunk's last range merges them.
 #pragma once
 
 #include <cuda.h>
@@ -56,9 +53,10 @@ struct CascadeArgs {
   const int32_t* context_lens;
   const int32_t* chunk_seqs;   // members, chunk by chunk
   const int4* chunks;          // [2 * chunks]: (member offset, members, shared blocks, first
-                               // slot), (virtual blocks, ranges, blocks per range, -)
-  const int2* items;           // (chunk, range)
-  const int32_t* total;        // number of (chunk, range) items
+                               // slot), (ranges, -, -, -)
+  const int4* ranges;          // [slots]: (chunk, member or -1 for shared, first block, end
+                               // block): table entries of the leader (shared) or the member
+  const int32_t* total;        // number of ranges
   int32_t* counter;            // work counter (zeroed by the planning kernel)
   int32_t* arrived;            // [chunks * Hkv] ranges finished
   float* lse_part;             // [slots * Hkv * 16]
@@ -72,23 +70,20 @@ __global__ void __launch_bounds__(kDecodeThreads)
 cascade_kernel(const __grid_constant__ CascadeArgs a) {
   using C = DecodeCfg<kBF16 ? kCacheBF16 : kCacheF16, D, BS>;
   constexpr int kStages = C::kStages;
-  constexpr int kNT = D / 8;  // output n-tiles (8 dims each)
+  constexpr int kNT = D / 8;  // 16-row path: output n-tiles (8 dims each)
   constexpr int kRows = kCascadeRows;
   static_assert(C::kWarpBytes >= (kRows * D + 2 * kRows) * 4, "warp ring too small for the merge");
   static_assert(kDecodeWarps * C::kWarpBytes >= (kCascadeMaxRanges + 1) * kRows * 4,
                 "rings too small for the range weights");
-  static_assert(kStages <= 8, "stage info array");
   extern __shared__ __align__(128) uint8_t smem[];
   __shared__ int s_item;
   __shared__ int s_flag;
-  __shared__ int s_seq[kRows];           // the chunk's members
-  __shared__ int s_tail[kRows];          // their own blocks (after the shared ones)
+  __shared__ int s_seq[kRows];  // the chunk's members
   __shared__ int s_ctx[kRows];
-  __shared__ int s_binfo[kDecodeWarps][8];  // per warp and stage: owner + 1 | valid keys << 8
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int g = lane >> 2;   // fragment row (and row + 8)
+  const int g = lane >> 2;   // fragment row group
   const int tig = lane & 3;  // thread in group
   const int li = lane >> 3;  // which 8x8 matrix of an ldmatrix.x4 this lane addresses
 
@@ -96,6 +91,7 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
   const uint32_t ring_s = (smem_s + kBarrierBytes + kTileAlign - 1) & ~uint32_t(kTileAlign - 1);
   const uint32_t wbase_s = ring_s + warp * C::kWarpBytes;
   uint8_t* const ring = smem + (ring_s - smem_s);
+  float* const scr = reinterpret_cast<float*>(ring + warp * C::kWarpBytes);  // merge scratch
   const uint32_t bar0 = smem_s + warp * kStages * 8;
   if (lane == 0) {
 #pragma unroll
@@ -110,6 +106,7 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
   __syncthreads();
 
   const int total = *a.total * a.hkv;
+  const int G = a.group;
   uint32_t n_issued = 0, n_consumed = 0;
   uint32_t skip_stage = 0;
   bool failed = false;
@@ -118,73 +115,49 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
     const int item = s_item;
     if (item >= total) break;
     const int kvh = item % a.hkv;
-    const int2 cr = a.items[item / a.hkv];
-    const int chunk = cr.x, range = cr.y;
-    const int4 c0 = a.chunks[2 * chunk], c1 = a.chunks[2 * chunk + 1];
-    const int members = c0.y, P = c0.z, slot0 = c0.w;
-    const int vblocks = c1.x, nranges = c1.y, R = c1.z;
-    const int rows = members * a.group;
+    const int slot = item / a.hkv;
+    const int4 rd = a.ranges[slot];
+    const int chunk = rd.x, member = rd.y, b0 = rd.z, b1 = rd.w;
+    const bool shared = member < 0;
+    const int4 c0 = a.chunks[2 * chunk];
+    const int members = c0.y, slot0 = c0.w;
+    const int nranges = a.chunks[2 * chunk + 1].x;
+    const int rows = members * G;
     if (threadIdx.x < members) {
       const int seq = a.chunk_seqs[c0.x + threadIdx.x];
-      const int c = a.context_lens[seq];  // validated by the planning kernel
       s_seq[threadIdx.x] = seq;
-      s_ctx[threadIdx.x] = c;
-      s_tail[threadIdx.x] = (c + BS - 1) / BS - P;
+      s_ctx[threadIdx.x] = a.context_lens[seq];  // validated by the planning kernel
     }
     __syncthreads();
-    const int vb0 = range * R;
-    const int nblk = max(0, min(vblocks, vb0 + R) - vb0);
+    const int own_seq = s_seq[shared ? 0 : member];
+    const int nblk = b1 - b0;
     const int nb_w = nblk > warp ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
+    const int32_t* table = a.block_tables + static_cast<int64_t>(own_seq) * a.max_blocks;
 
-    // ---- virtual block -> (physical block, owner + 1 | valid keys << 8)
-    auto resolve = [&](int v, int& phys) -> int {
-      int seq, j, info;
-      if (v < P) {
-        seq = s_seq[0];
-        j = v;
-        info = BS << 8;  // every row, every key
-      } else {
-        int u = v - P, i = 0;
-        while (i < members - 1 && u >= s_tail[i]) u -= s_tail[i++];
-        seq = s_seq[i];
-        j = P + u;
-        info = (i + 1) | (min(BS, s_ctx[i] - j * BS) << 8);
-      }
-      phys = a.block_tables[static_cast<int64_t>(seq) * a.max_blocks + j];
-      return info;
+    // ---- table entries of the warp's blocks, 32 ahead in registers (lane l
+    // holds the warp's block 32 * chunk + l)
+    auto load_chunk = [&](int c) -> int {
+      const int i = c * 32 + lane;
+      return i < nb_w ? table[b0 + warp + i * kDecodeWarps] : -1;
     };
-    // lane l holds the warp's block 32 * chunk + l; cur / nxt as in decode
-    int tab_chunk = 0, phys_cur = -1, info_cur = 0, phys_nxt = -1, info_nxt = 0;
-    auto load_chunk = [&](int ch, int& phys, int& info) {
-      const int i = ch * 32 + lane;
-      if (i < nb_w) {
-        info = resolve(vb0 + warp + i * kDecodeWarps, phys);
-      } else {
-        phys = -1;
-        info = 0;
-      }
-    };
-    load_chunk(0, phys_cur, info_cur);
-    load_chunk(1, phys_nxt, info_nxt);
-
+    int tab_chunk = 0;
+    int tab_cur = load_chunk(0);
+    int tab_nxt = load_chunk(1);
     auto issue = [&](int i) {
       const int st = n_issued % kStages;
       const uint32_t bar = bar0 + 8 * st;
       const uint32_t sK = wbase_s + st * C::kStageBytes;
       if ((i >> 5) != tab_chunk) {
         tab_chunk = i >> 5;
-        phys_cur = phys_nxt;
-        info_cur = info_nxt;
-        load_chunk(tab_chunk + 1, phys_nxt, info_nxt);
+        tab_cur = tab_nxt;
+        tab_nxt = load_chunk(tab_chunk + 1);
       }
-      const int phys = __shfl_sync(0xffffffffu, phys_cur, i & 31);
-      const int info = __shfl_sync(0xffffffffu, info_cur, i & 31);
+      const int phys = __shfl_sync(0xffffffffu, tab_cur, i & 31);
       const bool ok = phys >= 0 && phys < a.num_blocks;
       skip_stage = ok ? (skip_stage & ~(1u << st)) : (skip_stage | (1u << st));
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
-        s_binfo[warp][st] = info;
         if (ok) {
           mbar_arrive_expect_tx(bar, 2u * C::kTileBytes);
           tma_load_5d(sK, &a.tmap_k, 0, 0, 0, kvh, phys, bar);
@@ -200,41 +173,9 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
       const int pro = min(kStages, nb_w);
       for (int i = 0; i < pro; ++i) issue(i);
     }
-
-    // ---- query rows as the A operand: rows g and g + 8 of each 16-dim step
-    uint32_t qa[D / 16][4];
-    {
-      const uint16_t* qrow[2];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int r = g + 8 * h;
-        const int rr = r < rows ? r : 0;
-        qrow[h] = reinterpret_cast<const uint16_t*>(a.q) +
-                  (static_cast<int64_t>(s_seq[rr / a.group]) * a.hq + kvh * a.group +
-                   rr % a.group) * D;
-      }
-      const bool ok0 = g < rows, ok1 = g + 8 < rows;
-#pragma unroll
-      for (int ks = 0; ks < D / 16; ++ks) {
-        const int d0 = ks * 16 + 2 * tig;
-        qa[ks][0] = ok0 ? *reinterpret_cast<const uint32_t*>(qrow[0] + d0) : 0u;
-        qa[ks][1] = ok1 ? *reinterpret_cast<const uint32_t*>(qrow[1] + d0) : 0u;
-        qa[ks][2] = ok0 ? *reinterpret_cast<const uint32_t*>(qrow[0] + d0 + 8) : 0u;
-        qa[ks][3] = ok1 ? *reinterpret_cast<const uint32_t*>(qrow[1] + d0 + 8) : 0u;
-      }
-    }
-    const int own0 = g / a.group, own1 = (g + 8) / a.group;  // member of rows g, g + 8
-
-    float acc[kNT][4];
-#pragma unroll
-    for (int n = 0; n < kNT; ++n)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
-    float m_run[2] = {-INFINITY, -INFINITY};  // rows g, g + 8 (log2 units)
-    float l_run[2] = {0.f, 0.f};              // this thread's share of the row sums
-
-    for (int i = 0; i < nb_w; ++i) {
-      const int st = n_consumed % kStages;
+    // wait for the warp's next block; false when it is skipped or failed
+    auto consume = [&](int& st) -> bool {
+      st = n_consumed % kStages;
       const uint32_t par = (n_consumed / kStages) & 1u;
       if (!failed) {
         const bool ok = __all_sync(0xffffffffu, mbar_wait_bounded(bar0 + 8 * st, par));
@@ -243,128 +184,136 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
           if (lane == 0) record_error(PA_ERR_TIMEOUT);
         }
       }
-      __syncwarp();  // lane 0's s_binfo write of this stage is visible
-      if (!failed && !((skip_stage >> st) & 1u)) {
-        const uint32_t sK = wbase_s + st * C::kStageBytes;
-        const uint32_t sV = sK + C::kTileBytes;
-        const int info = s_binfo[warp][st];
-        const int owner = (info & 0xff) - 1;  // -1: a shared block
-        const int valid = info >> 8;           // keys of the block inside the context
-        // rows that attend this block: every member's for a shared block,
-        // the owner's G rows for an own block
-        const bool act0 = owner < 0 || own0 == owner;
-        const bool act1 = owner < 0 || own1 == owner;
-        const bool full = owner < 0;           // shared blocks are whole and seen by all
-#pragma unroll
-        for (int kt = 0; kt < BS / 16; ++kt) {
-          // ---- S = Q K^T for 16 keys: two n-tiles of 8 keys, even / odd
-          // dim steps in separate accumulators (four independent chains)
-          float s[2][4], so[2][4];
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) s[nt][e] = so[nt][e] = 0.f;
-#pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            const int key = kt * 16 + nt * 8 + (lane & 7);
-#pragma unroll
-            for (int ks = 0; ks < D / 16; ks += 2) {
-              uint32_t b0, b1, b2, b3;
-              ldsm_x4(sK + tile_off<C>(key, ((ks + (li >> 1)) * 16 + (li & 1) * 8) * 2), b0, b1,
-                      b2, b3);
-              mma_16816<kBF16>(s[nt], qa[ks], b0, b1);
-              mma_16816<kBF16>(so[nt], qa[ks + 1], b2, b3);
-            }
-          }
-          // ---- online softmax of rows g (elements 0, 1) and g + 8 (2, 3)
-          float alpha[2];
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const bool act = h == 0 ? act0 : act1;
-            float x[4];
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-              for (int e = 0; e < 2; ++e) {
-                const int key = kt * 16 + nt * 8 + 2 * tig + e;
-                const float v = (s[nt][2 * h + e] + so[nt][2 * h + e]) * a.sl2;
-                x[2 * nt + e] = (full || (act && key < valid)) ? v : -INFINITY;
-              }
-            float bm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-            bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
-            const float mn = fmaxf(m_run[h], bm);
-            alpha[h] = mn == -INFINITY ? 1.f : fast_exp2(m_run[h] - mn);
-            m_run[h] = mn;
-            float ps = 0.f;
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              x[e] = x[e] == -INFINITY ? 0.f : fast_exp2(x[e] - mn);
-              ps += x[e];
-            }
-            l_run[h] = l_run[h] * alpha[h] + ps;
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt) {
-              s[nt][2 * h] = x[2 * nt];
-              s[nt][2 * h + 1] = x[2 * nt + 1];
-            }
-          }
-#pragma unroll
-          for (int n = 0; n < kNT; ++n) {
-            acc[n][0] *= alpha[0];
-            acc[n][1] *= alpha[0];
-            acc[n][2] *= alpha[1];
-            acc[n][3] *= alpha[1];
-          }
-          // ---- P as the A operand (16 rows x 16 keys): the S accumulator
-          // layout of two n-tiles is the A fragment layout.  bf16 keeps P as
-          // hi + lo parts: one bf16 value (8 significant bits) errs by up to
-          // 2^-9 of a weight, which outputs formed by cancellation cannot
-          // absorb; fp16 P keeps 11 bits and stays one part.
-          uint32_t pa[4], pl[4];
-          pa[0] = pack2<kBF16>(s[0][0], s[0][1]);
-          pa[1] = pack2<kBF16>(s[0][2], s[0][3]);
-          pa[2] = pack2<kBF16>(s[1][0], s[1][1]);
-          pa[3] = pack2<kBF16>(s[1][2], s[1][3]);
-          if constexpr (kBF16) {
-            pl[0] = pack_bf16x2(s[0][0] - to_float<true>(pa[0] & 0xffff), s[0][1] - to_float<true>(pa[0] >> 16));
-            pl[1] = pack_bf16x2(s[0][2] - to_float<true>(pa[1] & 0xffff), s[0][3] - to_float<true>(pa[1] >> 16));
-            pl[2] = pack_bf16x2(s[1][0] - to_float<true>(pa[2] & 0xffff), s[1][1] - to_float<true>(pa[2] >> 16));
-            pl[3] = pack_bf16x2(s[1][2] - to_float<true>(pa[3] & 0xffff), s[1][3] - to_float<true>(pa[3] >> 16));
-          }
-          // ---- O += P V: B = V (keys x dims) through ldmatrix.trans.  Keys
-          // past the member's length (the end of its last block) may hold
-          // anything, NaN included: their values are zeroed here.
-          uint32_t m_lo = 0xffffffffu, m_hi = 0xffffffffu;  // keys 2tig(+1), 2tig+8(+9)
-          if (valid < BS) {
-            const int tk = kt * 16 + 2 * tig;
-            m_lo = pair_mask(tk < valid, tk + 1 < valid);
-            m_hi = pair_mask(tk + 8 < valid, tk + 9 < valid);
-          }
-          const int vkey = kt * 16 + (li & 1) * 8 + (lane & 7);
-#pragma unroll
-          for (int n2 = 0; n2 < D / 16; ++n2) {
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_trans(sV + tile_off<C>(vkey, (n2 * 16 + (li >> 1) * 8) * 2), b0, b1, b2, b3);
-            b0 &= m_lo; b1 &= m_hi; b2 &= m_lo; b3 &= m_hi;
-            mma_16816<kBF16>(acc[2 * n2], pa, b0, b1);
-            mma_16816<kBF16>(acc[2 * n2 + 1], pa, b2, b3);
-            if constexpr (kBF16) {
-              mma_16816<kBF16>(acc[2 * n2], pl, b0, b1);
-              mma_16816<kBF16>(acc[2 * n2 + 1], pl, b2, b3);
-            }
-          }
-        }
-      }
+      return !failed && !((skip_stage >> st) & 1u);
+    };
+    auto release = [&](int i) {
       __syncwarp();
       ++n_consumed;
       if (!failed && i + kStages < nb_w) issue(i + kStages);
-    }
+    };
 
-    // ---- merge the warps' states through shared memory (the rings are
-    // idle: every load of this item has been consumed)
-    {
-      float* scr = reinterpret_cast<float*>(ring + warp * C::kWarpBytes);
+    if (shared) {
+      // ================= shared range: 16-row tiles =====================
+      uint32_t qa[D / 16][4];
+      {
+        const uint16_t* qrow[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int r = g + 8 * h;
+          const int rr = r < rows ? r : 0;
+          qrow[h] = reinterpret_cast<const uint16_t*>(a.q) +
+                    (static_cast<int64_t>(s_seq[rr / G]) * a.hq + kvh * G + rr % G) * D;
+        }
+        const bool ok0 = g < rows, ok1 = g + 8 < rows;
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const int d0 = ks * 16 + 2 * tig;
+          qa[ks][0] = ok0 ? *reinterpret_cast<const uint32_t*>(qrow[0] + d0) : 0u;
+          qa[ks][1] = ok1 ? *reinterpret_cast<const uint32_t*>(qrow[1] + d0) : 0u;
+          qa[ks][2] = ok0 ? *reinterpret_cast<const uint32_t*>(qrow[0] + d0 + 8) : 0u;
+          qa[ks][3] = ok1 ? *reinterpret_cast<const uint32_t*>(qrow[1] + d0 + 8) : 0u;
+        }
+      }
+      float acc[kNT][4];
+#pragma unroll
+      for (int n = 0; n < kNT; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[n][e] = 0.f;
+      float m_run[2] = {-INFINITY, -INFINITY};  // rows g, g + 8 (log2 units)
+      float l_run[2] = {0.f, 0.f};              // this thread's share of the row sums
+      for (int i = 0; i < nb_w; ++i) {
+        int st;
+        if (consume(st)) {
+          const uint32_t sK = wbase_s + st * C::kStageBytes;
+          const uint32_t sV = sK + C::kTileBytes;
+#pragma unroll
+          for (int kt = 0; kt < BS / 16; ++kt) {
+            // S = Q K^T for 16 keys: two n-tiles, even / odd dim steps apart
+            float s[2][4], so[2][4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+              for (int e = 0; e < 4; ++e) s[nt][e] = so[nt][e] = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+              const int key = kt * 16 + nt * 8 + (lane & 7);
+#pragma unroll
+              for (int ks = 0; ks < D / 16; ks += 2) {
+                uint32_t k0, k1, k2, k3;
+                ldsm_x4(sK + tile_off<C>(key, ((ks + (li >> 1)) * 16 + (li & 1) * 8) * 2), k0, k1,
+                        k2, k3);
+                mma_16816<kBF16>(s[nt], qa[ks], k0, k1);
+                mma_16816<kBF16>(so[nt], qa[ks + 1], k2, k3);
+              }
+            }
+            // online softmax of rows g (elements 0, 1) and g + 8 (2, 3): the
+            // shared blocks are whole and every row attends them
+            float alpha[2];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              float x[4];
+#pragma unroll
+              for (int nt = 0; nt < 2; ++nt) {
+                x[2 * nt] = (s[nt][2 * h] + so[nt][2 * h]) * a.sl2;
+                x[2 * nt + 1] = (s[nt][2 * h + 1] + so[nt][2 * h + 1]) * a.sl2;
+              }
+              float bm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+              bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+              bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+              const float mn = fmaxf(m_run[h], bm);
+              alpha[h] = fast_exp2(m_run[h] - mn);
+              m_run[h] = mn;
+              float ps = 0.f;
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                x[e] = fast_exp2(x[e] - mn);
+                ps += x[e];
+              }
+              l_run[h] = l_run[h] * alpha[h] + ps;
+#pragma unroll
+              for (int nt = 0; nt < 2; ++nt) {
+                s[nt][2 * h] = x[2 * nt];
+                s[nt][2 * h + 1] = x[2 * nt + 1];
+              }
+            }
+#pragma unroll
+            for (int n = 0; n < kNT; ++n) {
+              acc[n][0] *= alpha[0];
+              acc[n][1] *= alpha[0];
+              acc[n][2] *= alpha[1];
+              acc[n][3] *= alpha[1];
+            }
+            // P as the A operand (the S accumulators of two n-tiles are the A
+            // fragment); bf16 keeps P as hi + lo parts (one bf16 value errs by
+            // up to 2^-9 of a weight), fp16 P keeps 11 bits in one part
+            uint32_t pa[4], pl[4];
+            pa[0] = pack2<kBF16>(s[0][0], s[0][1]);
+            pa[1] = pack2<kBF16>(s[0][2], s[0][3]);
+            pa[2] = pack2<kBF16>(s[1][0], s[1][1]);
+            pa[3] = pack2<kBF16>(s[1][2], s[1][3]);
+            if constexpr (kBF16) {
+              pl[0] = pack_bf16x2(s[0][0] - to_float<true>(pa[0] & 0xffff), s[0][1] - to_float<true>(pa[0] >> 16));
+              pl[1] = pack_bf16x2(s[0][2] - to_float<true>(pa[1] & 0xffff), s[0][3] - to_float<true>(pa[1] >> 16));
+              pl[2] = pack_bf16x2(s[1][0] - to_float<true>(pa[2] & 0xffff), s[1][1] - to_float<true>(pa[2] >> 16));
+              pl[3] = pack_bf16x2(s[1][2] - to_float<true>(pa[3] & 0xffff), s[1][3] - to_float<true>(pa[3] >> 16));
+            }
+            const int vkey = kt * 16 + (li & 1) * 8 + (lane & 7);
+#pragma unroll
+            for (int n2 = 0; n2 < D / 16; ++n2) {
+              uint32_t v0, v1, v2, v3;
+              ldsm_x4_trans(sV + tile_off<C>(vkey, (n2 * 16 + (li >> 1) * 8) * 2), v0, v1, v2, v3);
+              mma_16816<kBF16>(acc[2 * n2], pa, v0, v1);
+              mma_16816<kBF16>(acc[2 * n2 + 1], pa, v2, v3);
+              if constexpr (kBF16) {
+                mma_16816<kBF16>(acc[2 * n2], pl, v0, v1);
+                mma_16816<kBF16>(acc[2 * n2 + 1], pl, v2, v3);
+              }
+            }
+          }
+        }
+        release(i);
+      }
+      // the warp's state into its scratch: O [16][D], max [16], sum [16]
       float lsum[2];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -385,20 +334,165 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
         scr[kRows * D + kRows + g] = lsum[0];
         scr[kRows * D + kRows + g + 8] = lsum[1];
       }
+    } else {
+      // ================= own range: the member's heads as N = 8 ==========
+      // (the decode kernel's form: S^T = K Q^T, P^T by movmatrix, O^T += V^T P^T)
+      constexpr int kDT = D / 16;
+      const int own_ctx = s_ctx[member];
+      uint32_t qf[kDT][2];
+      {
+        const bool hv = g < G;
+        const uint16_t* qrow = reinterpret_cast<const uint16_t*>(a.q) +
+                               (static_cast<int64_t>(own_seq) * a.hq + kvh * G + (hv ? g : 0)) * D;
+#pragma unroll
+        for (int ks = 0; ks < kDT; ++ks) {
+          qf[ks][0] = hv ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * tig) : 0u;
+          qf[ks][1] = hv ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * tig) : 0u;
+        }
+      }
+      float acc[kDT][4];
+#pragma unroll
+      for (int dt = 0; dt < kDT; ++dt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[dt][e] = 0.f;
+      float m_run[2] = {-INFINITY, -INFINITY};  // heads 2tig, 2tig + 1 (log2 units)
+      float l_run[2] = {0.f, 0.f};              // this thread's share of the sums
+      for (int i = 0; i < nb_w; ++i) {
+        int st;
+        if (consume(st)) {
+          const uint32_t sK = wbase_s + st * C::kStageBytes;
+          const uint32_t sV = sK + C::kTileBytes;
+          const int j = b0 + warp + i * kDecodeWarps;       // the block's table entry
+          const int valid = min(BS, own_ctx - j * BS);      // its tokens inside the context
+          // S^T = K Q^T (rows: tokens, cols: the member's heads), four chains
+          float s[BS / 16][4];
+#pragma unroll
+          for (int mt = 0; mt < BS / 16; ++mt) {
+            float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
+            float s2[4] = {0.f, 0.f, 0.f, 0.f}, s3[4] = {0.f, 0.f, 0.f, 0.f};
+            const int row = mt * 16 + (lane & 7) + (li & 1) * 8;
+#pragma unroll
+            for (int ks = 0; ks < kDT; ++ks) {
+              uint32_t af[4];
+              ldsm_x4(sK + tile_off<C>(row, (ks * 16 + (li >> 1) * 8) * 2), af[0], af[1], af[2],
+                      af[3]);
+              if ((ks & 3) == 0) mma_16816<kBF16>(s0, af, qf[ks][0], qf[ks][1]);
+              else if ((ks & 3) == 1) mma_16816<kBF16>(s1, af, qf[ks][0], qf[ks][1]);
+              else if ((ks & 3) == 2) mma_16816<kBF16>(s2, af, qf[ks][0], qf[ks][1]);
+              else mma_16816<kBF16>(s3, af, qf[ks][0], qf[ks][1]);
+            }
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int tok = mt * 16 + g + (e >> 1) * 8;
+              const float x = ((s0[e] + s1[e]) + (s2[e] + s3[e])) * a.sl2;
+              s[mt][e] = tok < valid ? x : -INFINITY;
+            }
+          }
+          // online softmax per head column (every block has a valid token)
+          float alpha[2];
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            float bm = -INFINITY;
+#pragma unroll
+            for (int mt = 0; mt < BS / 16; ++mt) bm = fmaxf(bm, fmaxf(s[mt][c], s[mt][2 + c]));
+            bm = shfl_xor_max(bm);
+            const float mn = fmaxf(m_run[c], bm);
+            alpha[c] = fast_exp2(m_run[c] - mn);
+            m_run[c] = mn;
+            float ps = 0.f;
+#pragma unroll
+            for (int mt = 0; mt < BS / 16; ++mt) {
+              s[mt][c] = fast_exp2(s[mt][c] - mn);
+              s[mt][2 + c] = fast_exp2(s[mt][2 + c] - mn);
+              ps += s[mt][c] + s[mt][2 + c];
+            }
+            l_run[c] = l_run[c] * alpha[c] + ps;
+          }
+#pragma unroll
+          for (int dt = 0; dt < kDT; ++dt) {
+            acc[dt][0] *= alpha[0];
+            acc[dt][1] *= alpha[1];
+            acc[dt][2] *= alpha[0];
+            acc[dt][3] *= alpha[1];
+          }
+          // P^T as the B operand (8x8 (token, head) tiles transposed in
+          // registers); bf16 keeps hi + lo parts
+          uint32_t pb[BS / 16][2], pl[BS / 16][2];
+#pragma unroll
+          for (int mt = 0; mt < BS / 16; ++mt) {
+            const uint32_t h0 = pack2<kBF16>(s[mt][0], s[mt][1]);
+            const uint32_t h1 = pack2<kBF16>(s[mt][2], s[mt][3]);
+            pb[mt][0] = movmatrix_trans(h0);
+            pb[mt][1] = movmatrix_trans(h1);
+            if constexpr (kBF16) {
+              pl[mt][0] = movmatrix_trans(pack_bf16x2(s[mt][0] - to_float<true>(h0 & 0xffff),
+                                                      s[mt][1] - to_float<true>(h0 >> 16)));
+              pl[mt][1] = movmatrix_trans(pack_bf16x2(s[mt][2] - to_float<true>(h1 & 0xffff),
+                                                      s[mt][3] - to_float<true>(h1 >> 16)));
+            }
+          }
+          // O^T += V^T P^T; in the member's last block the value rows past its
+          // length are zeroed in the fragments (they may hold anything)
+#pragma unroll
+          for (int mt = 0; mt < BS / 16; ++mt) {
+            uint32_t m_lo = 0xffffffffu, m_hi = 0xffffffffu;  // tokens 2tig(+1), 2tig+8(+9)
+            if (valid < BS) {
+              const int tk = mt * 16 + 2 * tig;
+              m_lo = pair_mask(tk < valid, tk + 1 < valid);
+              m_hi = pair_mask(tk + 8 < valid, tk + 9 < valid);
+            }
+            const int tok = mt * 16 + (lane & 7) + (li >> 1) * 8;
+#pragma unroll
+            for (int dt = 0; dt < kDT; ++dt) {
+              uint32_t af[4];
+              ldsm_x4_trans(sV + tile_off<C>(tok, (dt * 16 + (li & 1) * 8) * 2), af[0], af[1],
+                            af[2], af[3]);
+              af[0] &= m_lo; af[1] &= m_lo; af[2] &= m_hi; af[3] &= m_hi;
+              mma_16816<kBF16>(acc[dt], af, pb[mt][0], pb[mt][1]);
+              if constexpr (kBF16) mma_16816<kBF16>(acc[dt], af, pl[mt][0], pl[mt][1]);
+            }
+          }
+        }
+        release(i);
+      }
+      // the warp's state into its scratch: O [8][D] (head-major), max [8], sum [8]
+      const float lsum0 = shfl_xor_sum(l_run[0]);
+      const float lsum1 = shfl_xor_sum(l_run[1]);
+#pragma unroll
+      for (int dt = 0; dt < kDT; ++dt) {
+        const int dlo = dt * 16 + g, dhi = dlo + 8;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int h = 2 * tig + c;
+          scr[h * D + dlo] = acc[dt][c];
+          scr[h * D + dhi] = acc[dt][2 + c];
+        }
+      }
+      if (g == 0) {
+        scr[8 * D + 2 * tig] = m_run[0];
+        scr[8 * D + 2 * tig + 1] = m_run[1];
+        scr[8 * D + 8 + 2 * tig] = lsum0;
+        scr[8 * D + 8 + 2 * tig + 1] = lsum1;
+      }
     }
     __syncthreads();
     {
+      // combine the 4 warps; a shared range covers the chunk's rows 0..rows-1
+      // (scratch: O [16][D], max at 16 D, sums at 16 D + 16), an own range the
+      // member's G rows (scratch: O [8][D], max at 8 D, sums at 8 D + 8)
+      const int nrow = shared ? rows : G;
+      const int mrow = shared ? kRows : 8;
       constexpr int kVec = 8;
-      const int units = rows * (D / kVec);
+      const int units = nrow * (D / kVec);
       for (int u = threadIdx.x; u < units; u += kDecodeThreads) {
-        const int r = u / (D / kVec);
+        const int rl = u / (D / kVec);
         const int d0 = (u % (D / kVec)) * kVec;
         float mw[kDecodeWarps];
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kDecodeWarps; ++w) {
-          const float* scr = reinterpret_cast<const float*>(ring + w * C::kWarpBytes);
-          mw[w] = scr[kRows * D + r];
+          const float* sw = reinterpret_cast<const float*>(ring + w * C::kWarpBytes);
+          mw[w] = sw[mrow * D + rl];
           M = fmaxf(M, mw[w]);
         }
         float o[kVec];
@@ -408,11 +502,11 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
         if (M != -INFINITY) {
 #pragma unroll
           for (int w = 0; w < kDecodeWarps; ++w) {
-            const float* scr = reinterpret_cast<const float*>(ring + w * C::kWarpBytes);
+            const float* sw = reinterpret_cast<const float*>(ring + w * C::kWarpBytes);
             const float f = fast_exp2(mw[w] - M);
-            L += f * scr[kRows * D + kRows + r];
-            const float4 x0 = *reinterpret_cast<const float4*>(scr + r * D + d0);
-            const float4 x1 = *reinterpret_cast<const float4*>(scr + r * D + d0 + 4);
+            L += f * sw[mrow * D + mrow + rl];
+            const float4 x0 = *reinterpret_cast<const float4*>(sw + rl * D + d0);
+            const float4 x1 = *reinterpret_cast<const float4*>(sw + rl * D + d0 + 4);
             o[0] += f * x0.x; o[1] += f * x0.y; o[2] += f * x0.z; o[3] += f * x0.w;
             o[4] += f * x1.x; o[5] += f * x1.y; o[6] += f * x1.z; o[7] += f * x1.w;
           }
@@ -420,9 +514,9 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
 #pragma unroll
           for (int v = 0; v < kVec; ++v) o[v] *= inv;
         }
+        const int r = shared ? rl : member * G + rl;  // the chunk's row
         if (nranges == 1) {
-          const int64_t qh = static_cast<int64_t>(s_seq[r / a.group]) * a.hq + kvh * a.group +
-                             r % a.group;
+          const int64_t qh = static_cast<int64_t>(s_seq[r / G]) * a.hq + kvh * G + r % G;
           uint4 pk;
           pk.x = pack2<kBF16>(o[0], o[1]);
           pk.y = pack2<kBF16>(o[2], o[3]);
@@ -430,18 +524,25 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
           pk.w = pack2<kBF16>(o[6], o[7]);
           *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.out) + qh * D + d0) = pk;
         } else {
-          const int64_t pi = (static_cast<int64_t>(slot0 + range) * a.hkv + kvh) * kRows + r;
+          const int64_t pi = (static_cast<int64_t>(slot) * a.hkv + kvh) * kRows + r;
           float* op = a.o_part + pi * D + d0;
           *reinterpret_cast<float4*>(op) = make_float4(o[0], o[1], o[2], o[3]);
           *reinterpret_cast<float4*>(op + 4) = make_float4(o[4], o[5], o[6], o[7]);
           if (d0 == 0) a.lse_part[pi] = (M == -INFINITY) ? -INFINITY : M + log2f(L);
         }
       }
+      // the rows an own range does not attend carry no weight
+      if (!shared && nranges > 1)
+        for (int r = threadIdx.x; r < rows; r += kDecodeThreads)
+          if (r / G != member)
+            a.lse_part[(static_cast<int64_t>(slot) * a.hkv + kvh) * kRows + r] = -INFINITY;
     }
     if (nranges > 1) {
       // the CTA that finishes the chunk's last range merges every range:
       // out = sum_i w_i o_i / sum_i w_i, w_i = 2^(lse_i - max lse); partials
-      // are published with a fence before the arrival count, read through L2
+      // are published with a fence before the arrival count, read through L2;
+      // a range with no weight for a row (-inf) is skipped (its vector for
+      // that row was not written)
       __threadfence();
       __syncthreads();
       if (threadIdx.x == 0) {
@@ -454,7 +555,7 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
         float* w_s = reinterpret_cast<float*>(ring);   // [nranges][16] weights
         float* wsum_s = w_s + nranges * kRows;         // [16]
         const int64_t base = (static_cast<int64_t>(slot0) * a.hkv + kvh) * kRows;
-        const int64_t rstride = static_cast<int64_t>(a.hkv) * kRows;  // between ranges
+        const int64_t rstride = static_cast<int64_t>(a.hkv) * kRows;  // between slots
         for (int k2 = threadIdx.x; k2 < nranges * rows; k2 += kDecodeThreads) {
           const int i = k2 / rows, r = k2 % rows;
           w_s[i * kRows + r] = __ldcg(a.lse_part + base + i * rstride + r);
@@ -483,16 +584,16 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
           const int d0 = (u % (D / kVec)) * kVec;
           float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
           const float* op = a.o_part + (base + r) * D + d0;
-#pragma unroll 8
           for (int i = 0; i < nranges; ++i) {
             const float w = w_s[i * kRows + r];
-            const float4 x = __ldcg(reinterpret_cast<const float4*>(op + i * rstride * D));
-            o0 += w * x.x; o1 += w * x.y; o2 += w * x.z; o3 += w * x.w;
+            if (w > 0.f) {
+              const float4 x = __ldcg(reinterpret_cast<const float4*>(op + i * rstride * D));
+              o0 += w * x.x; o1 += w * x.y; o2 += w * x.z; o3 += w * x.w;
+            }
           }
           const float W = wsum_s[r];
           const float inv = W > 0.f ? 1.f / W : 0.f;
-          const int64_t qh = static_cast<int64_t>(s_seq[r / a.group]) * a.hq + kvh * a.group +
-                             r % a.group;
+          const int64_t qh = static_cast<int64_t>(s_seq[r / G]) * a.hq + kvh * G + r % G;
           uint2 pk;
           pk.x = pack2<kBF16>(o0 * inv, o1 * inv);
           pk.y = pack2<kBF16>(o2 * inv, o3 * inv);
@@ -514,11 +615,10 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
   }
 }
 
-
 // ------------------------------------------------------------- planning
 // One CTA of 1024 threads, once per call:
 //  1. members are counted; a sequence listed twice, or outside [0, B),
-//     invalidates every group holding it (those decode plainly; reported);
+//     invalidates every group holding it (those decode unshared; reported);
 //  2. one warp per group: the shared blocks P = the longest run of leading
 //     table entries equal in every member's row, cut so that every member
 //     keeps at least one token of its own (P * bs <= len - 1).  Groups of
@@ -526,12 +626,14 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
 //     group with P > 0 becomes chunks of up to 16 / G members;
 //  3. every other sequence is a chunk of its own (P = 0); a length outside
 //     [0, min(max_ctx, max_blocks * bs)] counts as 0 and is reported;
-//  4. virtual lengths V (blocks), then the range length R = the largest of
-//     r_floor, T * Hkv / kCascadeTargetItems (T = all chunks' blocks) and
-//     max V / kCascadeMaxRanges; a chunk is cut into ceil(V / R) ranges of
-//     equal length, each with its partial slot;
-//  5. the (chunk, range) work list, the item count, arrival counters and the
-//     work counter.
+//  4. the range length R = the largest of r_floor, T * Hkv /
+//     kCascadeTargetItems (T = all chunks' blocks, shared ones once) and
+//     what keeps a chunk under kCascadeMaxRanges ranges;
+//  5. each chunk's shared blocks are cut into ceil(P / R) equal ranges and
+//     each member's own blocks into max(1, ceil(n / R)) (an empty range
+//     still writes a zero output), every range with its partial slot; the
+//     work list holds one (chunk, member or -1, first block, end block) per
+//     slot, and the arrival counters and the work counter are zeroed.
 // Chunk and slot numbers come from atomics (their order varies), but every
 // output depends only on its chunk's ranges, merged in range order: results
 // are the same from call to call.
@@ -539,12 +641,12 @@ __global__ void __launch_bounds__(1024) cascade_plan_kernel(
     const int32_t* __restrict__ ctx_lens, const int32_t* __restrict__ block_tables,
     const int32_t* __restrict__ group_start, const int32_t* __restrict__ group_seqs,
     int num_groups, int B, int max_ctx, int max_blocks, int bs, int group, int hkv, int r_floor,
-    int32_t* seen, int32_t* chunk_seqs, int4* chunks, int2* items, int32_t* total,
+    int32_t* seen, int32_t* chunk_seqs, int4* chunks, int4* ranges, int32_t* total,
     int32_t* counter, int32_t* arrived) {
-  __shared__ int n_chunks, n_used, tv_sum, v_max, n_items;
+  __shared__ int n_chunks, n_used, tv_sum, v_max, n_slots;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) {
-    n_chunks = n_used = tv_sum = v_max = n_items = 0;
+    n_chunks = n_used = tv_sum = v_max = n_slots = 0;
     *counter = 0;
   }
   for (int s = tid; s < B; s += 1024) seen[s] = 0;
@@ -617,18 +719,21 @@ __global__ void __launch_bounds__(1024) cascade_plan_kernel(
   }
   __syncthreads();
   const int nc = n_chunks;
+  auto own_blocks = [&](int seq, int P) {  // a member's blocks from P on (0 if invalid)
+    int len = ctx_lens[seq];
+    if (len < 0 || len > max_ctx || len > max_blocks * bs) len = 0;  // only unshared ones
+    return max(0, (len + bs - 1) / bs - P);
+  };
   for (int c = tid; c < nc; c += 1024) {
     const int4 d = chunks[2 * c];
     int V = d.z;
     for (int i = 0; i < d.y; ++i) {
-      int len = ctx_lens[chunk_seqs[d.x + i]];
-      if (len < 0 || len > max_ctx || len > max_blocks * bs) {  // only unshared ones get here
+      const int seq = chunk_seqs[d.x + i];
+      const int len = ctx_lens[seq];
+      if (d.z == 0 && (len < 0 || len > max_ctx || len > max_blocks * bs))
         record_error(PA_ERR_DEVICE_BOUNDS);
-        len = 0;
-      }
-      V += (len + bs - 1) / bs - d.z;
+      V += own_blocks(seq, d.z);
     }
-    chunks[2 * c + 1] = make_int4(V, 0, 0, 0);
     atomicAdd(&tv_sum, V);
     atomicMax(&v_max, V);
   }
@@ -636,19 +741,33 @@ __global__ void __launch_bounds__(1024) cascade_plan_kernel(
   const int R = max(max(r_floor, 1),
                     max(static_cast<int>((static_cast<int64_t>(tv_sum) * hkv + kCascadeTargetItems - 1) /
                                          kCascadeTargetItems),
-                        (v_max + kCascadeMaxRanges - 1) / kCascadeMaxRanges));
+                        (v_max + (kCascadeMaxRanges - kCascadeRows - 1) - 1) /
+                            (kCascadeMaxRanges - kCascadeRows - 1)));
   for (int c = tid; c < nc; c += 1024) {
-    const int V = chunks[2 * c + 1].x;
-    const int nr = max(1, (V + R - 1) / R);
-    const int rc = V > 0 ? (V + nr - 1) / nr : 1;  // equal ranges of at most R blocks
-    const int slot0 = atomicAdd(&n_items, nr);    // one slot per range
-    chunks[2 * c].w = slot0;
-    chunks[2 * c + 1] = make_int4(V, nr, rc, 0);
-    for (int r = 0; r < nr; ++r) items[slot0 + r] = make_int2(c, r);
+    const int4 d = chunks[2 * c];
+    const int P = d.z;
+    const int nsh = P > 0 ? (P + R - 1) / R : 0;
+    int nr = nsh;
+    for (int i = 0; i < d.y; ++i) nr += max(1, (own_blocks(chunk_seqs[d.x + i], P) + R - 1) / R);
+    const int slot0 = atomicAdd(&n_slots, nr);
+    chunks[2 * c] = make_int4(d.x, d.y, P, slot0);
+    chunks[2 * c + 1] = make_int4(nr, 0, 0, 0);
+    int sl = slot0;
+    if (nsh > 0) {
+      const int len = (P + nsh - 1) / nsh;  // equal shared ranges
+      for (int k = 0; k < nsh; ++k) ranges[sl++] = make_int4(c, -1, k * len, min(P, (k + 1) * len));
+    }
+    for (int i = 0; i < d.y; ++i) {
+      const int n = own_blocks(chunk_seqs[d.x + i], P);
+      const int no = max(1, (n + R - 1) / R);
+      const int len = n > 0 ? (n + no - 1) / no : 0;  // equal own ranges
+      for (int k = 0; k < no; ++k)
+        ranges[sl++] = make_int4(c, i, P + min(n, k * len), P + min(n, (k + 1) * len));
+    }
     for (int h = 0; h < hkv; ++h) arrived[c * hkv + h] = 0;
   }
   __syncthreads();
-  if (tid == 0) *total = n_items;
+  if (tid == 0) *total = n_slots;
 }
 
 }  // namespace pa

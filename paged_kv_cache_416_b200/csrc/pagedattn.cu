@@ -116,14 +116,15 @@ WsLayout ws_layout(int32_t B, int32_t hq, int32_t hkv, int32_t D, int32_t max_ct
   return w;
 }
 
-// Shared-prefix (cascade) decode workspace: work counter and item count,
-// then seen [B], chunk members [B], chunk descriptors [2B] int4, the work
-// list [slots] int2, arrival counters [B * Hkv], and the partials: fp32 lse
+// Shared-prefix (cascade) decode workspace: work counter and range count,
+// then seen [B], chunk members [B], chunk descriptors [2B] int4, the ranges
+// [slots] int4, arrival counters [B * Hkv], and the partials: fp32 lse
 // [slots * Hkv * 16] and fp32 outputs [slots * Hkv * 16 * D].  Slots are
-// bounded through the shortest range r_floor: at most B * max_blocks /
-// r_floor + B (a chunk of V blocks takes max(1, ceil(V / R)) <= V / R + 1).
+// bounded through the shortest range r_floor: a chunk takes at most
+// P / R + 1 shared ranges and n_i / R + 1 per member, so all chunks together
+// at most B * max_blocks / r_floor + 2 B.
 struct CascadeWs {
-  size_t counter = 0, total = 4, seen = 256, chunk_seqs = 0, chunks = 0, items = 0, arrived = 0,
+  size_t counter = 0, total = 4, seen = 256, chunk_seqs = 0, chunks = 0, ranges = 0, arrived = 0,
          lse = 0, o = 0, bytes = 0;
   int32_t r_floor = 1;
   int64_t slots = 0;
@@ -136,12 +137,12 @@ CascadeWs cascade_ws_layout(int32_t B, int32_t hkv, int32_t D, int32_t bs, int32
   const int64_t auto_floor = cdiv(static_cast<int64_t>(B) * max_nb * hkv, 4 * pa::kCascadeTargetItems);
   const int64_t user_floor = split_tokens > 0 ? cdiv(split_tokens, bs) : 1;
   w.r_floor = static_cast<int32_t>(std::max<int64_t>(std::max<int64_t>(4, auto_floor), user_floor));
-  w.slots = cdiv(static_cast<int64_t>(B) * max_nb, w.r_floor) + B;
+  w.slots = cdiv(static_cast<int64_t>(B) * max_nb, w.r_floor) + 2 * static_cast<int64_t>(B);
   const size_t arr = static_cast<size_t>(round_up(static_cast<int64_t>(B) * 4, 256));
   w.chunk_seqs = w.seen + arr;
   w.chunks = w.chunk_seqs + arr;
-  w.items = w.chunks + static_cast<size_t>(round_up(static_cast<int64_t>(B) * 32, 256));
-  w.arrived = w.items + static_cast<size_t>(round_up(w.slots * 8, 256));
+  w.ranges = w.chunks + static_cast<size_t>(round_up(static_cast<int64_t>(B) * 32, 256));
+  w.arrived = w.ranges + static_cast<size_t>(round_up(w.slots * 16, 256));
   w.lse = w.arrived + static_cast<size_t>(round_up(static_cast<int64_t>(B) * hkv * 4, 256));
   w.o = w.lse + static_cast<size_t>(round_up(w.slots * hkv * pa::kCascadeRows * 4, 256));
   w.bytes = w.o + static_cast<size_t>(w.slots * hkv * pa::kCascadeRows * D * 4);
@@ -583,7 +584,7 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype q_dtype, co
   a.context_lens = context_lens;
   a.chunk_seqs = reinterpret_cast<const int32_t*>(ws + w.chunk_seqs);
   a.chunks = reinterpret_cast<const int4*>(ws + w.chunks);
-  a.items = reinterpret_cast<const int2*>(ws + w.items);
+  a.ranges = reinterpret_cast<const int4*>(ws + w.ranges);
   a.total = reinterpret_cast<const int32_t*>(ws + w.total);
   a.counter = reinterpret_cast<int32_t*>(ws + w.counter);
   a.arrived = reinterpret_cast<int32_t*>(ws + w.arrived);
@@ -600,7 +601,7 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype q_dtype, co
       context_lens, block_tables, group_start, group_seqs, num_groups, num_seqs, max_context_len,
       max_blocks_per_seq, block_size, a.group, num_kv_heads, w.r_floor,
       reinterpret_cast<int32_t*>(ws + w.seen), reinterpret_cast<int32_t*>(ws + w.chunk_seqs),
-      reinterpret_cast<int4*>(ws + w.chunks), reinterpret_cast<int2*>(ws + w.items),
+      reinterpret_cast<int4*>(ws + w.chunks), reinterpret_cast<int4*>(ws + w.ranges),
       reinterpret_cast<int32_t*>(ws + w.total), a.counter, a.arrived);
   const int64_t items_upper = w.slots * num_kv_heads;
   const pa_status s = cache_dtype == PA_BF16
