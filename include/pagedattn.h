@@ -263,8 +263,8 @@ size_t pa_decode_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_he
  *     with a length outside [1, max_context_len], share nothing.
  *   - up to 16 / (Hq/Hkv) members form a chunk whose query heads are the
  *     rows of one tile: the shared blocks are attended once by all rows,
- *     each member's own blocks by its rows only, in one pass over the
- *     chunk's blocks, cut into ranges merged by log-sum-exp.
+ *     each member's own blocks by its own heads, in ranges of blocks whose
+ *     partial results are merged by log-sum-exp.
  * Supported: q and cache both f16 or both bf16 (no e4m3), head_dim 64 or
  * 128, block_size 16 or 32, Hq / Hkv <= 8.  split_tokens: 0 = automatic,
  * else the shortest range in tokens.  workspace: at least
