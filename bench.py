@@ -377,7 +377,31 @@ def run_ours(args, rank, local, world):
     torch.cuda.synchronize()
     barrier(world, device)
     pa.sync_status()
-    e2e_sec = reduce_max(e0.elapsed_time(e1) / 1e3, world, device)
+    serial_sec = reduce_max(e0.elapsed_time(e1) / 1e3, world, device)
+    serial_value, _ = aggregate(w.kv_bytes, w.seq_tokens, E, serial_sec, world, device)
+
+    # the same steps through DecodePipeline: each step's inputs still come in
+    # from pinned host memory and its output goes back every step, but on two
+    # copy streams that overlap them with the neighbouring steps' device work
+    from paged_kv_cache_416_b200.pipeline import DecodePipeline
+    pipe = DecodePipeline(kp, vp, w.scale, w.max_context_len, w.k_scale, w.v_scale, workspace=ws)
+    host_pipe = {n: t for n, t in host_in.items() if n != "pairs" or len(w.cow_pairs)}
+    outs_host = [torch.empty(out.shape, dtype=out.dtype, pin_memory=True) for _ in range(2)]
+    for i in range(max(3, args.warmup)):
+        pipe.submit(host_pipe, outs_host[i % 2])
+    torch.cuda.synchronize()
+    barrier(world, device)
+    e2, e3 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2.record(stream)
+    pipe.start_after(e2)
+    for i in range(E):
+        pipe.submit(host_pipe, outs_host[i % 2])
+    pipe.drain(stream)
+    e3.record(stream)
+    torch.cuda.synchronize()
+    barrier(world, device)
+    pa.sync_status()
+    e2e_sec = reduce_max(e2.elapsed_time(e3) / 1e3, world, device)
     e2e_value, _ = aggregate(w.kv_bytes, w.seq_tokens, E, e2e_sec, world, device)
 
     peak, peak_kind = measured_peaks()
@@ -426,7 +450,12 @@ def run_ours(args, rank, local, world):
         },
         "cpu_baseline": cpu,
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": int(h2d),
-                "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_sec / E * 1e3, 4)},
+                "d2h_bytes_per_step": int(d2h), "ms_per_step": round(e2e_sec / E * 1e3, 4),
+                "how": "DecodePipeline: pinned host inputs in and the output out every step, "
+                       "on two copy streams overlapped with the neighbouring steps' kernels"},
+        "e2e_serial": {"value": round(serial_value, 2), "unit": "GB/s",
+                       "ms_per_step": round(serial_sec / E * 1e3, 4),
+                       "how": "the same copies and kernels in one stream, one step after another"},
         "gpu_launches": launches_per_step * K,
         "clocks": clocks.summary(),
     }
