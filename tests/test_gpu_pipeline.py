@@ -38,4 +38,6 @@ def test_pipeline_matches_direct_calls(pa, name):
     pa.sync_status()
     for o in outs:
         assert torch.equal(o, ref.cpu()), f"{name}: pipelined output differs"
-    assert torch.equal(kp.cpu(), kd.cpu()) and torch.equal(vp.cpu(), vd.cpu())
+    # the pools hold NaN poison in unused slots: compare their bytes
+    raw = lambda t: t.contiguous().view(torch.uint8).cpu()
+    assert torch.equal(raw(kp), raw(kd)) and torch.equal(raw(vp), raw(vd))
