@@ -40,7 +40,9 @@
  *   src_dst_pairs int64 [P, 2]
  *
  * Supported: D in {64, 128}; bs in {16, 32}; Hq a multiple of Hkv with
- * Hq / Hkv <= 8; cache dtype f16 (q f16), bf16 (q bf16) or e4m3 (q f16 or
+ * Hq / Hkv <= 64 for pa_decode (a kv head's query heads are taken 8 at a
+ * time: more than 8 read its blocks once per group of 8), <= 8 for the
+ * shared-prefix decode; cache dtype f16 (q f16), bf16 (q bf16) or e4m3 (q f16 or
  * bf16).  With an e4m3 cache the query is converted to fp16 for the tensor-
  * core products, so |q| must stay inside the fp16 range (< 65504).
  */
@@ -68,7 +70,7 @@ typedef enum pa_status {
   PA_ERR_NULL = 1,          /* a required pointer is NULL */
   PA_ERR_DTYPE = 2,         /* unsupported dtype or dtype combination */
   PA_ERR_SHAPE = 3,         /* unsupported or inconsistent size */
-  PA_ERR_HEADS = 4,         /* Hq not a multiple of Hkv, or Hq / Hkv > 8 */
+  PA_ERR_HEADS = 4,         /* Hq not a multiple of Hkv, or too many query heads per kv head */
   PA_ERR_RANGE = 5,         /* an index is out of range (pa_validate_*) */
   PA_ERR_ALIAS = 6,         /* duplicate destinations, or a destination that is
                                also a source (pa_validate_*) */

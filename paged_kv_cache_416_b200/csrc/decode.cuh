@@ -41,7 +41,8 @@ enum CacheKind : int { kCacheF16 = 0, kCacheBF16 = 1, kCacheE4M3 = 2 };
 
 constexpr int kDecodeWarps = 4;
 constexpr int kDecodeThreads = kDecodeWarps * 32;
-constexpr int kMaxGroup = 8;          // packed query heads per kv head (MMA N)
+constexpr int kMaxGroup = 8;          // packed query heads per work item (MMA N); a kv
+                                      // head with more query heads is several items
 constexpr int kBarrierBytes = 256;    // mbarrier area at the start of smem
 constexpr int kTileAlign = 1024;      // swizzled tiles start on this boundary
 constexpr int kMaxRanges = 1024;      // context ranges per sequence (fused merge uses smem)
@@ -124,6 +125,7 @@ struct DecodeArgs {
   float* lse_part;         // workspace: [ranges * Hq]
   float* o_part;           // workspace: [ranges * Hq * D]
   int num_seqs, hq, hkv, group, max_blocks, num_blocks, max_ctx, split_tokens;
+  int ncg;                 // column groups per kv head: ceil(group / 8) items read its blocks
   float sl2;               // scale * k_scale * log2(e)
   float out_scale;         // v_scale
 };
@@ -296,7 +298,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
   auto fetch_next = [&]() {
     const int it = atomicAdd(a.counter, 1);
     s_item = it;
-    if (it < total) s_desc = a.order[it / a.hkv];
+    if (it < total) s_desc = a.order[it / (a.hkv * a.ncg)];
   };
   if (threadIdx.x == 0) fetch_next();
   __syncthreads();
@@ -307,7 +309,11 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
 
     // ---- item -> (sequence, range, kv head); kv heads innermost, so the
     // heads of one range run side by side and share the table's cache lines
-    const int kvh = item % a.hkv;
+    // the kv head's query heads are cut into column groups of at most 8 (the
+    // MMA's N); each group is its own item over the same blocks
+    const int kvh_cg = item % (a.hkv * a.ncg);
+    const int kvh = kvh_cg / a.ncg, cg = kvh_cg % a.ncg;
+    const int ncols = min(kMaxGroup, a.group - cg * kMaxGroup);  // heads of this item
     const int4 desc = s_desc;
     const int seq = desc.x;
     const int split = desc.y;
@@ -318,7 +324,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
     const int nblk = t1 > t0 ? (t1 + BS - 1) / BS - jb0 : 0;
     const int nb_w = nblk > warp ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
     const int32_t* table = a.block_tables + static_cast<int64_t>(seq) * a.max_blocks;
-    const int h0 = kvh * a.group;
+    const int h0 = kvh * a.group + cg * kMaxGroup;
 
     // ---- block-table entries of the warp's blocks, prefetched in registers:
     // lane l holds the entry of the warp's block (32 * chunk + l); tab_cur is
@@ -364,7 +370,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
     // ---- query fragments (B operand of S^T = K Q^T): rows = dims, cols = heads
     uint32_t qf[C::kDimTiles][2];
     {
-      const bool hv = g < a.group;
+      const bool hv = g < ncols;
       const uint16_t* qrow = reinterpret_cast<const uint16_t*>(a.q) +
                              (static_cast<int64_t>(seq) * a.hq + h0 + (hv ? g : 0)) * D;
 #pragma unroll
@@ -582,7 +588,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
     __syncthreads();
     {
       constexpr int kVec = 8;
-      const int units = a.group * (D / kVec);
+      const int units = ncols * (D / kVec);
       for (int u = threadIdx.x; u < units; u += kDecodeThreads) {
         const int h = u / (D / kVec);
         const int d0 = (u % (D / kVec)) * kVec;
@@ -638,7 +644,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
       __threadfence();
       __syncthreads();
       if (threadIdx.x == 0) {
-        const int prev = atomicAdd(&a.arrived[seq * a.hkv + kvh], 1);
+        const int prev = atomicAdd(&a.arrived[(seq * a.hkv + kvh) * a.ncg + cg], 1);
         s_flag = (prev == nsplit - 1) ? 1 : 0;
       }
       __syncthreads();
@@ -649,23 +655,23 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
         // and the weights w_i = 2^(lse_i - max), (3) the weighted sum of the
         // partial outputs with independent (unrolled) loads
         float* lse_s = reinterpret_cast<float*>(ring);           // [nsplit][group]
-        float* wsum_s = lse_s + nsplit * a.group;                // [group]
+        float* wsum_s = lse_s + nsplit * ncols;                  // [ncols]
         const int64_t base = static_cast<int64_t>(a.seq_off[seq]) * a.hq + h0;
-        const int npairs = nsplit * a.group;
+        const int npairs = nsplit * ncols;
         for (int k = threadIdx.x; k < npairs; k += kDecodeThreads) {
-          const int i = k / a.group, h = k % a.group;
+          const int i = k / ncols, h = k % ncols;
           lse_s[k] = __ldcg(a.lse_part + base + static_cast<int64_t>(i) * a.hq + h);
         }
         __syncthreads();
-        for (int h = warp; h < a.group; h += kDecodeWarps) {
+        for (int h = warp; h < ncols; h += kDecodeWarps) {
           float M = -INFINITY;
-          for (int i = lane; i < nsplit; i += 32) M = fmaxf(M, lse_s[i * a.group + h]);
+          for (int i = lane; i < nsplit; i += 32) M = fmaxf(M, lse_s[i * ncols + h]);
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
           float W = 0.f;
           for (int i = lane; i < nsplit; i += 32) {
-            const float w = (M == -INFINITY) ? 0.f : fast_exp2(lse_s[i * a.group + h] - M);
-            lse_s[i * a.group + h] = w;  // now the weight
+            const float w = (M == -INFINITY) ? 0.f : fast_exp2(lse_s[i * ncols + h] - M);
+            lse_s[i * ncols + h] = w;  // now the weight
             W += w;
           }
 #pragma unroll
@@ -674,7 +680,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
         }
         __syncthreads();
         constexpr int kVec = 4;
-        const int units = a.group * (D / kVec);
+        const int units = ncols * (D / kVec);
         for (int u = threadIdx.x; u < units; u += kDecodeThreads) {
           const int h = u / (D / kVec);
           const int d0 = (u % (D / kVec)) * kVec;
@@ -682,7 +688,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
           const float* op = a.o_part + (base + h) * D + d0;
 #pragma unroll 8
           for (int i = 0; i < nsplit; ++i) {
-            const float w = lse_s[i * a.group + h];
+            const float w = lse_s[i * ncols + h];
             const float4 x = __ldcg(reinterpret_cast<const float4*>(op + static_cast<int64_t>(i) * a.hq * D));
             o0 += w * x.x; o1 += w * x.y; o2 += w * x.z; o3 += w * x.w;
           }

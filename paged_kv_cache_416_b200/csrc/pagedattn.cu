@@ -70,6 +70,12 @@ int64_t round_up(int64_t a, int64_t b) { return cdiv(a, b) * b; }
 // fixed so that the split, and so the rounding of every result, depends on
 // the call's arguments only and not on the device it runs on.
 constexpr int64_t kPlanCtas = 296;
+// query heads per kv head pa_decode accepts: column groups of kMaxGroup heads,
+// each its own work item over the kv head's blocks
+constexpr int kMaxQHeadsPerKv = 64;
+int32_t col_groups(int32_t hq, int32_t hkv) {
+  return hkv > 0 ? std::max<int32_t>(1, static_cast<int32_t>(cdiv(hq / hkv, pa::kMaxGroup))) : 1;
+}
 constexpr int64_t kMinSplit = 256;        // shortest range worth its partial
 constexpr int64_t kLongContext = 4096;    // above this, cap ranges ...
 constexpr int64_t kLongSplit = 1024;      // ... at this many tokens
@@ -417,7 +423,8 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads, int32_t n
       (block_size != 16 && block_size != 32) || max_context_len < 0 || split_tokens < 0)
     return 0;
   const int32_t S = choose_split(num_seqs, num_kv_heads, block_size, max_context_len, split_tokens);
-  return ws_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, S).bytes;
+  return ws_layout(num_seqs, num_q_heads, num_kv_heads * col_groups(num_q_heads, num_kv_heads),
+                   head_dim, max_context_len, S).bytes;
 }
 
 pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_pool,
@@ -442,9 +449,10 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_po
     return fail(PA_ERR_SHAPE, "pa_decode: max_context_len %d exceeds max_blocks_per_seq * bs",
                 max_context_len);
   if (num_q_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
-      num_q_heads / num_kv_heads > pa::kMaxGroup)
+      num_q_heads / num_kv_heads > kMaxQHeadsPerKv)
     return fail(PA_ERR_HEADS, "pa_decode: num_q_heads %d must be a multiple of num_kv_heads %d "
-                "with at most %d query heads per kv head", num_q_heads, num_kv_heads, pa::kMaxGroup);
+                "with at most %d query heads per kv head", num_q_heads, num_kv_heads,
+                kMaxQHeadsPerKv);
   if (!std::isfinite(scale) || (fp8 && !(std::isfinite(k_scale) && k_scale > 0.f &&
                                          std::isfinite(v_scale) && v_scale > 0.f)))
     return fail(PA_ERR_SHAPE, "pa_decode: scales must be finite (and positive for e4m3)");
@@ -452,7 +460,9 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_po
   if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens)
     return fail(PA_ERR_NULL, "pa_decode: null pointer");
   const int32_t S = choose_split(num_seqs, num_kv_heads, block_size, max_context_len, split_tokens);
-  const WsLayout w = ws_layout(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, S);
+  const int32_t ncg = col_groups(num_q_heads, num_kv_heads);
+  const WsLayout w = ws_layout(num_seqs, num_q_heads, num_kv_heads * ncg, head_dim,
+                               max_context_len, S);
   if (!workspace || workspace_bytes < w.bytes || (reinterpret_cast<uintptr_t>(workspace) & 255))
     return fail(PA_ERR_WORKSPACE, "pa_decode: workspace needs %zu bytes, 256-byte aligned (got %zu)",
                 w.bytes, workspace_bytes);
@@ -491,15 +501,16 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_po
   a.split_tokens = w.split ? S : std::max(S, max_context_len);
   a.sl2 = scale * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
   a.out_scale = fp8 ? v_scale : 1.f;
+  a.ncg = ncg;
 
   pa::plan_kernel<<<1, 1024, 0, st>>>(context_lens, num_seqs, max_context_len, max_blocks_per_seq,
-                                      block_size, a.split_tokens, num_kv_heads,
+                                      block_size, a.split_tokens, num_kv_heads * ncg,
                                       reinterpret_cast<int32_t*>(ws + w.counter),
                                       reinterpret_cast<int32_t*>(ws + w.total),
                                       reinterpret_cast<int32_t*>(ws + w.seq_off),
                                       reinterpret_cast<int4*>(ws + w.order),
                                       w.split ? reinterpret_cast<int32_t*>(ws + w.arrived) : nullptr);
-  const int64_t items_upper = w.ranges * num_kv_heads;
+  const int64_t items_upper = w.ranges * num_kv_heads * ncg;
   const bool qbf = q_dtype == PA_BF16;
   pa_status s;
   if (cache_dtype == PA_F16)

@@ -76,7 +76,8 @@ def _decode(pa, **kw):
     (dict(bs=8), 3),
     (dict(max_ctx=65), 3),                       # exceeds max_blocks * bs
     (dict(hq=7), 4),
-    (dict(hq=32, hkv=2), 4),                     # 16 query heads per kv head
+    (dict(hq=160, hkv=2), 4),                    # 80 query heads per kv head (> 64)
+    (dict(hq=32, hkv=2), 1),                     # 16 per kv head: two column groups, valid
     (dict(cache_dtype=2, k_scale=0.0), 3),
     (dict(scale=float("inf")), 3),
     (dict(), 1),                                 # valid sizes, null pointers

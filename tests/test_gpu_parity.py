@@ -353,3 +353,18 @@ def test_decode_short_contexts_many_sequences(pa, cache):
     out, _, _ = gpu_step(pa, w)
     ref, _, _ = oracle_step(w)
     assert_attention_close(as_f64(out), ref, f"short contexts {cache}")
+
+
+@pytest.mark.parametrize("hq,hkv,cache,split", [(96, 8, "bf16", 0), (128, 8, "bf16", 64),
+                                                (16, 1, "e4m3", 32), (48, 4, "f16", 0)])
+def test_decode_more_than_eight_query_heads_per_kv_head(pa, hq, hkv, cache, split):
+    """12 and 16 query heads per kv head: the heads are taken 8 at a time, each
+    group its own work item over the kv head's blocks (split ranges merged
+    per group)."""
+    rng = np.random.default_rng(hq + hkv)
+    lens = rng.integers(1, 300, size=9)
+    qd = "f16" if cache == "f16" else "bf16"
+    w = W._generic("wide_groups", lens, hq, hkv, 128, 16, qd, cache, seed=hq, device="cpu")
+    out, _, _ = gpu_step(pa, w, split_tokens=split)
+    ref, _, _ = oracle_step(w)
+    assert_attention_close(as_f64(out), ref, f"{hq}/{hkv} {cache} split {split}")
