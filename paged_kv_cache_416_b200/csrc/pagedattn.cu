@@ -638,9 +638,12 @@ pa_status pa_prefill(void* out, const void* q, pa_dtype q_dtype, const void* k_p
       max_blocks_per_seq <= 0 || !cache_shape_ok(num_blocks, block_size, num_kv_heads, head_dim) ||
       static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * block_size)
     return fail(PA_ERR_SHAPE, "pa_prefill: unsupported sizes (head_dim must be %d)", pa::kPfD);
+  // a CTA takes T = floor(128 / G) new tokens (T * G rows of its 128; the
+  // rest are padding rows that are never loaded or written)
   if (num_q_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
-      pa::kPfRows % (num_q_heads / num_kv_heads) != 0)
-    return fail(PA_ERR_HEADS, "pa_prefill: num_q_heads / num_kv_heads must divide %d", pa::kPfRows);
+      num_q_heads / num_kv_heads > pa::kPfRows)
+    return fail(PA_ERR_HEADS, "pa_prefill: num_q_heads must be a multiple of num_kv_heads with "
+                "at most %d query heads per kv head", pa::kPfRows);
   if (!std::isfinite(scale)) return fail(PA_ERR_SHAPE, "pa_prefill: scale must be finite");
   if (num_seqs == 0 || max_query_len == 0) return ok();
   if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens || !query_start)

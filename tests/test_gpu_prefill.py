@@ -52,11 +52,19 @@ def test_prefill_of_one_token_equals_decode(pa):
     assert_attention_close(as_f64(out), ref(pw), "prefill one token")
 
 
+@pytest.mark.parametrize("hq,hkv", [(12, 4), (96, 8)])
+def test_prefill_group_sizes_that_do_not_divide_the_tile(pa, hq, hkv):
+    # G = 3 and G = 12: a CTA takes floor(128 / G) tokens, the other rows of
+    # its 128 are padding
+    pw = W.prefill(ctxs=(90, 200), nqs=(90, 61), hq=hq, hkv=hkv, bs=16, dtype="bf16")
+    assert_attention_close(as_f64(run(pa, pw)), ref(pw), f"prefill {hq}/{hkv}")
+
+
 def test_prefill_rejects_unsupported_shapes(pa):
-    pw = W.prefill(ctxs=(40,), nqs=(40,), hq=12, hkv=4, bs=16, dtype="bf16")  # G = 3
+    pw = W.prefill(ctxs=(40,), nqs=(40,), hq=16, hkv=4, d=64, bs=16, dtype="bf16")  # D = 64
     with pytest.raises(pa.PagedAttnError) as e:
         run(pa, pw)
-    assert e.value.status == 4
+    assert e.value.status == 3
 
 
 def grow_keys(pw, rate):
