@@ -297,7 +297,7 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype q_dtype,
  * h / (Hq / Hkv)):
  *   out = sum_{t <= p} softmax_t(scale * <q, K_s[t]>) V_s[t]
  * accumulated in fp32, rounded to q's dtype.  query_start is int32 [B + 1],
- * device memory.  Supported: head_dim 128; q and cache both f16 or both
+ * device memory.  Supported: head_dim 64 or 128; q and cache both f16 or both
  * bf16; G = Hq / Hkv <= 128 (a CTA takes floor(128 / G) new tokens);
  * block_size 16 or 32.  max_query_len must
  * bound every n_s (rows past it are not computed) and max_context_len every

@@ -634,10 +634,11 @@ pa_status pa_prefill(void* out, const void* q, pa_dtype q_dtype, const void* k_p
   if (!valid_dtype(q_dtype) || !valid_dtype(cache_dtype) || q_dtype == PA_FP8_E4M3 ||
       cache_dtype != q_dtype)
     return fail(PA_ERR_DTYPE, "pa_prefill: q and the cache must share a 16-bit dtype");
-  if (head_dim != pa::kPfD || num_seqs < 0 || max_query_len < 0 || max_context_len < 0 ||
+  if ((head_dim != 64 && head_dim != pa::kPfMaxD) || num_seqs < 0 || max_query_len < 0 || max_context_len < 0 ||
       max_blocks_per_seq <= 0 || !cache_shape_ok(num_blocks, block_size, num_kv_heads, head_dim) ||
       static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * block_size)
-    return fail(PA_ERR_SHAPE, "pa_prefill: unsupported sizes (head_dim must be %d)", pa::kPfD);
+    return fail(PA_ERR_SHAPE, "pa_prefill: unsupported sizes (head_dim must be 64 or %d)",
+                pa::kPfMaxD);
   // a CTA takes T = floor(128 / G) new tokens (T * G rows of its 128; the
   // rest are padding rows that are never loaded or written)
   if (num_q_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
@@ -685,12 +686,14 @@ pa_status pa_prefill(void* out, const void* q, pa_dtype q_dtype, const void* k_p
   };
   pa_status ls;
   const bool bf = q_dtype == PA_BF16;
-  if (block_size == 16)
-    ls = bf ? launch(pa::prefill_kernel<true, 16>, pa::PrefillCfg<16>::kSmemBytes)
-            : launch(pa::prefill_kernel<false, 16>, pa::PrefillCfg<16>::kSmemBytes);
+#define PA_PF_LAUNCH(BS_, D_)                                                              \
+  (bf ? launch(pa::prefill_kernel<true, BS_, D_>, pa::PrefillCfg<BS_, D_>::kSmemBytes)     \
+      : launch(pa::prefill_kernel<false, BS_, D_>, pa::PrefillCfg<BS_, D_>::kSmemBytes))
+  if (head_dim == 64)
+    ls = block_size == 16 ? PA_PF_LAUNCH(16, 64) : PA_PF_LAUNCH(32, 64);
   else
-    ls = bf ? launch(pa::prefill_kernel<true, 32>, pa::PrefillCfg<32>::kSmemBytes)
-            : launch(pa::prefill_kernel<false, 32>, pa::PrefillCfg<32>::kSmemBytes);
+    ls = block_size == 16 ? PA_PF_LAUNCH(16, 128) : PA_PF_LAUNCH(32, 128);
+#undef PA_PF_LAUNCH
   if (ls != PA_OK) return ls;
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pa_prefill launch");

@@ -56,19 +56,20 @@ constexpr int kPfRowThreads = 128;  // warps 0-3: thread r owns query row r (TME
 constexpr int kPfThreads = 192;     // + warp 4: MMA issue, warp 5: TMA loads
 constexpr int kPfRows = 128;      // MMA M: (token, head) rows per CTA
 constexpr int kPfKeys = 64;       // keys per tile
-constexpr int kPfD = 128;         // head_dim
+constexpr int kPfMaxD = 128;      // head_dim 64 or 128: one or two 64-dim (128-byte) halves
 constexpr int kPfTmemCols = 256;  // S/P buffers [0, 64) and [64, 128), O [128, 256)
 constexpr float kPfRescaleLog2 = 8.f;  // rescale O when the max grows by more than this
 
-template <int BS>
+template <int BS, int D>
 struct PrefillCfg {
-  static constexpr int kQBytes = kPfRows * kPfD * 2;      // [2 dim halves][128 rows][128 B]
-  static constexpr int kKBytes = kPfKeys * kPfD * 2;      // [2 dim halves][64 keys][128 B]
+  static constexpr int kHalves = D / 64;                  // 128-byte dim halves of a row
+  static constexpr int kQBytes = kPfRows * D * 2;         // [halves][128 rows][128 B]
+  static constexpr int kKBytes = kPfKeys * D * 2;         // [halves][64 keys][128 B]
   static constexpr int kBlocksPerTile = kPfKeys / BS;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;           // 2 stages
   static constexpr int kOffV = kOffK + 2 * kKBytes;       // 2 stages
-  static constexpr int kTiles = kOffV + 2 * kKBytes;      // 96 KiB: two CTAs per SM
+  static constexpr int kTiles = kOffV + 2 * kKBytes;      // 96 KiB at D 128: two CTAs per SM
   static constexpr int kHead = 256;                       // 12 mbarriers, TMEM slot, block ids
   static constexpr int kSmemBytes = kTiles + kHead;
   static_assert(kPfKeys % BS == 0, "a key tile holds whole blocks");
@@ -76,7 +77,7 @@ struct PrefillCfg {
 
 struct PrefillArgs {
   // Pools viewed as 5-D bytes (x, token, half, kv head, block) =
-  // (128, bs, 2, Hkv, N); box (128, bs, 1, 1, 1): one dim half of one block.
+  // (128, bs, D / 64, Hkv, N); box (128, bs, 1, 1, 1): one dim half of one block.
   CUtensorMap tmap_k;
   CUtensorMap tmap_v;
   void* out;                   // [total_q, Hq, D], q's dtype
@@ -95,9 +96,10 @@ __device__ __forceinline__ uint32_t swz128(int r, int c) {
 
 // One CTA per (query tile, kv head, sequence): grid (ceil(max_query_len / T),
 // Hkv, B) with T = 128 / G tokens; CTAs past a sequence's new tokens exit.
-template <bool kBF16, int BS>
+template <bool kBF16, int BS, int D>
 __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_constant__ PrefillArgs a) {
-  using C = PrefillCfg<BS>;
+  using C = PrefillCfg<BS, D>;
+  static_assert(D == 64 || D == 128, "head_dim 64 or 128");
   extern __shared__ __align__(1024) uint8_t pf_smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool producer = warp >= kPfRowThreads / 32;     // warps 4 (MMA) and 5 (loads)
@@ -115,11 +117,11 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
   const int hr = kvh * G + r % G;             // its query head
   const bool row_ok = !producer && tok < nt;
   const int ctx = a.context_lens[s];
-  const int64_t orow_off = (static_cast<int64_t>(q0 + i0 + tok) * a.hq + hr) * (kPfD * 2 / 16);
+  const int64_t orow_off = (static_cast<int64_t>(q0 + i0 + tok) * a.hq + hr) * (D * 2 / 16);
   if (ctx < n || ctx > a.max_ctx || ctx > a.max_blocks * BS) {
     if (tid == 0) record_error(PA_ERR_DEVICE_BOUNDS);
     if (row_ok)
-      for (int j = 0; j < kPfD * 2 / 16; ++j)
+      for (int j = 0; j < D * 2 / 16; ++j)
         reinterpret_cast<uint4*>(a.out)[orow_off + j] = make_uint4(0, 0, 0, 0);
     return;
   }
@@ -164,7 +166,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     uint32_t bytes = 0;
 #pragma unroll
     for (int b = 0; b < C::kBlocksPerTile; ++b)
-      if (phys[b] >= 0) bytes += 2u * BS * 128u;
+      if (phys[b] >= 0) bytes += C::kHalves * BS * 128u;
     const uint32_t bar = (is_v ? full_v : full_k) + 8 * st;
     const uint32_t dst = (is_v ? sV : sK) + st * C::kKBytes;
     const CUtensorMap* map = is_v ? &a.tmap_v : &a.tmap_k;
@@ -173,7 +175,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     for (int b = 0; b < C::kBlocksPerTile; ++b) {
       if (phys[b] < 0) continue;
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf)
+      for (int hf = 0; hf < C::kHalves; ++hf)
         tma_load_5d(dst + hf * (kPfKeys * 128) + b * BS * 128, map, 0, 0, hf, kvh, phys[b], bar);
     }
   };
@@ -201,10 +203,10 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     tmem_alloc(tmem_slot_s, kPfTmemCols);
     tmem_relinquish();
   }
-  if (!producer) {  // Q tile: thread r writes its row (256 B) into the two dim halves
+  if (!producer) {  // Q tile: thread r writes its row (2 D bytes) into the dim halves
     const uint4* src = reinterpret_cast<const uint4*>(a.q) + orow_off;
 #pragma unroll
-    for (int j = 0; j < 16; ++j) {
+    for (int j = 0; j < D / 8; ++j) {
       const uint4 v = row_ok ? src[j] : make_uint4(0, 0, 0, 0);
       *reinterpret_cast<uint4*>(base + C::kOffQ + (j >> 3) * (kPfRows * 128) + swz128(r, j & 7)) = v;
     }
@@ -246,14 +248,14 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
   if (mma_warp) {
     // ======================= MMA warp (lane 0 issues) ====================
     constexpr uint32_t kIdescS = umma_idesc_f16(kPfRows, kPfKeys, kBF16);
-    constexpr uint32_t kIdescO = umma_idesc_f16(kPfRows, kPfD, kBF16, /*b_mn_major=*/true);
+    constexpr uint32_t kIdescO = umma_idesc_f16(kPfRows, D, kBF16, /*b_mn_major=*/true);
     auto issue_s = [&](int kt) {  // S(kt) = Q K(kt)^T; then K(kt)'s stage is free
       wait(full_k + 8 * (kt & 1), (kt >> 1) & 1);
       if (failed || lane != 0) return;
       tc_fence_after_sync();
       const uint32_t k_st = sK + (kt & 1) * C::kKBytes;
 #pragma unroll
-      for (int k = 0; k < kPfD / 16; ++k)
+      for (int k = 0; k < D / 16; ++k)
         umma_f16(tbuf(kt), umma_desc_k128(sQ + (k >> 2) * (kPfRows * 128) + (k & 3) * 32),
                  umma_desc_k128(k_st + (k >> 2) * (kPfKeys * 128) + (k & 3) * 32), kIdescS,
                  k > 0 ? 1u : 0u);
@@ -277,7 +279,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
       const int bad = bad_of(kt);
       if ((kt + 1) * kPfKeys > ctx || bad) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
+        for (int i = 0; i < 2 * C::kHalves; ++i) {  // (half, key) rows of the stage
           const int row = lane + 32 * i, key = row & (kPfKeys - 1), hf = row >> 6;
           if (kt * kPfKeys + key >= ctx || ((bad >> (key / BS)) & 1)) {
             uint4* dst = reinterpret_cast<uint4*>(base + C::kOffV + st * C::kKBytes +
@@ -429,7 +431,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
         {  // tcgen05.ld / st are warp-wide
           const uint64_t al2 = f2(alpha, alpha);
 #pragma unroll
-          for (int c = 0; c < kPfD / 32; ++c) {
+          for (int c = 0; c < D / 32; ++c) {
             uint32_t ot[32];
             tmem_ld32(tO + lane_off + 32 * c, ot);
             tmem_wait_ld();
@@ -460,7 +462,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
     uint4* const orow = reinterpret_cast<uint4*>(a.out) + orow_off;
 #pragma unroll
-    for (int c = 0; c < kPfD / 32; ++c) {
+    for (int c = 0; c < D / 32; ++c) {
       uint32_t ot[32];
       tmem_ld32(tO + lane_off + 32 * c, ot);
       tmem_wait_ld();

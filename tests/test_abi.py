@@ -156,7 +156,8 @@ def _prefill(pa, **kw):
 @pytest.mark.parametrize("kw,status", [
     (dict(cache_dtype=2), 2),                    # tensor-core path: 16-bit caches only
     (dict(q_dtype=0), 2),
-    (dict(D=64), 3),
+    (dict(D=64), 1),                             # head_dim 64: valid
+    (dict(D=96), 3),
     (dict(hq=24, hkv=8), 1),                     # G = 3: floor(128 / 3) tokens a CTA, valid
     (dict(hq=258, hkv=2), 4),                    # G = 129 > 128 rows
     (dict(), 1),

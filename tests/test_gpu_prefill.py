@@ -60,11 +60,24 @@ def test_prefill_group_sizes_that_do_not_divide_the_tile(pa, hq, hkv):
     assert_attention_close(as_f64(run(pa, pw)), ref(pw), f"prefill {hq}/{hkv}")
 
 
+@pytest.mark.parametrize("hq,hkv,bs,dtype", [(16, 4, 16, "bf16"), (8, 8, 32, "f16")])
+def test_prefill_head_dim_64(pa, hq, hkv, bs, dtype):
+    # one 128-byte dim half per row: half the S k-steps, an O product of N = 64
+    pw = W.prefill(ctxs=(40, 300, 130), nqs=(40, 90, 130), hq=hq, hkv=hkv, d=64, bs=bs,
+                   dtype=dtype)
+    assert_attention_close(as_f64(run(pa, pw)), ref(pw), f"prefill D64 {hq}/{hkv} bs{bs} {dtype}")
+
+
 def test_prefill_rejects_unsupported_shapes(pa):
-    pw = W.prefill(ctxs=(40,), nqs=(40,), hq=16, hkv=4, d=64, bs=16, dtype="bf16")  # D = 64
-    with pytest.raises(pa.PagedAttnError) as e:
-        run(pa, pw)
-    assert e.value.status == 3
+    pw = W.prefill(ctxs=(40,), nqs=(40,), hq=16, hkv=4, d=64, bs=16, dtype="bf16")
+    b = pw.base
+    with pytest.raises(pa.PagedAttnError) as e:  # e4m3 caches take no tensor-core path
+        pa.prefill(pw.q.cuda(), b.k_pool.cuda().view(torch.float8_e4m3fn),
+                   b.v_pool.cuda().view(torch.float8_e4m3fn),
+                   torch.from_numpy(b.block_tables).cuda(), torch.from_numpy(b.context_lens).cuda(),
+                   torch.from_numpy(pw.query_start).cuda(), b.scale, pw.max_query_len,
+                   b.max_context_len)
+    assert e.value.status == 2
 
 
 def grow_keys(pw, rate):
