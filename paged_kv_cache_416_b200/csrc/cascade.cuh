@@ -98,6 +98,8 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
     for (int s = 0; s < kStages; ++s) mbar_init(bar0 + 8 * s, 1);
     mbar_init_fence();
   }
+  // launched behind cascade_plan_kernel: nothing from global memory before it is done
+  grid_dependency_wait();
   if (threadIdx.x == 0) {
     prefetch_tensormap(&a.tmap_k);
     prefetch_tensormap(&a.tmap_v);
@@ -645,6 +647,7 @@ __global__ void __launch_bounds__(1024) cascade_plan_kernel(
     int32_t* counter, int32_t* arrived) {
   __shared__ int n_chunks, n_used, tv_sum, v_max, n_slots;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  grid_launch_dependents();  // the cascade grid may set up while the plan runs
   if (tid == 0) {
     n_chunks = n_used = tv_sum = v_max = n_slots = 0;
     *counter = 0;

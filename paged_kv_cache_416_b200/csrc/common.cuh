@@ -35,6 +35,19 @@ __device__ __forceinline__ unsigned long long global_timer_ns() {
   return t;
 }
 
+// ------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may be scheduled
+// while the kernel before it still runs, once that kernel's CTAs have all
+// executed grid_launch_dependents (or exited).  grid_dependency_wait blocks
+// until the kernel before it has completed and its writes are visible; on a
+// normal launch both are no-ops.
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+__device__ __forceinline__ void grid_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");

@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
   __shared__ int carry;
   __shared__ int hist[kPlanBuckets];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  grid_launch_dependents();  // the decode grid may set up while the plan runs
   const int max_nb = (min(S, max_ctx) + bs - 1) / bs;  // blocks of the longest range
   auto bucket = [&](int nb) {  // longer ranges -> higher class
     return max_nb < kPlanBuckets ? nb : static_cast<int>((static_cast<int64_t>(nb) * (kPlanBuckets - 1)) / max_nb);
@@ -287,6 +288,8 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
     prefetch_tensormap(&a.tmap_k);
     prefetch_tensormap(&a.tmap_v);
   }
+  // launched behind plan_kernel: nothing from global memory before it is done
+  grid_dependency_wait();
   __syncthreads();
 
   const int total = *a.total;

@@ -208,6 +208,26 @@ pa_status encode_pool_map(CUtensorMap* map, const void* pool, int32_t num_blocks
 }
 
 // ------------------------------------------------------ decode dispatch
+// Launch a persistent attention kernel behind its planning kernel with
+// programmatic stream serialization: its CTAs are scheduled, initialise their
+// barriers and prefetch the tensor maps while the plan finishes, then wait in
+// grid_dependency_wait for the plan's writes.
+template <typename Args>
+cudaError_t launch_behind_plan(void (*kern)(Args), unsigned grid, int threads, int smem_bytes,
+                               cudaStream_t stream, const Args& args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem_bytes);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args);
+}
+
 template <int CK, bool kQBF16, int D, int BS>
 pa_status launch_decode_main(const pa::DecodeArgs& args, int64_t items_upper, int dev,
                              cudaStream_t stream) {
@@ -225,7 +245,9 @@ pa_status launch_decode_main(const pa::DecodeArgs& args, int64_t items_upper, in
   }
   const int64_t grid = std::max<int64_t>(
       1, std::min<int64_t>(items_upper, static_cast<int64_t>(device_sms(dev)) * occ[dev]));
-  kern<<<static_cast<unsigned>(grid), pa::kDecodeThreads, C::kSmemBytes, stream>>>(args);
+  const cudaError_t e = launch_behind_plan(kern, static_cast<unsigned>(grid), pa::kDecodeThreads,
+                                           C::kSmemBytes, stream, args);
+  if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
   return PA_OK;
 }
 
@@ -256,7 +278,9 @@ pa_status launch_cascade(const pa::CascadeArgs& args, int64_t items_upper, int d
   }
   const int64_t grid = std::max<int64_t>(
       1, std::min<int64_t>(items_upper, static_cast<int64_t>(device_sms(dev)) * occ[dev]));
-  kern<<<static_cast<unsigned>(grid), pa::kDecodeThreads, C::kSmemBytes, stream>>>(args);
+  const cudaError_t e = launch_behind_plan(kern, static_cast<unsigned>(grid), pa::kDecodeThreads,
+                                           C::kSmemBytes, stream, args);
+  if (e != cudaSuccess) return cuda_fail(e, "pa_decode_shared_prefix launch");
   return PA_OK;
 }
 
