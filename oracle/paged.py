@@ -185,12 +185,19 @@ def prefill(q_raw, q_dtype: str, k_pool, v_pool, cache_dtype: str, block_tables,
         K = gather(decode_cache(k_pool[ids], cache_dtype, k_scale), np.arange(nb), ctx)
         V = gather(decode_cache(v_pool[ids], cache_dtype, v_scale), np.arange(nb), ctx)
         for i in range(n):
-            pos = ctx - n + i
+            nk = visible_keys(ctx, n, i)
             for h in range(hq):
                 kv = h // group
-                w = attention_weights(q[qs[s] + i, h], K[: pos + 1, kv, :], scale)
-                out[qs[s] + i, h] = w @ V[: pos + 1, kv, :]
+                w = attention_weights(q[qs[s] + i, h], K[:nk, kv, :], scale)
+                out[qs[s] + i, h] = w @ V[:nk, kv, :]
     return out
+
+
+def visible_keys(context_len: int, num_new: int, i: int) -> int:
+    """Keys new token i of a chunk of ``num_new`` sees: it sits at position
+    ``context_len - num_new + i`` (the chunk is the end of the context) and
+    attends causally to positions 0 .. that position."""
+    return context_len - num_new + i + 1
 
 
 def shared_prefix_blocks(block_tables, context_lens, members, block_size: int) -> int:

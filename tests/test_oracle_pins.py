@@ -564,3 +564,59 @@ def test_shared_prefix_decode_equals_plain_decode(phase):
     np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
     # every sample shares its prompt's full blocks: 64 + r tokens -> 4 blocks at bs 16
     assert (pre == 4).all()
+
+
+# ---- planted mistakes in the prefill, shared-prefix and hash oracles -------
+@pytest.mark.parametrize("bad", [
+    lambda orig: (lambda ctx, n, i: orig(ctx, n, i) + 1),           # one future key seen
+    lambda orig: (lambda ctx, n, i: max(orig(ctx, n, i) - 1, 1)),   # own key left out
+    lambda orig: (lambda ctx, n, i: i + 1),                         # chunk taken as positions 0..n-1
+])
+def test_planted_prefill_position_mistakes_are_caught(monkeypatch, bad):
+    monkeypatch.setattr(paged, "visible_keys", bad(paged.visible_keys))
+    with pytest.raises(AssertionError):
+        test_prefill_matches_library_sdpa_with_causal_offset()
+
+
+def test_planted_merge_mistakes_are_caught(monkeypatch):
+    orig_merge, orig_part = paged.merge_partials, paged.partial_attention
+
+    def flipped(parts):  # weights exp(max - lse_i) instead of exp(lse_i - max)
+        l = np.array([p[0] for p in parts])
+        w = np.where(np.isfinite(l), np.exp(np.where(np.isfinite(l), l.max() - l, 0.0)), 0.0)
+        return sum(wi * p[1] for wi, p in zip(w, parts)) / w.sum()
+
+    def unnormalised(parts):  # the weighted sum not divided by the weights' sum
+        l = np.array([p[0] for p in parts])
+        w = np.exp(l - l.max())
+        return sum(wi * p[1] for wi, p in zip(w, parts))
+
+    def max_for_lse(q, K, V, scale):  # lse replaced by the part's max score
+        lse, o = orig_part(q, K, V, scale)
+        return (float(scale) * (K @ q)).max() if K.shape[0] else lse, o
+
+    for name, fn in [("merge_partials", flipped), ("merge_partials", unnormalised),
+                     ("partial_attention", max_for_lse)]:
+        monkeypatch.setattr(paged, "merge_partials", orig_merge)
+        monkeypatch.setattr(paged, "partial_attention", orig_part)
+        monkeypatch.setattr(paged, name, fn)
+        with pytest.raises(AssertionError):
+            test_partial_attention_and_merge_by_brute_force()
+        with pytest.raises(AssertionError):
+            test_shared_prefix_decode_equals_plain_decode("tails")
+
+
+def test_planted_shared_prefix_past_the_last_token_is_caught(monkeypatch):
+    def no_cut(block_tables, context_lens, members, block_size):  # limit ctx // bs
+        members = [int(m) for m in members]
+        if len(members) < 2:
+            return 0
+        limit = min(int(context_lens[m]) // block_size for m in members)
+        p = 0
+        while p < limit and all(int(block_tables[m][p]) == int(block_tables[members[0]][p])
+                                for m in members):
+            p += 1
+        return p
+    monkeypatch.setattr(paged, "shared_prefix_blocks", no_cut)
+    with pytest.raises(AssertionError):
+        test_shared_prefix_blocks_by_hand()

@@ -74,3 +74,19 @@ def test_gpu_block_hashes_match_the_oracle(pa):
         assert [int(x) for x in got[s, :len(ref)]] == ref
         assert not got[s, len(ref):].any()
     assert (got[7, :20] == got[5, :20]).all() and got[7, 20] != got[5, 20]
+
+
+def test_planted_unchained_hash_is_caught(monkeypatch):
+    """A block hash that leaves out its parent (each block hashed alone) fails
+    the chain pin: equal blocks after different prefixes would hash equal."""
+    import oracle.prefix_hash as ph
+
+    def unchained(token_ids, num_tokens, block_size):
+        toks = np.asarray(token_ids, dtype=np.int64)[: int(num_tokens)]
+        return [fnv1a64(b"".join(int(t & 0xFFFFFFFF).to_bytes(4, "little")
+                                 for t in toks[j * block_size:(j + 1) * block_size]))
+                for j in range(int(num_tokens) // block_size)]
+    monkeypatch.setitem(globals(), "block_hashes", unchained)
+    monkeypatch.setattr(ph, "block_hashes", unchained)
+    with pytest.raises(AssertionError):
+        test_chain_properties()
