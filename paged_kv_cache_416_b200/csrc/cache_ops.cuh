@@ -140,25 +140,37 @@ __global__ void __launch_bounds__(256) swap_blocks_kernel(
 // 64-bit FNV-1a (Fowler / Noll / Vo): per byte, xor then multiply by the
 // prime, mod 2^64, from the offset basis.
 constexpr unsigned long long kFnvOffset = 0xcbf29ce484222325ull;
-constexpr unsigned long long kFnvPrime = 0x100000001b3ull;
+constexpr uint32_t kFnvPrimeLow = 0x1b3u;  // the prime is 2^40 + 0x1b3
 
-__device__ __forceinline__ unsigned long long fnv1a_u32(unsigned long long h, uint32_t w) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {  // the word's 4 bytes, little-endian order
-    h ^= (w >> (8 * i)) & 0xffu;
-    h *= kFnvPrime;
-  }
-  return h;
+// One FNV-1a byte step on the hash's 32-bit halves (lo, hi): with
+// l = lo ^ byte, (l + hi 2^32)(2^40 + 0x1b3) mod 2^64 has low word
+// low32(l 0x1b3) and high word high32(l 0x1b3) + hi 0x1b3 + (l << 8), all
+// mod 2^32 (hi 2^72 vanishes mod 2^64).  One wide multiply on the low word's
+// path instead of a full 64 x 64-bit product.
+__device__ __forceinline__ void fnv1a_byte(uint32_t& lo, uint32_t& hi, uint32_t byte) {
+  const uint32_t l = lo ^ byte;
+  const unsigned long long p = static_cast<unsigned long long>(l) * kFnvPrimeLow;
+  lo = static_cast<uint32_t>(p);
+  hi = static_cast<uint32_t>(p >> 32) + hi * kFnvPrimeLow + (l << 8);
 }
 
-// One CTA per sequence.  Phase 1 (all threads): inner_j = FNV-1a over the 4
-// little-endian bytes of each of block j's token ids, for every full block
-// j.  Phase 2 (one thread, in order): hash_j = FNV-1a over hash_{j-1} then
-// inner_j (8 little-endian bytes each), hash_{-1} = 0.  Entries of blocks
-// that are not full are 0.
-__global__ void __launch_bounds__(256) hash_blocks_kernel(
+// FNV-1a over the 4 little-endian bytes of w
+__device__ __forceinline__ void fnv1a_u32(uint32_t& lo, uint32_t& hi, uint32_t w) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) fnv1a_byte(lo, hi, (w >> (8 * i)) & 0xffu);
+}
+
+constexpr int kHashChunk = 256;  // blocks hashed per pass (one per thread)
+
+// One CTA per sequence, over its full blocks in chunks of 256.  Phase 1 (all
+// threads): inner_j = FNV-1a over the 4 little-endian bytes of each of block
+// j's token ids, into shared memory.  Phase 2 (one thread, in order): hash_j
+// = FNV-1a over hash_{j-1} then inner_j (8 little-endian bytes each),
+// hash_{-1} = 0.  Entries of blocks that are not full are 0.
+__global__ void __launch_bounds__(kHashChunk) hash_blocks_kernel(
     const int32_t* __restrict__ tokens, int64_t token_stride, const int32_t* __restrict__ num_tokens,
     int bs, unsigned long long* __restrict__ hashes, int max_blocks) {
+  __shared__ uint32_t s_lo[kHashChunk], s_hi[kHashChunk];
   const int s = blockIdx.x;
   int n = num_tokens[s];
   if (n < 0 || n > token_stride) {
@@ -172,26 +184,34 @@ __global__ void __launch_bounds__(256) hash_blocks_kernel(
   }
   const int32_t* row = tokens + static_cast<int64_t>(s) * token_stride;
   unsigned long long* out = hashes + static_cast<int64_t>(s) * max_blocks;
-  for (int j = threadIdx.x; j < max_blocks; j += blockDim.x) {
-    unsigned long long h = 0;
+  for (int j = full + static_cast<int>(threadIdx.x); j < max_blocks; j += blockDim.x) out[j] = 0;
+  constexpr uint32_t kOffLo = static_cast<uint32_t>(kFnvOffset);
+  constexpr uint32_t kOffHi = static_cast<uint32_t>(kFnvOffset >> 32);
+  uint32_t plo = 0, phi = 0;  // the parent hash (thread 0)
+  for (int j0 = 0; j0 < full; j0 += kHashChunk) {  // the same trip count in every thread
+    const int j = j0 + static_cast<int>(threadIdx.x);
     if (j < full) {
-      h = kFnvOffset;
-      for (int t = 0; t < bs; ++t) h = fnv1a_u32(h, static_cast<uint32_t>(row[j * bs + t]));
+      uint32_t lo = kOffLo, hi = kOffHi;
+      for (int t = 0; t < bs; ++t) fnv1a_u32(lo, hi, static_cast<uint32_t>(row[static_cast<int64_t>(j) * bs + t]));
+      s_lo[threadIdx.x] = lo;
+      s_hi[threadIdx.x] = hi;
     }
-    out[j] = h;
-  }
-  __syncthreads();  // the inner hashes are visible to thread 0
-  if (threadIdx.x == 0) {
-    unsigned long long parent = 0;
-    for (int j = 0; j < full; ++j) {
-      const unsigned long long inner = out[j];
-      unsigned long long h = kFnvOffset;
-      h = fnv1a_u32(h, static_cast<uint32_t>(parent));
-      h = fnv1a_u32(h, static_cast<uint32_t>(parent >> 32));
-      h = fnv1a_u32(h, static_cast<uint32_t>(inner));
-      h = fnv1a_u32(h, static_cast<uint32_t>(inner >> 32));
-      out[j] = parent = h;
+    __syncthreads();  // the chunk's inner hashes are visible to thread 0
+    if (threadIdx.x == 0) {
+      const int m = min(kHashChunk, full - j0);
+      for (int i = 0; i < m; ++i) {
+        const uint32_t ilo = s_lo[i], ihi = s_hi[i];
+        uint32_t lo = kOffLo, hi = kOffHi;
+        fnv1a_u32(lo, hi, plo);
+        fnv1a_u32(lo, hi, phi);
+        fnv1a_u32(lo, hi, ilo);
+        fnv1a_u32(lo, hi, ihi);
+        plo = lo;
+        phi = hi;
+        out[j0 + i] = (static_cast<unsigned long long>(hi) << 32) | lo;
+      }
     }
+    __syncthreads();  // the chunk's slots are free again
   }
 }
 

@@ -423,7 +423,7 @@ pa_status pa_hash_blocks(const int32_t* token_ids, int64_t token_stride,
     return fail(PA_ERR_SHAPE, "pa_hash_blocks: bad sizes");
   if (num_seqs == 0) return ok();
   if (!token_ids || !num_tokens || !block_hashes) return fail(PA_ERR_NULL, "pa_hash_blocks: null pointer");
-  pa::hash_blocks_kernel<<<static_cast<unsigned>(num_seqs), 256, 0,
+  pa::hash_blocks_kernel<<<static_cast<unsigned>(num_seqs), pa::kHashChunk, 0,
                            reinterpret_cast<cudaStream_t>(stream)>>>(
       token_ids, token_stride, num_tokens, block_size,
       reinterpret_cast<unsigned long long*>(block_hashes), max_blocks);

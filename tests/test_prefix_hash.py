@@ -76,6 +76,27 @@ def test_gpu_block_hashes_match_the_oracle(pa):
     assert (got[7, :20] == got[5, :20]).all() and got[7, 20] != got[5, 20]
 
 
+@pytest.mark.gpu
+@pytest.mark.parametrize("bs", [16, 32])
+def test_gpu_block_hashes_across_chunks_of_256_blocks(pa, bs):
+    # the kernel hashes a sequence's blocks 256 at a time: exactly one
+    # chunk, one block past it, several chunks, and a ragged tail
+    rng = np.random.default_rng(6)
+    full = [256, 257, 600, 3]
+    L = max(full) * bs + bs
+    toks = rng.integers(-2**31, 2**31 - 1, size=(len(full), L), dtype=np.int64).astype(np.int32)
+    lens = np.array([f * bs + (s % 2) * (bs - 1) for s, f in enumerate(full)], dtype=np.int32)
+    got = pa.hash_blocks(torch.from_numpy(toks).cuda(), torch.from_numpy(lens).cuda(), bs,
+                         max_blocks=L // bs)
+    pa.sync_status()
+    got = got.cpu().numpy().view(np.uint64)
+    for s in range(len(full)):
+        ref = block_hashes(toks[s].astype(np.int64), int(lens[s]), bs)
+        assert len(ref) == full[s]
+        assert [int(x) for x in got[s, :len(ref)]] == ref
+        assert not got[s, len(ref):].any()
+
+
 def test_planted_unchained_hash_is_caught(monkeypatch):
     """A block hash that leaves out its parent (each block hashed alone) fails
     the chain pin: equal blocks after different prefixes would hash equal."""
