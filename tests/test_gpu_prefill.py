@@ -124,3 +124,33 @@ def test_prefill_bad_table_entry_masks_its_block(pa):
     # rows before block 3 never see it: they equal the oracle on the intact table
     good = ref(W.prefill(seed=12, ctxs=(160,), nqs=(160,), hq=32, hkv=8, bs=16, dtype="bf16"))
     assert_attention_close(got[:48], good[:48], "rows before the bad block")
+
+
+def test_prefill_full_size_sampled(pa):
+    """The benchmark's prefill (8 sequences x 4096 new tokens, 64/8 heads,
+    D 128, bf16, bs 16, the benchmark's seed) in the launch configuration it
+    times.  Sampled rows are checked one by one: the token at position p
+    attends to keys 0..p, which is the oracle's decode of that query over a
+    context of p + 1 tokens through the same block table."""
+    n = 4096
+    pw = W.prefill(seed=3, device="cuda", ctxs=(n,) * 8, nqs=(n,) * 8, hq=64, hkv=8, bs=16,
+                   dtype="bf16")
+    b = pw.base
+    out = pa.prefill(pw.q, b.k_pool, b.v_pool, torch.from_numpy(b.block_tables).cuda(),
+                     torch.from_numpy(b.context_lens).cuda(),
+                     torch.from_numpy(pw.query_start).cuda(), b.scale, pw.max_query_len,
+                     b.max_context_len)
+    pa.sync_status()
+    assert torch.isfinite(out.float()).all()
+    rng = np.random.default_rng(0)
+    picks = [(0, 0), (0, 15), (1, 16), (2, 63), (3, 64), (4, 127), (5, 128), (6, 2047),
+             (7, n - 1), (5, n - 1)] + [(int(s), int(i)) for s, i in
+                                        zip(rng.integers(0, 8, 6), rng.integers(0, n, 6))]
+    kp, vp = raw(b.k_pool), raw(b.v_pool)
+    for s, i in picks:
+        row = int(pw.query_start[s]) + i
+        pos = int(b.context_lens[s]) - n + i
+        ref = oracle.decode(raw(pw.q[row:row + 1]), b.q_dtype, kp, vp, b.cache_dtype,
+                            b.block_tables[s:s + 1], np.array([pos + 1]), b.scale,
+                            b.num_kv_heads)
+        assert_attention_close(as_f64(out[row:row + 1]), ref, f"prefill full size seq {s} token {i}")
