@@ -1,6 +1,6 @@
 """Run the oracle's decode over many sequences in a process pool.
 
-TEST / BASELINE INFRASTRUCTURE ONLY (see the package docstring).  Used by
+TEST AND CPU-TIMING INFRASTRUCTURE ONLY (see the package docstring).  Used by
 the CPU-baseline and reference legs of bench.py to time the oracle on the
 host's cores.  Each task is one sequence with its own compact pools, so a
 worker needs only numpy and this package.  The pool uses the "spawn" start
