@@ -126,6 +126,30 @@ def test_prefill_bad_table_entry_masks_its_block(pa):
     assert_attention_close(got[:48], good[:48], "rows before the bad block")
 
 
+def test_prefill_empty_chunks_and_an_inconsistent_length(pa):
+    # a sequence with no new tokens in the batch; then one whose context is
+    # shorter than its chunk: its rows are zeroed and reported, the others
+    # still equal the oracle
+    pw = W.prefill(seed=13, ctxs=(100, 50, 80, 30), nqs=(20, 0, 80, 10), hq=32, hkv=8, bs=16,
+                   dtype="bf16")
+    want = ref(pw)
+    assert_attention_close(as_f64(run(pa, pw)), want, "prefill with an empty chunk")
+    b = pw.base
+    lens = b.context_lens.copy()
+    lens[3] = 5  # 10 new tokens, 5 cached
+    out = pa.prefill(pw.q.cuda(), b.k_pool.cuda(), b.v_pool.cuda(),
+                     torch.from_numpy(b.block_tables).cuda(), torch.from_numpy(lens).cuda(),
+                     torch.from_numpy(pw.query_start).cuda(), b.scale, pw.max_query_len,
+                     b.max_context_len)
+    with pytest.raises(pa.PagedAttnError) as e:
+        pa.sync_status()
+    assert e.value.status == 8  # PA_ERR_DEVICE_BOUNDS
+    got = as_f64(out)
+    q3 = int(pw.query_start[3])
+    assert not got[q3:].any()
+    assert_attention_close(got[:q3], want[:q3], "the consistent sequences")
+
+
 def test_prefill_full_size_sampled(pa):
     """The benchmark's prefill (8 sequences x 4096 new tokens, 64/8 heads,
     D 128, bf16, bs 16, the benchmark's seed) in the launch configuration it

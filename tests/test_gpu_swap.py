@@ -78,3 +78,30 @@ def test_pageable_host_memory_is_refused(pa):
         pa.swap_blocks(dev, dev.clone(), dev.clone(), dev.clone(),
                        torch.tensor([[0, 9]], dtype=torch.int64, device="cuda"))
         pa.sync_status()
+
+
+def test_swap_benchmark_size_bit_exact(pa):
+    """The benchmark's swap: 2048 scattered blocks of an 8192-block bf16
+    pool (bs 16, 8 kv heads, D 128) out to pinned host memory and back into
+    their original slots, byte for byte against the oracle's indexed copy."""
+    nb, n_dev, shape = 2048, 8192, (16, 8, 128)
+    g = torch.Generator().manual_seed(3)
+    dev_k = torch.randint(-30000, 30000, (n_dev,) + shape, generator=g, dtype=torch.int16).view(torch.bfloat16).cuda()
+    dev_v = torch.randint(-30000, 30000, (n_dev,) + shape, generator=g, dtype=torch.int16).view(torch.bfloat16).cuda()
+    host_k = torch.zeros((nb,) + shape, dtype=torch.bfloat16).pin_memory()
+    host_v = torch.zeros((nb,) + shape, dtype=torch.bfloat16).pin_memory()
+    src = torch.randperm(n_dev, generator=g)[:nb]
+    dst = torch.randperm(nb, generator=g)
+    out_pairs = torch.stack([src, dst], 1).to(torch.int64)
+    dk0, dv0 = raw(dev_k), raw(dev_v)
+    hk, hv = raw(host_k).copy(), raw(host_v).copy()
+    oracle.swap_blocks(dk0, dv0, hk, hv, out_pairs.numpy())
+    pa.swap_blocks(dev_k, dev_v, host_k, host_v, out_pairs.cuda())
+    pa.sync_status()
+    assert np.array_equal(raw(host_k), hk) and np.array_equal(raw(host_v), hv)
+    dev_k[src.cuda()] = 0  # evicted
+    dev_v[src.cuda()] = 0
+    in_pairs = torch.stack([dst, src], 1).to(torch.int64)
+    pa.swap_blocks(host_k, host_v, dev_k, dev_v, in_pairs.cuda())
+    pa.sync_status()
+    assert np.array_equal(raw(dev_k), dk0) and np.array_equal(raw(dev_v), dv0)
