@@ -223,6 +223,11 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
  * 16-byte aligned (they are read through TMA tensor maps).
  * workspace: device memory of at least pa_decode_workspace_size(...) bytes,
  * 256-byte aligned, used only during the call (stream-ordered).
+ * The call enqueues two kernels on `stream`: a one-block planning kernel,
+ * then the attention kernel, launched with programmatic stream
+ * serialization so that its blocks set up while the plan runs and read the
+ * plan only once it has completed.  Work before and after the call on the
+ * stream is ordered as usual; the pair can be captured in a CUDA graph.
  */
 pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype,
                     const void* k_pool, const void* v_pool, pa_dtype cache_dtype,
