@@ -368,3 +368,54 @@ def test_decode_more_than_eight_query_heads_per_kv_head(pa, hq, hkv, cache, spli
     out, _, _ = gpu_step(pa, w, split_tokens=split)
     ref, _, _ = oracle_step(w)
     assert_attention_close(as_f64(out), ref, f"{hq}/{hkv} {cache} split {split}")
+
+
+@pytest.mark.parametrize("name", ["fp8_longtail_bs16", "llama70b_gqa_ragged"])
+def test_decode_step_replays_in_a_cuda_graph(pa, name):
+    """The step (copy-on-write, write, decode: the planning kernel and the
+    attention kernel launched behind it) captured once in a CUDA graph and
+    replayed on fresh pools gives the bytes of the direct calls."""
+    w = small(name)
+    direct, dkp, dvp = gpu_step(pa, w)
+    k0, v0 = w.k_pool.cuda().clone(), w.v_pool.cuda().clone()
+    kp, vp = k0.clone(), v0.clone()
+    q = w.q.cuda().contiguous()
+    nk, nv = w.new_k.cuda().contiguous(), w.new_v.cuda().contiguous()
+    slots = torch.from_numpy(w.slot_mapping).cuda()
+    tables = torch.from_numpy(w.block_tables).cuda()
+    lens = torch.from_numpy(w.context_lens).cuda()
+    pairs = torch.from_numpy(w.cow_pairs).cuda() if len(w.cow_pairs) else None
+    out = torch.empty_like(q)
+    B, hq, d = q.shape
+    _, bs, hkv, _ = kp.shape
+    ws = torch.empty(max(256, pa.decode_workspace_size(B, hq, hkv, d, bs, w.max_context_len, 0)),
+                     dtype=torch.uint8, device="cuda")
+
+    def step():
+        if pairs is not None:
+            pa.copy_blocks(kp, vp, pairs)
+        pa.write_kv(nk, nv, slots, kp, vp, w.k_scale, w.v_scale)
+        pa.decode(q, kp, vp, tables, lens, w.scale, w.max_context_len, k_scale=w.k_scale,
+                  v_scale=w.v_scale, out=out, workspace=ws)
+
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        step()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    pa.sync_status()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        step()
+    for _ in range(2):
+        kp.copy_(k0)
+        vp.copy_(v0)
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        pa.sync_status()
+        assert torch.equal(out, direct)
+        assert torch.equal(kp.view(torch.uint8), dkp.view(torch.uint8))
+        assert torch.equal(vp.view(torch.uint8), dvp.view(torch.uint8))
+    del g
