@@ -11,29 +11,30 @@
 // dense contraction (128 query rows x 64 keys x 128 dims per tile pair), so
 // both products run on tcgen05.mma:
 //
-//   CTA   = 5 warps on one (sequence, kv head, 128 query rows) tile.  Warps
-//           0-3 own the rows: query row r = (token r / G, head r % G) lives
-//           in TMEM lane r and thread r runs its softmax.  Warp 4 is the
-//           producer: TMA loads, the MMA issue (one lane), and the zeroing of
-//           values that must not reach O.  The two sides hand over through
-//           mbarriers only (S done, S read, P ready, O done), never a
-//           CTA-wide barrier inside the key loop.
-//   TMEM  = two S/P buffers [0, 64) and [64, 128) | O [128, 256): S(kt) in
-//           buffer kt & 1 (fp32), then P(kt) over it (P_hi in its first 32
-//           columns, P_lo in the next 32, two 16-bit values per column)
+//   CTA   = 6 warps on one (sequence, kv head, 128 query rows) tile, two
+//           CTAs per SM.  Warps 0-3 own the rows: query row r = (token r / G,
+//           head r % G) lives in TMEM lane r and thread r runs its softmax.
+//           Warp 4 issues the MMAs (one lane) and zeroes values that must not
+//           reach O; warp 5 issues the TMA loads.  They hand over through
+//           mbarriers only (S done, S read, P ready, O done, K / V full and
+//           empty per stage), never a CTA-wide barrier inside the key loop.
+//   TMEM  = two S/P buffers [0, 64) and [64, 128) | O [128, 128 + D): S(kt)
+//           in buffer kt & 1 (fp32), then P(kt) over it (P_hi in its first
+//           32 columns, P_lo in the next 32, two 16-bit values per column)
 //   per 64-key tile kt (K and V by TMA into two stages each, one box per
-//   (block, dim half); K(kt+2) is loaded once S(kt) has been read, V(kt+1)
-//   once O(kt-1) is done):
+//   (block, dim half); K(kt+2) is loaded once S(kt) is done, V(kt+2) once
+//   O(kt) is done; the load warp reads the block ids one tile ahead):
 //     S            = Q K^T      tcgen05.mma, A = Q and B = K from shared memory
-//                               (K-major), M128 N64, 8 x K16; S(kt+1) is
-//                               issued as soon as the rows have read S(kt),
-//                               so it runs under the softmax of tile kt
+//                               (K-major), M128 N64, D/16 x K16; S(kt+1) is
+//                               issued once the rows have read S(kt) and
+//                               O(kt-1), the last reader of its buffer, is
+//                               done, so it runs under the softmax of tile kt
 //     softmax      thread r: tcgen05.ld of its S row, causal and block masks
 //                  (only on tiles that need them), online max / sum in packed
 //                  fp32 pairs; P = P_hi + P_lo (two 16-bit parts, so P keeps
 //                  ~16 significant bits) by tcgen05.st into TMEM
 //     O           += P V        tcgen05.mma, A = P from TMEM, B = V from shared
-//                               memory read MN-major (no transpose), M128 N128,
+//                               memory read MN-major (no transpose), M128 N=D,
 //                               2 x 4 x K16, accumulated in TMEM across tiles
 //   O is rescaled (tcgen05.ld, multiply, tcgen05.st) only when a row's
 //   running max grows by more than 8 in log2 units; otherwise the weights
