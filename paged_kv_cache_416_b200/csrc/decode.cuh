@@ -10,7 +10,7 @@
 // query attention bullet).
 //
 // Work decomposition
-//   item  = (sequence, context range of split_tokens tokens, kv head)
+//   item  = (sequence, context range, kv head, group of <= 8 of its q heads)
 //   CTA   = 4 warps; a persistent grid pulls items from an atomic counter
 //   warp  = takes every 4th block of the item's range; each warp owns a ring
 //           of kStages shared-memory stages, one stage = the K tile and the V
