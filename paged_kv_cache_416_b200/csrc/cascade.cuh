@@ -40,8 +40,9 @@ namespace pa {
 constexpr int kCascadeRows = 16;        // query rows per chunk (members x heads)
 constexpr int kCascadeMaxRanges = 512;  // ranges per chunk (their weights sit in smem)
 // work items (x Hkv) the range length aims at: ~1.5 waves of 444 persistent
-// CTAs (on the shared-prefix workload 666 ran 80.1 us, 444: 84.3, 888: 81.7,
-// 1332: 87.4 -- shorter ranges pay the per-range start and merge more often)
+// CTAs (on the shared-prefix workload 666 ran 74.9 us, 555: 75.0, 888: 74.8,
+// 444: 78.0 -- too few items leave CTAs idle at the end; with one range form
+// 1332 had run 87.4 against 80.1, shorter ranges paying start and merge)
 constexpr int kCascadeTargetItems = 666;
 
 struct CascadeArgs {
