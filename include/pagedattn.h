@@ -186,7 +186,12 @@ int32_t pa_decode_split_tokens(int32_t num_seqs, int32_t num_kv_heads,
  * pa_decode_workspace_size -- bytes of device workspace pa_decode needs for
  * these sizes (work counter, per-sequence item offsets, and the split
  * partials: one fp32 log-sum-exp and one fp32 [D] vector per (item, q head)).
- * Returns 0 on invalid arguments.
+ * Returns 0 on invalid arguments.  With split_tokens == 0 the automatic
+ * split grows with num_seqs, so a smaller batch can need MORE workspace
+ * than a larger one: a caller that keeps one workspace for many batch
+ * sizes takes the largest size over them, or passes a fixed split_tokens
+ * (then the size grows with num_seqs).  pa_decode refuses a smaller
+ * workspace with PA_ERR_WORKSPACE before any launch.
  */
 size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
                                 int32_t num_kv_heads, int32_t head_dim,

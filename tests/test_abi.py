@@ -1,6 +1,7 @@
 """The C-ABI library loads and exports every entry point its header declares;
 host-side validation rejects bad arguments before any CUDA call (CPU only)."""
 
+import numpy as np
 import ctypes
 import os
 import re
@@ -164,3 +165,31 @@ def _prefill(pa, **kw):
 ])
 def test_prefill_rejects_bad_arguments_on_the_host(pa, kw, status):
     assert _prefill(pa, **kw) == status
+
+
+def test_split_rule_properties(pa):
+    """The split length stated in the header, over random sizes: a multiple
+    of the block size, at most 1024 ranges per sequence, a requested length
+    only ever raised (to a block multiple, then to the range cap); and the
+    workspace grows with the number of sequences when the split is fixed (the
+    automatic split grows with the batch, so there a smaller batch can need
+    more, as the header says)."""
+    rng = np.random.default_rng(7)
+    for _ in range(3000):
+        B = int(rng.integers(1, 4097))
+        hkv = int(rng.choice([1, 2, 4, 8, 16]))
+        bs = int(rng.choice([16, 32]))
+        ctx = int(rng.integers(1, 262145))
+        user = int(rng.choice([0, int(rng.integers(1, 70000))]))
+        S = pa.pa_decode_split_tokens(B, hkv, bs, ctx, user)
+        assert S >= bs and S % bs == 0, (B, hkv, bs, ctx, user, S)
+        assert -(-ctx // S) <= 1024, (B, hkv, bs, ctx, user, S)
+        if user:
+            assert S >= user and (S - bs < user or -(-ctx // (S - bs)) > 1024), (ctx, user, S)
+        hq = hkv * int(rng.choice([1, 4, 8]))
+        d = int(rng.choice([64, 128]))
+        w1 = pa.pa_decode_workspace_size(B, hq, hkv, d, bs, ctx, user)
+        w2 = pa.pa_decode_workspace_size(B + 1, hq, hkv, d, bs, ctx, user)
+        assert w1 > 0 and w2 > 0
+        if user:
+            assert w1 <= w2
