@@ -213,7 +213,10 @@ _ws_cache = {}
 
 
 def workspace_for(device, nbytes: int) -> torch.Tensor:
-    """A cached device byte buffer of at least nbytes (torch-allocated)."""
+    """A cached device byte buffer of at least nbytes (torch-allocated), one
+    per device, grown when a call needs more.  Calls that use it share it, so
+    they must not overlap on the GPU: calls on several streams at once pass
+    their own `workspace`."""
     key = torch.device(device)
     buf = _ws_cache.get(key)
     if buf is None or buf.numel() < nbytes:
