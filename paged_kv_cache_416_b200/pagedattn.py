@@ -9,8 +9,10 @@ Two layers:
 * ``pa_*``: the C entry points themselves, with ctypes signatures (raw
   pointers, sizes, dtype codes, stream handles);
 * ``write_kv``, ``copy_blocks``, ``decode``, ``decode_workspace_size``,
-  ``sync_status``: the same calls taking torch tensors, which read pointers,
-  sizes and dtypes off the tensors and pass the current torch stream.
+  ``decode_shared_prefix``, ``shared_prefix_workspace_size``, ``prefill``,
+  ``swap_blocks``, ``hash_blocks``, ``sync_status``: the same calls taking
+  torch tensors, which read pointers, sizes and dtypes off the tensors and
+  pass the current torch stream.
 """
 
 from __future__ import annotations
