@@ -38,9 +38,27 @@ METRIC = "paged decode attn: KV-read GB/s (% of HBM peak), seq-tokens/s"
 NOMINAL_HBM_GBS = 8000.0      # the "~8 TB/s" B200 figure the target is stated against
 FALLBACK_HBM_GBS = 6650.0     # used only when MEASURED_PEAKS.json is absent
 DEFAULT_WORKLOAD = "llama70b_gqa"
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "decode_kernel_llama70b_gqa.md")
-DECODE_SOURCES = [os.path.join(ROOT, "paged_kv_cache_416_b200", "csrc", f)
-                  for f in ("decode.cuh", "common.cuh")]
+# DRAM bytes per launch of each kernel, taken from ncu captures by
+# `bench.py --ingest-ncu`; an entry counts only while the kernel's sources
+# hash as they did when it was captured
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_traffic.json")
+CSRC = os.path.join(ROOT, "paged_kv_cache_416_b200", "csrc")
+KERNEL_SOURCES = {
+    "decode_kernel": ("decode.cuh", "common.cuh"),
+    "cascade_kernel": ("cascade.cuh", "decode.cuh", "common.cuh"),
+}
+# the five benchmark configurations as workloads (config 4 is two steps of one
+# batch, config 5 runs at block sizes 16 and 32), in the order they are named
+CONFIG_WORKLOADS = ["tiny", "llama13b_mha", "llama70b_gqa", "shared_prefix_fork",
+                    "shared_prefix_tails", "fp8_longtail_bs16", "fp8_longtail_bs32"]
+# tokens a contiguous (maximum-length) reservation would hold per sequence:
+# each generator's length bound (the tiny batch takes the 2048 of the pages'
+# worked example; shared prefix: 1024 + 15 prompt tokens, 512 own tokens, the
+# fork step's token and the step's token)
+RESERVATION_TOKENS = {"tiny": 2048, "llama13b_mha": 2048, "llama70b_gqa": 4096,
+                      "shared_prefix_fork": 1024 + 15 + 512 + 2,
+                      "shared_prefix_tails": 1024 + 15 + 512 + 2,
+                      "fp8_longtail_bs16": 32768, "fp8_longtail_bs32": 32768}
 
 
 def parse_args(argv=None):
@@ -54,6 +72,20 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--config-cpu-seconds", type=float, default=3.0,
+                    help="target CPU time of each configuration's oracle sample")
+    ap.add_argument("--config-iters", type=int, default=30,
+                    help="timed iterations per configuration in the `configs` object")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-configuration measurements (profiling runs)")
+    ap.add_argument("--ingest-ncu", default=None, metavar="CSV",
+                    help="read an ncu --csv capture of one kernel (dram__bytes_read.sum, "
+                         "dram__bytes_write.sum) of --workload [--num-seqs] and record its "
+                         "per-launch DRAM bytes, scaled to the full workload, in "
+                         "profiles/decode_traffic.json; no GPU work")
+    ap.add_argument("--ingest-kernel", default="decode_kernel", choices=sorted(KERNEL_SOURCES))
+    ap.add_argument("--ingest-command", default="",
+                    help="the command line that produced the capture (recorded)")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling only)")
@@ -200,65 +232,141 @@ def measured_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
-def decode_source_hash() -> str:
+def source_hash(kernel: str) -> str:
     h = hashlib.sha256()
-    for f in DECODE_SOURCES:
-        with open(f, "rb") as fh:
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(CSRC, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def profiled_traffic():
-    """DRAM bytes per decode launch from the committed ncu summary, if it was
-    taken on the current kernel source (else None)."""
-    if not os.path.exists(PROFILE_SUMMARY):
-        return None
-    src, traffic = None, None
-    with open(PROFILE_SUMMARY) as f:
-        for line in f:
-            if line.startswith("decode_source_sha256:"):
-                src = line.split(":", 1)[1].strip()
-            if line.startswith("dram_bytes_per_launch:"):
-                traffic = int(float(line.split(":", 1)[1].strip()))
-    return traffic if (src == decode_source_hash() and traffic) else None
+def _load_traffic():
+    if not os.path.exists(TRAFFIC_FILE):
+        return {}
+    with open(TRAFFIC_FILE) as f:
+        return json.load(f)
+
+
+def profiled_traffic(workload: str, kernel: str = "decode_kernel"):
+    """DRAM bytes per launch of `kernel` on the full `workload`, from the
+    recorded ncu capture, while the kernel's sources still hash as captured
+    (else None).  Returns (bytes or None, the record or None)."""
+    rec = _load_traffic().get(f"{kernel}:{workload}")
+    if rec is None:
+        return None, None
+    if rec.get("source_sha16") != source_hash(kernel):
+        return None, rec
+    return int(rec["dram_bytes_per_launch_full"]), rec
+
+
+_NCU_UNITS = {"byte": 1, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "tbyte": 1e12,
+              "nsecond": 1e-9, "usecond": 1e-6, "msecond": 1e-3, "second": 1.0}
+
+
+def parse_ncu_csv(path: str, kernel: str):
+    """Per-launch metric values of the launches of `kernel` in an ncu --csv
+    metrics log: {launch id: {metric: value in base units}}."""
+    import csv
+    with open(path, newline="") as f:
+        lines = [ln for ln in f if ln.startswith('"')]
+    rows = list(csv.DictReader(lines))
+    out = {}
+    for r in rows:
+        if kernel not in r.get("Kernel Name", ""):
+            continue
+        unit = r.get("Metric Unit", "").strip().lower()
+        val = float(r["Metric Value"].replace(",", ""))
+        out.setdefault(r["ID"], {})[r["Metric Name"]] = val * _NCU_UNITS.get(unit, 1.0)
+    return out
+
+
+def ingest_ncu(args):
+    """Record the DRAM traffic of one captured kernel launch per workload."""
+    from paged_kv_cache_416_b200 import workloads as W
+    launches = parse_ncu_csv(args.ingest_ncu, args.ingest_kernel)
+    if not launches:
+        raise SystemExit(f"no {args.ingest_kernel} launch in {args.ingest_ncu}")
+    rd = [m["dram__bytes_read.sum"] for m in launches.values()]
+    wr = [m["dram__bytes_write.sum"] for m in launches.values()]
+    seed = args.seed if args.workload == DEFAULT_WORKLOAD else None
+    kw = _sample_kw(args.workload, args.num_seqs) if args.num_seqs else {}
+    cap_bytes = W.kv_bytes_of(args.workload, seed, **kw)
+    full_bytes = W.kv_bytes_of(args.workload, seed)
+    cap_seqs = len(W.context_lens(args.workload, seed, **kw))
+    full_seqs = len(W.context_lens(args.workload, seed))
+    scale = full_bytes / cap_bytes
+    per_launch = (sum(rd) + sum(wr)) / len(rd)
+    rec = {
+        "kernel": args.ingest_kernel, "workload": args.workload,
+        "source_sha16": source_hash(args.ingest_kernel),
+        "sources": list(KERNEL_SOURCES[args.ingest_kernel]),
+        "captured_num_seqs": cap_seqs, "full_num_seqs": full_seqs,
+        "launches": len(rd),
+        "dram_bytes_read_per_launch": round(sum(rd) / len(rd)),
+        "dram_bytes_write_per_launch": round(sum(wr) / len(wr)),
+        "algorithmic_kv_bytes_captured": cap_bytes,
+        "scale_to_full": scale,
+        "dram_bytes_per_launch_full": round(per_launch * scale),
+        "ratio_to_algorithmic": round(per_launch / cap_bytes, 4),
+        "command": args.ingest_command,
+    }
+    if "gpu__time_duration.sum" in next(iter(launches.values())):
+        rec["ncu_us_per_launch"] = round(sum(m["gpu__time_duration.sum"] for m in launches.values())
+                                         / len(launches) * 1e6, 2)
+    if "lts__t_sector_hit_rate.pct" in next(iter(launches.values())):
+        rec["l2_sector_hit_rate_pct"] = round(sum(m["lts__t_sector_hit_rate.pct"]
+                                                  for m in launches.values()) / len(launches), 2)
+    data = _load_traffic()
+    data[f"{args.ingest_kernel}:{args.workload}"] = rec
+    with open(TRAFFIC_FILE, "w") as f:
+        json.dump(data, f, indent=1, sort_keys=True)
+        f.write("\n")
+    print(json.dumps(rec))
 
 
 # ------------------------------------------------------------ CPU baseline
-def oracle_rate(name: str, seed: int, target_seconds: float, workers: int):
-    """Time the oracle (as it stands) on a bounded sample of sequences of the
-    workload on the host's cores.  Returns (GB/s of KV read, seq-tokens/s,
-    description, cores, seconds)."""
+def _oracle_tasks(w):
+    """One oracle task per sequence: its q row and compact K/V pools."""
     import numpy as np
-    from oracle.parallel import run_decode_tasks
-    from paged_kv_cache_416_b200 import workloads as W
     from paged_kv_cache_416_b200.workloads import raw
+    ts = []
+    bs = w.block_size
+    for s in range(w.num_seqs):
+        nb = -(-int(w.context_lens[s]) // bs)
+        ids = w.block_tables[s, :nb].astype(np.int64)
+        ts.append((raw(w.q[s:s + 1]), w.q_dtype, raw(w.k_pool)[ids], raw(w.v_pool)[ids],
+                   w.cache_dtype, np.arange(nb)[None], w.context_lens[s:s + 1], w.scale,
+                   w.num_kv_heads, w.k_scale, w.v_scale))
+    return ts
 
-    def tasks_for(n):
+
+def oracle_rate(name: str, seed, target_seconds: float, pool):
+    """Time the oracle (as it stands) on a bounded sample of sequences of the
+    workload on the host's cores (`pool`: an oracle.parallel.OraclePool).
+    Returns a cpu_baseline dict (GB/s of KV read, seq-tokens/s, the sample,
+    cores, CPU model, seconds)."""
+    from oracle.parallel import cpu_model
+    from paged_kv_cache_416_b200 import workloads as W
+
+    def sample(n):
         w = W.make(name, seed=seed, device="cpu", **_sample_kw(name, n))
-        ts = []
-        bs = w.block_size
-        for s in range(w.num_seqs):
-            nb = -(-int(w.context_lens[s]) // bs)
-            ids = w.block_tables[s, :nb].astype(np.int64)
-            ts.append((raw(w.q[s:s + 1]), w.q_dtype, raw(w.k_pool)[ids], raw(w.v_pool)[ids],
-                       w.cache_dtype, np.arange(nb)[None], w.context_lens[s:s + 1], w.scale,
-                       w.num_kv_heads, w.k_scale, w.v_scale))
-        return w, ts
+        return w, _oracle_tasks(w)
 
     # calibrate on one sequence per worker, then size the sample
-    w, ts = tasks_for(workers)
-    _, wall = run_decode_tasks(ts, workers)
-    per_round = max(wall, 1e-3)
-    rounds = max(1, int(target_seconds / per_round))
+    workers = pool.workers
+    w, ts = sample(workers)
+    _, wall = pool.run(ts)
+    rounds = max(1, int(target_seconds / max(wall, 1e-3)))
     n = min(workers * rounds, _full_seqs(name))
-    if n > workers:
-        w, ts = tasks_for(n)
-        _, wall = run_decode_tasks(ts, workers)
-    gbs = w.kv_bytes / wall / 1e9
-    tps = w.seq_tokens / wall
+    if n > w.num_seqs:
+        w, ts = sample(n)
+        _, wall = pool.run(ts)
     desc = (f"oracle (numpy fp64) decode of {w.num_seqs} of the workload's {_full_seqs(name)} "
-            f"sequences (same shapes and lengths), {workers} spawned workers, 1 BLAS thread each")
-    return gbs, tps, desc, workers, wall
+            f"sequences (same shapes; lengths from the same generator), {workers} spawned "
+            f"workers, 1 BLAS thread each")
+    return {"value": round(w.kv_bytes / wall / 1e9, 4), "unit": "GB/s", "cores": workers,
+            "kind": "oracle", "sample": desc, "cpu_model": cpu_model(),
+            "seq_tokens_per_s": round(w.seq_tokens / wall, 1), "seconds": round(wall, 2)}
 
 
 def _full_seqs(name):
@@ -287,7 +395,7 @@ def run_ours(args, rank, local, world):
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
-    kw = {"num_seqs": args.num_seqs} if args.num_seqs else {}
+    kw = _sample_kw(args.workload, args.num_seqs) if args.num_seqs else {}
     w = W.make(args.workload, seed=args.seed + rank, device=device, **kw)
     stream = torch.cuda.current_stream()
     kp, vp = w.k_pool, w.v_pool
@@ -407,16 +515,22 @@ def run_ours(args, rank, local, world):
     peak, peak_kind = measured_peaks()
     dec_mean_s = float(np.mean(dec_ms)) / 1e3
     achieved = w.kv_bytes / dec_mean_s / 1e9
+    traffic, traffic_rec = profiled_traffic(w.name)
+
+    configs = None
+    if not args.no_configs and world == 1 and args.num_seqs is None:
+        configs = measure_configs(args, pa, W, device, w, dec_ms, peak, peak_kind)
 
     if rank != 0:
         return None
     cpu = None
     if not args.no_cpu_baseline and world == 1:
-        from oracle.parallel import host_cores
-        gbs, tps, desc, cores, wall = oracle_rate(args.workload, args.seed, args.cpu_seconds,
-                                                  host_cores())
-        cpu = {"value": round(gbs, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
-               "sample": desc, "seq_tokens_per_s": round(tps, 1), "seconds": round(wall, 2)}
+        from oracle.parallel import OraclePool, host_cores
+        with OraclePool(host_cores()) as pool:
+            cpu = oracle_rate(args.workload, args.seed, args.cpu_seconds, pool)
+            for name, c in (configs or {}).items():
+                seed = args.seed if name == args.workload else None
+                c["cpu_baseline"] = oracle_rate(name, seed, args.config_cpu_seconds, pool)
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -443,7 +557,8 @@ def run_ours(args, rank, local, world):
         "pct_of_8tbs": round(100 * value / NOMINAL_HBM_GBS, 2),
         "roofline": {
             "bound": "hbm", "achieved": round(achieved, 2), "peak": peak, "unit": "GB/s",
-            "frac": round(achieved / peak, 4), "traffic": profiled_traffic(),
+            "frac": round(achieved / peak, 4), "traffic": traffic,
+            "traffic_source": _traffic_note(traffic_rec, traffic),
             "kernel": "pa_decode (plan_kernel + decode_kernel)",
             "algorithmic_bytes_per_launch": w.kv_bytes, "peak_kind": peak_kind,
             "mean_launch_us": round(dec_mean_s * 1e6, 2),
@@ -459,7 +574,184 @@ def run_ours(args, rank, local, world):
         "gpu_launches": launches_per_step * K,
         "clocks": clocks.summary(),
     }
+    if configs is not None:
+        line["configs"] = configs
     return line
+
+
+def _traffic_note(rec, traffic):
+    if rec is None:
+        return "no ncu capture recorded for this workload"
+    if traffic is None:
+        return "the kernel changed since its capture: traffic not counted"
+    return (f"ncu capture of {rec['captured_num_seqs']} of {rec['full_num_seqs']} sequences "
+            f"({rec['launches']} launch(es)) scaled x{rec['scale_to_full']:.4g} by the K/V bytes; "
+            f"profiles/decode_traffic.json")
+
+
+def _stats_us(xs):
+    import numpy as np
+    a = np.asarray(xs, dtype=np.float64)
+    return {"median": round(float(np.median(a)), 2), "min": round(float(a.min()), 2),
+            "mean": round(float(a.mean()), 2)}
+
+
+def config_memory(w, name):
+    """Closed-form memory figures of one configuration's batch: slots left
+    unused by paging (the unfilled tail of each last block) against a
+    contiguous reservation of the generator's length bound per sequence, and
+    for the shared-prefix batch the physical blocks in use against the blocks
+    the same sequences would hold without sharing."""
+    import numpy as np
+    bs = w.block_size
+    lens = w.context_lens.astype(np.int64)
+    nb = -(-lens // bs)
+    alloc_slots = int(nb.sum()) * bs
+    used = int(lens.sum())
+    R = RESERVATION_TOKENS[name]
+    out = {
+        "paged_unused_slots": alloc_slots - used,
+        "paged_waste_pct": round(100.0 * (alloc_slots - used) / alloc_slots, 3),
+        "reservation_tokens_per_seq": R,
+        "reserved_unused_slots": len(lens) * R - used,
+        "reserved_waste_pct": round(100.0 * (len(lens) * R - used) / (len(lens) * R), 2),
+    }
+    if name.startswith("shared_prefix"):
+        phys = set()
+        for s in range(w.num_seqs):
+            phys.update(int(b) for b in w.block_tables[s, :int(nb[s])])
+        out.update({"blocks_unshared": int(nb.sum()), "blocks_shared": len(phys),
+                    "memory_saved_pct": round(100.0 * (1 - len(phys) / int(nb.sum())), 2)})
+    return out
+
+
+def measure_configs(args, pa, W, device, head_w, head_dec_ms, peak, peak_kind):
+    """Every benchmark configuration, each on its own seeded batch: pa_decode
+    (plan + attention kernel) and the whole step (copy-on-write copies, cache
+    write, decode) timed per iteration by CUDA events on the launching stream,
+    median / min / mean over the iterations.  A configuration whose distinct
+    K/V bytes are under 4x the L2 size gets L2 flushed (a 4x-L2 buffer
+    written) before every timed iteration, outside the events."""
+    import numpy as np
+    import torch
+    l2 = int(torch.cuda.get_device_properties(device).L2_cache_size)
+    flush_buf = torch.empty(4 * l2, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+    iters = max(3, args.config_iters)
+    results = {}
+    for name in CONFIG_WORKLOADS:
+        own = name != head_w.name
+        w = W.make(name, device=device) if own else head_w
+        kp, vp = w.k_pool, w.v_pool
+        q = w.q.contiguous()
+        nk, nv = w.new_k.contiguous(), w.new_v.contiguous()
+        slots = torch.from_numpy(w.slot_mapping).to(device)
+        tables = torch.from_numpy(w.block_tables).to(device)
+        lens = torch.from_numpy(w.context_lens).to(device)
+        pairs = torch.from_numpy(w.cow_pairs).to(device) if len(w.cow_pairs) else None
+        out = torch.empty_like(q)
+        ws = torch.empty(max(256, pa.decode_workspace_size(
+            w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
+            w.max_context_len)), dtype=torch.uint8, device=device)
+        unique = unique_kv_bytes(w)
+        flush = unique < 4 * l2
+
+        def step(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            if pairs is not None:
+                pa.copy_blocks(kp, vp, pairs)
+            pa.write_kv(nk, nv, slots, kp, vp, w.k_scale, w.v_scale)
+            if ev is not None:
+                ev[1].record(stream)
+            pa.decode(q, kp, vp, tables, lens, w.scale, w.max_context_len, k_scale=w.k_scale,
+                      v_scale=w.v_scale, out=out, workspace=ws)
+            if ev is not None:
+                ev[2].record(stream)
+
+        for _ in range(max(3, args.warmup)):
+            step()
+        torch.cuda.synchronize()
+        pa.sync_status()
+        evs = [tuple(torch.cuda.Event(enable_timing=True) for _ in range(3)) for _ in range(iters)]
+        clocks = ClockSampler(device.index)
+        clocks.start()
+        for i in range(iters):
+            if flush:
+                flush_buf.zero_()
+            step(evs[i])
+        torch.cuda.synchronize()
+        clocks.stop()
+        pa.sync_status()
+        dec = [b.elapsed_time(c) * 1e3 for a, b, c in evs]
+        stp = [a.elapsed_time(c) * 1e3 for a, b, c in evs]
+        dstat, sstat = _stats_us(dec), _stats_us(stp)
+        med_s = dstat["median"] / 1e6
+        gbs = w.kv_bytes / med_s / 1e9
+        traffic, rec = profiled_traffic(name)
+        r = {
+            "num_seqs": w.num_seqs, "heads": f"{w.num_q_heads}/{w.num_kv_heads}",
+            "head_dim": w.head_dim, "block_size": w.block_size, "cache_dtype": w.cache_dtype,
+            "q_dtype": w.q_dtype, "context_lens": _lens_desc(w), "cow_pairs": int(len(w.cow_pairs)),
+            "kv_bytes": w.kv_bytes, "unique_kv_bytes": unique,
+            "pa_decode_us": dstat, "step_us": sstat, "iterations": iters,
+            "gbs": round(gbs, 1), "pct_of_8tbs": round(100 * gbs / NOMINAL_HBM_GBS, 2),
+            "seq_tokens_per_s": round(w.seq_tokens / med_s, 1),
+            "seq_tokens_per_s_step": round(w.seq_tokens / (sstat["median"] / 1e6), 1),
+            "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peak, "unit": "GB/s",
+                         "frac": round(gbs / peak, 4), "peak_kind": peak_kind,
+                         "bytes": "algorithmic (logical) K/V bytes, median pa_decode time",
+                         "traffic": traffic, "traffic_source": _traffic_note(rec, traffic)},
+            "l2": (f"flushed before every timed iteration ({4 * l2 / 2**20:.0f} MiB written): "
+                   f"{unique / 2**20:.1f} MiB of distinct K/V < 4x L2" if flush else
+                   f"no flush: {unique / 2**30:.2f} GiB of distinct K/V >= 4x L2"),
+            "memory": config_memory(w, name),
+            "clocks": clocks.summary(),
+        }
+        if unique != w.kv_bytes:
+            ug = unique / med_s / 1e9
+            r["gbs_unique"] = round(ug, 1)
+            r["roofline_unique"] = {"achieved": round(ug, 1), "frac": round(ug / peak, 4)}
+        if "group_start" in w.meta:
+            gs = torch.from_numpy(w.meta["group_start"]).to(device)
+            gq = torch.from_numpy(w.meta["group_seqs"]).to(device)
+            sws = torch.empty(max(256, pa.shared_prefix_workspace_size(
+                w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, w.block_size,
+                w.max_context_len)), dtype=torch.uint8, device=device)
+            out2 = torch.empty_like(q)
+
+            def shared():
+                pa.decode_shared_prefix(q, kp, vp, tables, lens, gs, gq, w.scale,
+                                        w.max_context_len, out=out2, workspace=sws)
+
+            for _ in range(3):
+                shared()
+            sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                   for _ in range(iters)]
+            for i in range(iters):
+                if flush:
+                    flush_buf.zero_()
+                sev[i][0].record(stream)
+                shared()
+                sev[i][1].record(stream)
+            torch.cuda.synchronize()
+            pa.sync_status()
+            sp = _stats_us([a.elapsed_time(b) * 1e3 for a, b in sev])
+            sp_s = sp["median"] / 1e6
+            r["pa_decode_shared_prefix"] = {
+                "us": sp, "gbs_logical": round(w.kv_bytes / sp_s / 1e9, 1),
+                "gbs_unique": round(unique / sp_s / 1e9, 1),
+                "frac_unique": round(unique / sp_s / 1e9 / peak, 4),
+                "speedup_vs_pa_decode": round(dstat["median"] / sp["median"], 3)}
+            del out2, sws
+        results[name] = r
+        del kp, vp, q, out, ws
+        if own:
+            del w
+        torch.cuda.empty_cache()
+    del flush_buf
+    torch.cuda.empty_cache()
+    return results
 
 
 def _lens_desc(w):
@@ -582,10 +874,12 @@ def run_swap(args):
 
 def run_hash(args):
     """pa_hash_blocks over 256 sequences x 4096 token ids (bs 16, 65,536
-    full blocks).  Roofline: plain ALU -- about 20 integer instructions per
-    token (FNV-1a: xor + 64-bit multiply per byte of the 4-byte id, plus the
-    per-block chain step) against 148 SMs x 128 lanes x the SM clock; the
-    chain itself is serial along a sequence, which is what bounds the call."""
+    full blocks).  The bound is latency, not a unit's throughput: a
+    sequence's block hashes form a chain, each block's FNV-1a over its
+    parent's hash and its own inner hash being 16 dependent byte steps, so
+    one call is at least 256 x 16 = 4096 dependent steps long.  The line
+    reports the time per dependent step (the call's time over the chain
+    length) in ns and in SM clock cycles at the sampled clock."""
     import torch
     from paged_kv_cache_416_b200 import build as _build
     _build.build()
@@ -597,20 +891,30 @@ def run_hash(args):
     lens = torch.full((B,), L, dtype=torch.int32, device="cuda")
     out = torch.empty((B, L // bs), dtype=torch.int64, device="cuda")
     iters = max(3, min(args.steps, 50))
+    clocks = ClockSampler(0)
+    clocks.start()
     t = _events_time(lambda: pa.hash_blocks(toks, lens, bs, out=out), iters)
+    clocks.stop()
     pa.sync_status()
     tps = B * L / t
-    clock = ClockSampler(0).max_mhz or 1965.0
-    peak = 148 * 128 * clock * 1e6 / 20
+    chain = (L // bs) * 16               # dependent FNV byte steps of one sequence's chain
+    ck = clocks.summary()
+    mhz = ck.get("sm_mhz") or clocks.max_mhz or 1965.0
+    ns_step = t * 1e9 / chain
     return {
         "metric": "prefix-cache block hashing, token ids hashed per second", "op": "hash",
         "value": round(tps, 1), "unit": "tokens/s", "n_gpus": 1, "steps": iters,
         "higher_is_better": True, "dtype": "int32", "data": "synthetic",
         "config": {"workload": "256 sequences x 4096 token ids, block_size 16", "blocks": B * L // bs},
         "us_per_call": round(t * 1e6, 2),
-        "roofline": {"bound": "alu", "achieved": round(tps, 1), "peak": round(peak, 1),
-                     "unit": "tokens/s", "frac": round(tps / peak, 4),
-                     "peak_kind": "derived: 148 SMs x 128 int lanes x max SM clock / 20 instructions per token"},
+        "roofline": {"bound": "latency", "achieved": round(ns_step, 3),
+                     "unit": "ns per dependent step of the per-sequence hash chain",
+                     "peak": None, "frac": None, "chain_steps": chain,
+                     "cycles_per_step": round(ns_step * mhz / 1e3, 2), "sm_mhz": mhz,
+                     "note": "each sequence's 256 block hashes form a serial chain of 16 "
+                             "dependent FNV-1a byte steps per block; the call takes this many "
+                             "cycles per step, the inner hashes of the blocks included"},
+        "clocks": ck,
         "gpu_launches": iters,
     }
 
@@ -726,6 +1030,9 @@ def run_shared_prefix(args):
 
 def main(argv=None):
     args = parse_args(argv)
+    if args.ingest_ncu:
+        ingest_ncu(args)
+        return 0
     if args.warmup < 3:
         args.warmup = 3
     rank, local, world = dist_env()

@@ -43,8 +43,12 @@
  * Hq / Hkv <= 64 for pa_decode (a kv head's query heads are taken 8 at a
  * time: more than 8 read its blocks once per group of 8), <= 8 for the
  * shared-prefix decode; cache dtype f16 (q f16), bf16 (q bf16) or e4m3 (q f16 or
- * bf16).  With an e4m3 cache the query is converted to fp16 for the tensor-
- * core products, so |q| must stay inside the fp16 range (< 65504).
+ * bf16).  With an e4m3 cache the tensor-core products run in fp16: each
+ * head's query is first scaled by a power of two that brings its largest
+ * component into [2^14, 2^15), and the factor is taken back out of that
+ * head's scores, so any finite f16 or bf16 query is accepted (a component
+ * below 2^-28 of its head's largest falls into fp16's subnormal range, where
+ * it is kept to an absolute precision of 2^-39 of that largest component).
  */
 #ifndef PAGEDATTN_H_
 #define PAGEDATTN_H_
@@ -377,7 +381,10 @@ pa_status pa_validate_block_tables(const int32_t* block_tables, int32_t max_bloc
  * launch; a larger split_tokens (fewer context ranges) lowers the need.
  * The first call on a device looks up the array's device address with
  * cudaGetSymbolAddress (once per device, with that device current); make
- * that first call before any stream capture begins.  The call allocates
+ * that first call before any stream capture begins.  The address is kept
+ * per CUDA context: after cudaDeviceReset, or under another context of the
+ * same device, the next call looks it up again (so make that call, too,
+ * before a capture).  The call allocates
  * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  * Every call shares the one array and finds the previous call's contents in
  * it; the work counter that must start at zero is cleared by the call's own

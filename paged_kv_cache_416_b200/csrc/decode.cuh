@@ -370,22 +370,56 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
       ++n_issued;
     };
 
-    // ---- query fragments (B operand of S^T = K Q^T): rows = dims, cols = heads
+    if (!failed) {
+      const int pro = min(kStages, nb_w);
+      for (int i = 0; i < pro; ++i) issue(i);
+    }
+
+    // ---- query fragments (B operand of S^T = K Q^T): rows = dims, cols = heads.
+    // With an e4m3 cache the products run in fp16, so each head's query is
+    // first scaled by a power of two 2^-e that brings its largest |q| into
+    // [2^14, 2^15): any f16 or bf16 query fits, and 2^e goes back into that
+    // head's softmax scale (exact: a power of two scales every product and
+    // partial sum of the fp32 accumulation exactly).
     uint32_t qf[C::kDimTiles][2];
+    float sl2c[2] = {a.sl2, a.sl2};  // softmax scale of heads 2tig, 2tig+1 (log2 units)
     {
       const bool hv = g < ncols;
       const uint16_t* qrow = reinterpret_cast<const uint16_t*>(a.q) +
                              (static_cast<int64_t>(seq) * a.hq + h0 + (hv ? g : 0)) * D;
+      if constexpr (CK == kCacheE4M3) {
+        // dims 16ks + 4tig .. +3 (the order ldmatrix gives 8-bit K rows)
+        uint2 qw[C::kDimTiles];
+        float amax = 0.f;
 #pragma unroll
-      for (int ks = 0; ks < C::kDimTiles; ++ks) {
-        if constexpr (CK == kCacheE4M3) {
-          // dims 16ks + 4tig .. +3 (the order ldmatrix gives 8-bit K rows)
-          const uint2 w = *reinterpret_cast<const uint2*>(qrow + ks * 16 + 4 * tig);
-          const float f0 = to_float<kQBF16>(w.x & 0xffff), f1 = to_float<kQBF16>(w.x >> 16);
-          const float f2 = to_float<kQBF16>(w.y & 0xffff), f3 = to_float<kQBF16>(w.y >> 16);
-          qf[ks][0] = hv ? pack_f16x2(f0, f1) : 0u;
-          qf[ks][1] = hv ? pack_f16x2(f2, f3) : 0u;
-        } else {
+        for (int ks = 0; ks < C::kDimTiles; ++ks) {
+          qw[ks] = hv ? *reinterpret_cast<const uint2*>(qrow + ks * 16 + 4 * tig) : make_uint2(0u, 0u);
+          amax = fmax3(amax, fabsf(to_float<kQBF16>(qw[ks].x & 0xffff)),
+                       fabsf(to_float<kQBF16>(qw[ks].x >> 16)));
+          amax = fmax3(amax, fabsf(to_float<kQBF16>(qw[ks].y & 0xffff)),
+                       fabsf(to_float<kQBF16>(qw[ks].y >> 16)));
+        }
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));  // the head's 4 threads
+        amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+        // e in [-126, 126]; 0 for a zero (or non-finite) query
+        const int e = (amax > 0.f && amax < INFINITY) ? max(-126, min(126, ilogbf(amax) - 14)) : 0;
+        const float down = __int_as_float((127 - e) << 23);  // 2^-e
+#pragma unroll
+        for (int ks = 0; ks < C::kDimTiles; ++ks) {
+          qf[ks][0] = pack_f16x2(to_float<kQBF16>(qw[ks].x & 0xffff) * down,
+                                 to_float<kQBF16>(qw[ks].x >> 16) * down);
+          qf[ks][1] = pack_f16x2(to_float<kQBF16>(qw[ks].y & 0xffff) * down,
+                                 to_float<kQBF16>(qw[ks].y >> 16) * down);
+        }
+        // columns 2tig and 2tig+1 of the score tile are heads 2tig, 2tig+1,
+        // whose exponents sit in row groups 2tig and 2tig+1
+        const int e0 = __shfl_sync(0xffffffffu, e, 8 * tig);
+        const int e1 = __shfl_sync(0xffffffffu, e, 8 * tig + 4);
+        sl2c[0] = a.sl2 * __int_as_float((127 + e0) << 23);
+        sl2c[1] = a.sl2 * __int_as_float((127 + e1) << 23);
+      } else {
+#pragma unroll
+        for (int ks = 0; ks < C::kDimTiles; ++ks) {
           qf[ks][0] = hv ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * tig) : 0u;
           qf[ks][1] = hv ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * tig) : 0u;
         }
@@ -399,11 +433,6 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
       for (int e = 0; e < 4; ++e) acc[dt][e] = 0.f;
     float m_run[2] = {-INFINITY, -INFINITY};  // heads 2tig, 2tig+1 (log2 units)
     float l_run[2] = {0.f, 0.f};              // this thread's share of the sums
-
-    if (!failed) {
-      const int pro = min(kStages, nb_w);
-      for (int i = 0; i < pro; ++i) issue(i);
-    }
 
     const int li = lane >> 3;  // which 8x8 matrix of an ldmatrix.x4 this lane addresses
     for (int i = 0; i < nb_w; ++i) {
@@ -463,7 +492,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int tok = tbase + mt * 16 + g + (e >> 1) * 8;
-            const float x = ((s0[e] + s1[e]) + (s2[e] + s3[e])) * a.sl2;
+            const float x = ((s0[e] + s1[e]) + (s2[e] + s3[e])) * sl2c[e & 1];
             s[mt][e] = tok < t1 ? x : -INFINITY;
           }
         }

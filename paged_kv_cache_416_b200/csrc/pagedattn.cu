@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "cache_ops.cuh"
@@ -43,15 +44,38 @@ int current_device(int* dev) {
   return 0;
 }
 
-// SM count of the current device (cached per device).
+// SM count of the current device (cached per device; host threads that make
+// their first call at once may both query it and store the same value).
 int device_sms(int dev) {
-  static int cache[kMaxDevices] = {0};
-  if (cache[dev] == 0) {
-    int n = 0;
+  static std::atomic<int> cache[kMaxDevices] = {};
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cache[dev] = n > 0 ? n : 1;
+    n = n > 0 ? n : 1;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
+}
+
+// Resident CTAs per SM of a persistent kernel on device `dev`, cached per
+// (kernel, device) in `occ`.  The first call on a device raises the kernel's
+// dynamic shared-memory limit; concurrent first calls repeat that idempotent
+// step and store the same value.
+template <typename Kern>
+pa_status resident_ctas(std::atomic<int>* occ, int dev, Kern kern, int threads, int smem_bytes,
+                        const char* what, int* out) {
+  int n = occ[dev].load(std::memory_order_acquire);
+  if (n == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem_bytes);
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, threads, smem_bytes);
+    if (e != cudaSuccess) return cuda_fail(e, what);
+    n = n > 0 ? n : 1;
+    occ[dev].store(n, std::memory_order_release);
+  }
+  *out = n;
+  return PA_OK;
 }
 
 int elem_bytes(pa_dtype t) { return t == PA_FP8_E4M3 ? 1 : 2; }
@@ -233,18 +257,13 @@ pa_status launch_decode_main(const pa::DecodeArgs& args, int64_t items_upper, in
                              cudaStream_t stream) {
   using C = pa::DecodeCfg<CK, D, BS>;
   auto kern = pa::decode_kernel<CK, kQBF16, D, BS>;
-  static int occ[kMaxDevices] = {0};
-  if (occ[dev] == 0) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(decode)");
-    int n = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, pa::kDecodeThreads, C::kSmemBytes);
-    if (e != cudaSuccess) return cuda_fail(e, "occupancy(decode)");
-    occ[dev] = n > 0 ? n : 1;
-  }
+  static std::atomic<int> occ[kMaxDevices] = {};
+  int per_sm = 0;
+  const pa_status os = resident_ctas(occ, dev, kern, pa::kDecodeThreads, C::kSmemBytes,
+                                     "pa_decode: kernel set-up", &per_sm);
+  if (os != PA_OK) return os;
   const int64_t grid = std::max<int64_t>(
-      1, std::min<int64_t>(items_upper, static_cast<int64_t>(device_sms(dev)) * occ[dev]));
+      1, std::min<int64_t>(items_upper, static_cast<int64_t>(device_sms(dev)) * per_sm));
   const cudaError_t e = launch_behind_plan(kern, static_cast<unsigned>(grid), pa::kDecodeThreads,
                                            C::kSmemBytes, stream, args);
   if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
@@ -266,18 +285,13 @@ pa_status launch_cascade(const pa::CascadeArgs& args, int64_t items_upper, int d
                          cudaStream_t stream) {
   using C = pa::DecodeCfg<kBF16 ? pa::kCacheBF16 : pa::kCacheF16, D, BS>;
   auto kern = pa::cascade_kernel<kBF16, D, BS>;
-  static int occ[kMaxDevices] = {0};
-  if (occ[dev] == 0) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::kSmemBytes);
-    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(cascade)");
-    int n = 0;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, kern, pa::kDecodeThreads, C::kSmemBytes);
-    if (e != cudaSuccess) return cuda_fail(e, "occupancy(cascade)");
-    occ[dev] = n > 0 ? n : 1;
-  }
+  static std::atomic<int> occ[kMaxDevices] = {};
+  int per_sm = 0;
+  const pa_status os = resident_ctas(occ, dev, kern, pa::kDecodeThreads, C::kSmemBytes,
+                                     "pa_decode_shared_prefix: kernel set-up", &per_sm);
+  if (os != PA_OK) return os;
   const int64_t grid = std::max<int64_t>(
-      1, std::min<int64_t>(items_upper, static_cast<int64_t>(device_sms(dev)) * occ[dev]));
+      1, std::min<int64_t>(items_upper, static_cast<int64_t>(device_sms(dev)) * per_sm));
   const cudaError_t e = launch_behind_plan(kern, static_cast<unsigned>(grid), pa::kDecodeThreads,
                                            C::kSmemBytes, stream, args);
   if (e != cudaSuccess) return cuda_fail(e, "pa_decode_shared_prefix launch");
@@ -826,18 +840,58 @@ pa_status pa_validate_block_tables(const int32_t* block_tables, int32_t max_bloc
 static __device__ __align__(256) uint8_t g_noalloc_scratch[PA_DECODE_NOALLOC_SCRATCH_BYTES];
 
 namespace {
-// Device address of g_noalloc_scratch, looked up once per device.
-std::atomic<void*> g_noalloc_ptr[kMaxDevices];
+// Device address of g_noalloc_scratch, looked up once per device and CUDA
+// context: the array lives in the library's module of each context, so a
+// new context on the same device (after cudaDeviceReset, or a caller's own
+// non-primary context) gets its own address.  Contexts are told apart by
+// the driver's unique context id, which is never reused within a process.
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+template <typename Fn>
+Fn driver_fn(const char* name) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(p);
+}
+
+// Unique id of the calling thread's current context (0 if none).
+unsigned long long current_context_id() {
+  static const CtxGetCurrentFn get_ctx = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_ctx == nullptr || get_id == nullptr || get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+      get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+struct NoallocSlot {
+  unsigned long long ctx_id = 0;
+  void* ptr = nullptr;
+};
+std::mutex g_noalloc_mu;
+NoallocSlot g_noalloc_slot[kMaxDevices];
 
 pa_status noalloc_scratch(int dev, void** ptr) {
-  void* p = g_noalloc_ptr[dev].load(std::memory_order_acquire);
-  if (p == nullptr) {
+  // cudaGetDevice made the device's primary context current if the thread
+  // had none, so the id below is the context the launches will use
+  const unsigned long long id = current_context_id();
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoallocSlot& slot = g_noalloc_slot[dev];
+  if (slot.ptr == nullptr || id == 0 || slot.ctx_id != id) {
+    void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr)
       return cuda_fail(e, "pa_decode_noalloc: cudaGetSymbolAddress of the built-in scratch");
-    g_noalloc_ptr[dev].store(p, std::memory_order_release);
+    slot.ctx_id = id;
+    slot.ptr = p;
   }
-  *ptr = p;
+  *ptr = slot.ptr;
   return PA_OK;
 }
 }  // namespace

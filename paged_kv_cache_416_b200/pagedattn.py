@@ -25,6 +25,7 @@ import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libpagedattn.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "pagedattn.h")
 
 PA_F16, PA_BF16, PA_FP8_E4M3 = 0, 1, 2
 STATUS_NAMES = {
@@ -102,7 +103,24 @@ pa_validate_block_tables = _lib.pa_validate_block_tables
 # pa_decode for callers that cannot allocate device memory: the scratch comes
 # from an array the library reserves when it is loaded (see the header)
 pa_decode_noalloc = _lib.pa_decode_noalloc
-NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
+
+
+def _header_size_define(name: str) -> int:
+    """Value of a `#define NAME (a * b * ...)` size constant of the C header,
+    so that the binding and the library take it from one source."""
+    import re
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    m = re.search(r"#define\s+" + name + r"\s+\(([^)]*)\)", text)
+    if m is None:
+        raise ImportError(f"{name} is not defined in {HEADER_PATH}")
+    value = 1
+    for factor in m.group(1).split("*"):
+        value *= int(factor.strip().rstrip("uUlL"))
+    return value
+
+
+NOALLOC_SCRATCH_BYTES = _header_size_define("PA_DECODE_NOALLOC_SCRATCH_BYTES")
 
 ENTRY_POINTS = [
     "pa_write_kv", "pa_copy_blocks", "pa_swap_blocks", "pa_hash_blocks", "pa_decode_split_tokens", "pa_decode_workspace_size",

@@ -196,18 +196,36 @@ def _generic(name, lens, hq, hkv, d, bs, q_dtype, cache_dtype, seed, device,
     )
 
 
+def _lens_tiny(lens=(40, 16, 1, 63)):
+    return np.asarray(lens, dtype=np.int64)
+
+
+def _lens_llama13b(seed, num_seqs=64, max_len=2048, min_len=128):
+    rng = np.random.default_rng(seed + 1000)
+    return rng.integers(min_len, max_len + 1, size=num_seqs)
+
+
+def _lens_llama70b(num_seqs=256, context_len=4096):
+    return np.full(num_seqs, context_len, dtype=np.int64)
+
+
+def _lens_fp8(seed, num_seqs=128, max_len=32768):
+    rng = np.random.default_rng(seed + 1000)
+    return np.clip(np.rint(rng.lognormal(math.log(1024.0), 1.0, size=num_seqs)), 1,
+                   max_len).astype(np.int64)
+
+
 def tiny(seed=1, device="cpu", **kw) -> Workload:
     """4 sequences, lens [40,16,1,63], 4/4 heads, D 64, fp16, bs 16, a 64-block
     pool whose free list is a seeded shuffle (9 blocks used)."""
-    lens = kw.pop("lens", [40, 16, 1, 63])
+    lens = _lens_tiny(kw.pop("lens", (40, 16, 1, 63)))
     return _generic("tiny", lens, 4, 4, 64, 16, "f16", "f16", seed, device, num_blocks=64, **kw)
 
 
 def llama13b_mha(seed=2, device="cpu", num_seqs=64, max_len=2048, min_len=128, **kw) -> Workload:
     """LLaMA-13B-shaped MHA layer: 40/40 heads, D 128, fp16, bs 16,
     lens U{min_len..max_len}."""
-    rng = np.random.default_rng(seed + 1000)
-    lens = rng.integers(min_len, max_len + 1, size=num_seqs)
+    lens = _lens_llama13b(seed, num_seqs, max_len, min_len)
     return _generic("llama13b_mha", lens, 40, 40, 128, kw.pop("block_size", 16), "f16", "f16",
                     seed, device, **kw)
 
@@ -215,7 +233,7 @@ def llama13b_mha(seed=2, device="cpu", num_seqs=64, max_len=2048, min_len=128, *
 def llama70b_gqa(seed=3, device="cpu", num_seqs=256, context_len=4096, **kw) -> Workload:
     """Llama-3-70B-shaped GQA layer: 64/8 heads, D 128, bf16, bs 16, every
     sequence ``context_len`` tokens."""
-    lens = [context_len] * num_seqs
+    lens = _lens_llama70b(num_seqs, context_len)
     return _generic("llama70b_gqa", lens, 64, 8, 128, kw.pop("block_size", 16), "bf16", "bf16",
                     seed, device, **kw)
 
@@ -223,8 +241,7 @@ def llama70b_gqa(seed=3, device="cpu", num_seqs=256, context_len=4096, **kw) -> 
 def fp8_longtail(seed=5, device="cpu", num_seqs=128, block_size=16, max_len=32768, **kw) -> Workload:
     """Llama-3-8B-shaped layer, e4m3 cache: 32/8 heads, D 128, q bf16, lens
     lognormal(ln 1024, 1) rounded and clipped to [1, max_len]."""
-    rng = np.random.default_rng(seed + 1000)
-    lens = np.clip(np.rint(rng.lognormal(math.log(1024.0), 1.0, size=num_seqs)), 1, max_len).astype(np.int64)
+    lens = _lens_fp8(seed, num_seqs, max_len)
     w = _generic(f"fp8_longtail_bs{block_size}", lens, 32, 8, 128, block_size, "bf16", "e4m3",
                  seed, device, **kw)
     return w
@@ -237,13 +254,29 @@ def _sample_groups(prompts: int, samples: int) -> Dict:
             "group_seqs": np.arange(prompts * samples, dtype=np.int32)}
 
 
+def _shared_prefix_draws(seed, prompts, samples, prefix, max_tail, bs):
+    """Prompt lengths (prefix + r, r ~ U{1..bs-1}) and own-token counts
+    T ~ U{0..max_tail} per sample, and the generator that drew them (the
+    batch draws its free-list order from it next)."""
+    rng = np.random.default_rng(seed + 1000)
+    extra = rng.integers(1, bs, size=prompts)
+    tails = rng.integers(0, max_tail + 1, size=(prompts, samples))
+    return rng, prefix + extra, tails
+
+
+def _lens_shared_prefix(phase, seed, prompts=32, samples=4, prefix=1024, max_tail=512, bs=16,
+                        **_):
+    """Context lengths of the shared-prefix batch: the prompt and the fork
+    step's token; later also T own tokens and the step's token."""
+    _, plen, tails = _shared_prefix_draws(seed, prompts, samples, prefix, max_tail, bs)
+    first = np.repeat(plen + 1, samples)
+    return first if phase == "fork" else first + tails.reshape(-1) + 1
+
+
 def _shared_prefix(phase, seed, device, prompts=32, samples=4, prefix=1024,
                    max_tail=512, hq=32, hkv=8, d=128, bs=16) -> Workload:
     """Parallel sampling over a shared prompt (see the module docstring)."""
-    rng = np.random.default_rng(seed + 1000)
-    extra = rng.integers(1, bs, size=prompts)              # r ~ U{1..bs-1}
-    plen = prefix + extra                                  # shared prompt lengths
-    tails = rng.integers(0, max_tail + 1, size=(prompts, samples))
+    rng, plen, tails = _shared_prefix_draws(seed, prompts, samples, prefix, max_tail, bs)
     B = prompts * samples
     # pool: shared prompt blocks once, plus every sample's own blocks
     own = 0
@@ -376,6 +409,37 @@ def prefill(seed=6, device="cpu", ctxs=(200, 300, 1, 77), nqs=(200, 77, 1, 50), 
     gen = torch.Generator(device=device).manual_seed(int(seed) + 77)
     q = _to_storage(_randn((int(qs[-1]), hq, d), gen, device), dtype)
     return PrefillWorkload(base=base, q=q, query_start=qs)
+
+
+# (kv heads, head_dim, bytes per cache element) and the length rule of each
+# workload, for sizes without building pools
+_SHAPES = {"tiny": (4, 64, 2), "llama13b_mha": (40, 128, 2), "llama70b_gqa": (8, 128, 2),
+           "shared_prefix_fork": (8, 128, 2), "shared_prefix_tails": (8, 128, 2),
+           "fp8_longtail_bs16": (8, 128, 1), "fp8_longtail_bs32": (8, 128, 1)}
+_DEFAULT_SEEDS = {"tiny": 1, "llama13b_mha": 2, "llama70b_gqa": 3, "shared_prefix_fork": 4,
+                  "shared_prefix_tails": 4, "fp8_longtail_bs16": 5, "fp8_longtail_bs32": 5}
+
+
+def context_lens(name: str, seed: Optional[int] = None, **kw) -> np.ndarray:
+    """The context lengths :func:`make` gives for the same arguments, without
+    building the pools."""
+    seed = _DEFAULT_SEEDS[name] if seed is None else seed
+    if name == "tiny":
+        return _lens_tiny(kw.get("lens", (40, 16, 1, 63)))
+    if name == "llama13b_mha":
+        return _lens_llama13b(seed, **{k: kw[k] for k in ("num_seqs", "max_len", "min_len") if k in kw})
+    if name == "llama70b_gqa":
+        return _lens_llama70b(**{k: kw[k] for k in ("num_seqs", "context_len") if k in kw})
+    if name.startswith("fp8_longtail"):
+        return _lens_fp8(seed, **{k: kw[k] for k in ("num_seqs", "max_len") if k in kw})
+    return _lens_shared_prefix(name.split("_")[-1], seed, **kw)
+
+
+def kv_bytes_of(name: str, seed: Optional[int] = None, **kw) -> int:
+    """Algorithmic K+V bytes one decode of the workload reads (as
+    ``make(name, seed, **kw).kv_bytes``), from the lengths alone."""
+    hkv, d, e = _SHAPES[name]
+    return int(context_lens(name, seed, **kw).astype(np.int64).sum()) * hkv * d * 2 * e
 
 
 REGISTRY = {

@@ -84,3 +84,74 @@ def test_reference_arm_prints_one_line(capsys):
     assert line["impl"] == "reference" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle"
     assert line["e2e"]["h2d_bytes_per_step"] == 0
+
+
+NCU_CSV = '''==PROF== Connected to process 4242
+"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Block Size","Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"
+"3","4242","python3","127.0.0.1","void pa::plan_kernel(const int *, int)","1","7","(1024, 1, 1)","(1, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","byte","4,096"
+"4","4242","python3","127.0.0.1","void pa::decode_kernel<1, true, 128, 16>(pa::DecodeArgs)","1","7","(128, 1, 1)","(444, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","Mbyte","1,077.45"
+"4","4242","python3","127.0.0.1","void pa::decode_kernel<1, true, 128, 16>(pa::DecodeArgs)","1","7","(128, 1, 1)","(444, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","7,160,000"
+"4","4242","python3","127.0.0.1","void pa::decode_kernel<1, true, 128, 16>(pa::DecodeArgs)","1","7","(128, 1, 1)","(444, 1, 1)","0","10.0","Command line profiler metrics","gpu__time_duration.sum","usecond","183.90"
+'''
+
+
+def test_ingest_ncu_records_scaled_traffic(tmp_path, monkeypatch):
+    """An ncu metrics log of the decode kernel on 64 of the headline batch's
+    256 sequences becomes a traffic record scaled x4 to the full batch, keyed
+    to the kernel's source hash; bench reads it back only while the hash
+    matches."""
+    sys.path.insert(0, ROOT)
+    import json
+    import bench
+    csv_path = tmp_path / "launches.csv"
+    csv_path.write_text(NCU_CSV)
+    traffic = tmp_path / "traffic.json"
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(traffic))
+    launches = bench.parse_ncu_csv(str(csv_path), "decode_kernel")
+    assert list(launches) == ["4"]
+    m = launches["4"]
+    assert m["dram__bytes_read.sum"] == pytest.approx(1.07745e9)
+    assert m["gpu__time_duration.sum"] == pytest.approx(183.9e-6)
+    assert bench.main(["--ingest-ncu", str(csv_path), "--num-seqs", "64",
+                       "--ingest-command", "ncu ... bench.py --num-seqs 64"]) == 0
+    rec = json.loads(traffic.read_text())["decode_kernel:llama70b_gqa"]
+    assert rec["scale_to_full"] == pytest.approx(4.0)
+    assert rec["dram_bytes_per_launch_full"] == round((1.07745e9 + 7.16e6) * 4)
+    assert rec["source_sha16"] == bench.source_hash("decode_kernel")
+    got, _ = bench.profiled_traffic("llama70b_gqa")
+    assert got == rec["dram_bytes_per_launch_full"]
+    # a changed kernel source makes the figure stale
+    monkeypatch.setattr(bench, "source_hash", lambda k: "0" * 16)
+    assert bench.profiled_traffic("llama70b_gqa")[0] is None
+
+
+def test_config_memory_figures():
+    """Paged waste is the unfilled tail of each last block; a contiguous
+    reservation wastes its length minus the context; the shared-prefix batch
+    holds its prompt blocks once for four samples."""
+    sys.path.insert(0, ROOT)
+    import bench
+    from paged_kv_cache_416_b200 import workloads as W
+    w = W.make("tiny")
+    m = bench.config_memory(w, "tiny")
+    # lens [40, 16, 1, 63] in blocks of 16: 3 + 1 + 1 + 4 blocks, 144 slots, 120 used
+    assert m["paged_unused_slots"] == 24 and m["reserved_unused_slots"] == 4 * 2048 - 120
+    w = W.make("shared_prefix_tails", prompts=3)
+    m = bench.config_memory(w, "shared_prefix_tails")
+    assert m["blocks_shared"] < m["blocks_unshared"]
+    assert 0 < m["memory_saved_pct"] < 75
+
+
+@pytest.mark.parametrize("name,kw", [("tiny", {}), ("llama13b_mha", dict(num_seqs=6)),
+                                     ("llama70b_gqa", dict(num_seqs=3, context_len=1000)),
+                                     ("shared_prefix_fork", dict(prompts=3)),
+                                     ("shared_prefix_tails", dict(prompts=3)),
+                                     ("fp8_longtail_bs16", dict(num_seqs=10, max_len=6000)),
+                                     ("fp8_longtail_bs32", dict(num_seqs=10))])
+def test_lengths_without_pools_match_the_generators(name, kw):
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    from paged_kv_cache_416_b200 import workloads as W
+    w = W.make(name, **kw)
+    assert np.array_equal(W.context_lens(name, **kw), w.context_lens)
+    assert W.kv_bytes_of(name, **kw) == w.kv_bytes

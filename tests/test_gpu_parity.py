@@ -268,6 +268,26 @@ def test_e4m3_every_code_decodes_exactly(pa):
         np.testing.assert_array_equal(got[h], want[h // 2])
 
 
+@pytest.mark.parametrize("split", [0, 64])
+def test_e4m3_cache_takes_any_bf16_query_range(pa, split):
+    """With an e4m3 cache the products run in fp16: each head's query is
+    scaled by a power of two before its fp16 conversion, so queries far
+    outside the fp16 range (components of 1e5 and 1e20) and far below it
+    (1e-6, 1e-20) still match the oracle."""
+    rng = np.random.default_rng(43)
+    lens = rng.integers(1, 400, size=7)
+    hq, hkv = 8, 2
+    w = W._generic("q_range", lens, hq, hkv, 128, 16, "bf16", "e4m3", seed=43, device="cpu")
+    factors = torch.tensor([1e5, 1e-6, 1.0, 7e4, 1e20, 1e-20, 300.0, 2.5e5])
+    q = (w.q.float() * factors[None, :, None]).to(torch.bfloat16)
+    assert (q.float().abs().amax(dim=(0, 2))[[0, 3, 4, 7]] > 65504).all()
+    w2 = W.Workload(**{**w.__dict__, "q": q})
+    out, _, _ = gpu_step(pa, w2, split_tokens=split)
+    ref, _, _ = oracle_step(w2)
+    assert torch.isfinite(out.float()).all()
+    assert_attention_close(as_f64(out), ref, f"e4m3 cache, scaled queries, split {split}")
+
+
 # ------------------------------------------------------ device error word
 
 def test_out_of_range_indices_are_reported_not_faulted(pa):

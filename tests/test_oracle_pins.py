@@ -361,6 +361,37 @@ def test_write_kv_skips_padding_and_quantises_in_fp32():
     assert kp.sum() == kp[1, 1].sum() + kp[3, 3].sum()  # the padding token wrote nothing
 
 
+@pytest.mark.parametrize("in_dt", ["bf16", "f16"])
+def test_write_kv_e4m3_matches_library_cast(in_dt):
+    """The whole e4m3 branch of write_kv (decode of the 16-bit input, fp32
+    division by the scale, RNE, saturation) against torch's own cast of
+    (x.float() / scale).clamp(-448, 448) to float8_e4m3fn: random values at
+    two scales, exact ties between neighbouring codes, values past the
+    saturation boundary and infinities."""
+    td = W.TORCH_DTYPE[in_dt]
+    g = torch.Generator().manual_seed(31)
+    hkv, d = 2, 64
+    vals = torch.from_numpy(codecs.e4m3_finite_values())
+    mids = (vals[:-1] + vals[1:]) / 2               # ties: 4 significant bits, exact in 16 bits
+    edge = torch.tensor([440.0, 448.0, 456.0, 464.0, 480.0, 500.0, 1e4, float("inf"),
+                         -float("inf"), 2.0 ** -9, 2.0 ** -10, 3 * 2.0 ** -11])
+    for scale in (0.5, 0.0123):
+        pieces = [torch.randn(4096, generator=g) * 3 * scale]
+        if scale == 0.5:                            # a power of two keeps ties exact after /scale
+            pieces += [mids * scale, -mids * scale, edge * scale, -edge * scale]
+        x = torch.cat(pieces).to(td)
+        n = -(-x.numel() // (hkv * d)) * hkv * d
+        x = torch.cat([x, torch.zeros(n - x.numel(), dtype=td)]).reshape(-1, hkv, d)
+        T = x.shape[0]
+        xr = raw(x)
+        kp = np.zeros((T, 1, hkv, d), dtype=np.uint8)
+        vp = np.zeros((T, 1, hkv, d), dtype=np.uint8)
+        paged.write_kv(xr, xr, in_dt, np.arange(T), kp, vp, "e4m3", k_scale=scale, v_scale=scale)
+        ref = (x.float() / scale).clamp(-448, 448).to(torch.float8_e4m3fn).view(torch.uint8)
+        assert np.array_equal(kp[:, 0], ref.numpy())
+        assert np.array_equal(vp[:, 0], ref.numpy())
+
+
 def test_fp8_decode_dequantises_with_the_scales():
     """An e4m3 cache decodes to code value * scale: attention over it equals
     attention over the dequantised fp64 cache (here checked via SDPA)."""
