@@ -68,7 +68,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
-    ap.add_argument("--seed", type=int, default=3)
+    ap.add_argument("--seed", type=int, default=None,
+                    help="input seed (default: the workload's own, 1..5 by configuration)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -288,7 +289,7 @@ def ingest_ncu(args):
         raise SystemExit(f"no {args.ingest_kernel} launch in {args.ingest_ncu}")
     rd = [m["dram__bytes_read.sum"] for m in launches.values()]
     wr = [m["dram__bytes_write.sum"] for m in launches.values()]
-    seed = args.seed if args.workload == DEFAULT_WORKLOAD else None
+    seed = args.seed
     kw = _sample_kw(args.workload, args.num_seqs) if args.num_seqs else {}
     cap_bytes = W.kv_bytes_of(args.workload, seed, **kw)
     full_bytes = W.kv_bytes_of(args.workload, seed)
@@ -369,6 +370,12 @@ def oracle_rate(name: str, seed, target_seconds: float, pool):
             "seq_tokens_per_s": round(w.seq_tokens / wall, 1), "seconds": round(wall, 2)}
 
 
+def workload_seed(name: str, seed=None) -> int:
+    """The seed a run uses: --seed if given, else the workload's own."""
+    from paged_kv_cache_416_b200 import workloads as W
+    return W.default_seed(name) if seed is None else int(seed)
+
+
 def _full_seqs(name):
     return {"llama70b_gqa": 256, "llama13b_mha": 64, "fp8_longtail_bs16": 128,
             "fp8_longtail_bs32": 128, "shared_prefix_tails": 128, "shared_prefix_fork": 128,
@@ -396,7 +403,7 @@ def run_ours(args, rank, local, world):
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
     kw = _sample_kw(args.workload, args.num_seqs) if args.num_seqs else {}
-    w = W.make(args.workload, seed=args.seed + rank, device=device, **kw)
+    w = W.make(args.workload, seed=workload_seed(args.workload, args.seed) + rank, device=device, **kw)
     stream = torch.cuda.current_stream()
     kp, vp = w.k_pool, w.v_pool
     q = w.q.contiguous()
@@ -529,8 +536,7 @@ def run_ours(args, rank, local, world):
         with OraclePool(host_cores()) as pool:
             cpu = oracle_rate(args.workload, args.seed, args.cpu_seconds, pool)
             for name, c in (configs or {}).items():
-                seed = args.seed if name == args.workload else None
-                c["cpu_baseline"] = oracle_rate(name, seed, args.config_cpu_seconds, pool)
+                c["cpu_baseline"] = oracle_rate(name, None, args.config_cpu_seconds, pool)
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -834,12 +840,12 @@ def run_swap(args):
     from paged_kv_cache_416_b200 import pagedattn as pa
     torch.cuda.set_device(0)
     nb, shape = 2048, (16, 8, 128)
-    g = torch.Generator(device="cuda").manual_seed(args.seed)
+    g = torch.Generator(device="cuda").manual_seed(workload_seed("llama70b_gqa", args.seed))
     dev_k = torch.randn((8192,) + shape, generator=g, device="cuda").to(torch.bfloat16)
     dev_v = torch.randn((8192,) + shape, generator=g, device="cuda").to(torch.bfloat16)
     host_k = torch.empty((nb,) + shape, dtype=torch.bfloat16).pin_memory()
     host_v = torch.empty((nb,) + shape, dtype=torch.bfloat16).pin_memory()
-    gc = torch.Generator().manual_seed(args.seed)
+    gc = torch.Generator().manual_seed(workload_seed("llama70b_gqa", args.seed))
     src = torch.randperm(8192, generator=gc)[:nb]
     dst = torch.randperm(nb, generator=gc)
     out_pairs = torch.stack([src, dst], 1).to(torch.int64).cuda()
@@ -886,7 +892,7 @@ def run_hash(args):
     from paged_kv_cache_416_b200 import pagedattn as pa
     torch.cuda.set_device(0)
     B, L, bs = 256, 4096, 16
-    g = torch.Generator(device="cuda").manual_seed(args.seed)
+    g = torch.Generator(device="cuda").manual_seed(workload_seed("llama70b_gqa", args.seed))
     toks = torch.randint(0, 128256, (B, L), generator=g, device="cuda", dtype=torch.int32)
     lens = torch.full((B,), L, dtype=torch.int32, device="cuda")
     out = torch.empty((B, L // bs), dtype=torch.int64, device="cuda")
@@ -931,7 +937,7 @@ def run_prefill(args):
     from paged_kv_cache_416_b200 import workloads as W
     torch.cuda.set_device(0)
     n = 4096
-    pw = W.prefill(seed=args.seed, device="cuda", ctxs=(n,) * 8, nqs=(n,) * 8, hq=64, hkv=8,
+    pw = W.prefill(seed=workload_seed("llama70b_gqa", args.seed), device="cuda", ctxs=(n,) * 8, nqs=(n,) * 8, hq=64, hkv=8,
                    bs=16, dtype="bf16")
     b = pw.base
     q = pw.q
@@ -990,7 +996,7 @@ def run_shared_prefix(args):
     from paged_kv_cache_416_b200 import pagedattn as pa
     from paged_kv_cache_416_b200 import workloads as W
     torch.cuda.set_device(0)
-    w = W.make("shared_prefix_tails", seed=args.seed, device="cuda")
+    w = W.make("shared_prefix_tails", seed=args.seed, device="cuda")  # None: its own seed
     kp, vp = w.k_pool, w.v_pool
     pa.write_kv(w.new_k, w.new_v, torch.from_numpy(w.slot_mapping).cuda(), kp, vp)
     q = w.q.contiguous()

@@ -41,7 +41,7 @@
  *
  * Supported: D in {64, 128}; bs in {16, 32}; Hq a multiple of Hkv with
  * Hq / Hkv <= 64 for pa_decode (a kv head's query heads are taken 8 at a
- * time: more than 8 read its blocks once per group of 8), <= 8 for the
+ * time: more than 8 read its blocks once per group of 8), <= 16 for the
  * shared-prefix decode; cache dtype f16 (q f16), bf16 (q bf16) or e4m3 (q f16 or
  * bf16).  With an e4m3 cache the tensor-core products run in fp16: each
  * head's query is first scaled by a power of two that brings its largest
@@ -280,12 +280,14 @@ size_t pa_decode_shared_prefix_workspace_size(int32_t num_seqs, int32_t num_q_he
  *   - up to 16 / (Hq/Hkv) members form a chunk whose query heads are the
  *     rows of one tile: the shared blocks are attended once by all rows,
  *     each member's own blocks by its own heads, in ranges of blocks whose
- *     partial results are merged by log-sum-exp.
- * Supported: q and cache both f16 or both bf16 (no e4m3), head_dim 64 or
- * 128, block_size 16 or 32, Hq / Hkv <= 8.  split_tokens: 0 = automatic,
- * else the shortest range in tokens.  workspace: at least
- * pa_decode_shared_prefix_workspace_size(...) bytes, 256-byte aligned,
- * stream-ordered use only.  Other errors as pa_decode.
+ *     partial results are merged by log-sum-exp.  With more than 8 query
+ *     heads per kv head a chunk is one member (its heads fill the tile).
+ * Supported: as pa_decode's caches (f16 with q f16, bf16 with q bf16, e4m3
+ * with q f16 or bf16 and the per-tensor k_scale / v_scale, which are ignored
+ * for 16-bit caches), head_dim 64 or 128, block_size 16 or 32, Hq / Hkv <= 16.
+ * split_tokens: 0 = automatic, else the shortest range in tokens.
+ * workspace: at least pa_decode_shared_prefix_workspace_size(...) bytes,
+ * 256-byte aligned, stream-ordered use only.  Other errors as pa_decode.
  */
 pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype q_dtype,
                                   const void* k_pool, const void* v_pool, pa_dtype cache_dtype,
@@ -294,8 +296,9 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype q_dtype,
                                   const int32_t* group_start, const int32_t* group_seqs,
                                   int32_t num_groups, int32_t num_seqs, int32_t num_q_heads,
                                   int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
-                                  int32_t num_blocks, float scale, int32_t split_tokens,
-                                  void* workspace, size_t workspace_bytes, pa_stream_t stream);
+                                  int32_t num_blocks, float scale, float k_scale, float v_scale,
+                                  int32_t split_tokens, void* workspace, size_t workspace_bytes,
+                                  pa_stream_t stream);
 
 /*
  * pa_prefill -- paged prefill / chunked-prefill attention on the 5th-

@@ -47,11 +47,14 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(s) <= t for s in sources())
 
 
-def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
-    """Compile the library unless it is newer than every source; returns its path."""
-    if not force and up_to_date():
+def build(force: bool = False, verbose: bool = False, extra_flags=None, out=None) -> str:
+    """Compile the library unless it is newer than every source; returns its
+    path.  With `out` (a test build with its own `extra_flags`, e.g. -D
+    defines), always compile, to that path instead of the package's library."""
+    target = LIB if out is None else str(out)
+    if out is None and not force and up_to_date():
         return LIB
-    cmd = [nvcc_path(), *ARCH_FLAGS, *CXX_FLAGS, *(extra_flags or []), "-o", LIB + ".tmp", MAIN_SRC]
+    cmd = [nvcc_path(), *ARCH_FLAGS, *CXX_FLAGS, *(extra_flags or []), "-o", target + ".tmp", MAIN_SRC]
     if verbose:
         print(" ".join(cmd), flush=True)
     r = subprocess.run(cmd, capture_output=True, text=True)
@@ -59,8 +62,8 @@ def build(force: bool = False, verbose: bool = False, extra_flags=None) -> str:
         raise RuntimeError(f"nvcc failed ({r.returncode}):\n{r.stdout}\n{r.stderr}")
     if verbose and (r.stdout or r.stderr):
         print(r.stdout, r.stderr, file=sys.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(target + ".tmp", target)
+    return target
 
 
 def main(argv=None):

@@ -63,15 +63,38 @@ struct CascadeArgs {
   float* lse_part;             // [slots * Hkv * 16]
   float* o_part;               // [slots * Hkv * 16 * D]
   int hq, hkv, group, max_blocks, num_blocks;
-  float sl2;                   // scale * log2(e)
+  float sl2;                   // scale * k_scale * log2(e)
+  float out_scale;             // v_scale
 };
 
-template <bool kBF16, int D, int BS>
+// Query fragments of an e4m3 cache, whose products run in fp16: the
+// values of one query row (or head) are scaled by the power of two 2^-e that
+// brings their largest |q| into [2^14, 2^15) before the fp16 conversion, and
+// 2^e goes back into that row's softmax scale.  Returns e (0 for a zero or
+// non-finite row); `amax` is this thread's share, reduced over the 4 threads
+// of its fragment row group.
+__device__ __forceinline__ int q_row_exponent(float amax) {
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+  amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 2));
+  return (amax > 0.f && amax < INFINITY) ? max(-126, min(126, ilogbf(amax) - 14)) : 0;
+}
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
+
+template <bool kQBF16>
+__device__ __forceinline__ float amax4(uint2 w) {
+  return fmax3(fmax3(0.f, fabsf(to_float<kQBF16>(w.x & 0xffff)), fabsf(to_float<kQBF16>(w.x >> 16))),
+               fabsf(to_float<kQBF16>(w.y & 0xffff)), fabsf(to_float<kQBF16>(w.y >> 16)));
+}
+
+template <int CK, bool kQBF16, int D, int BS>
 __global__ void __launch_bounds__(kDecodeThreads)
 cascade_kernel(const __grid_constant__ CascadeArgs a) {
-  using C = DecodeCfg<kBF16 ? kCacheBF16 : kCacheF16, D, BS>;
+  using C = DecodeCfg<CK, D, BS>;
+  constexpr bool kE4M3 = CK == kCacheE4M3;
+  constexpr bool kMmaBF16 = C::kMmaBF16;  // bf16 cache: bf16 products; f16 and e4m3: fp16
+  constexpr bool kPBF16 = kMmaBF16;       // bf16 P is kept as hi + lo parts
   constexpr int kStages = C::kStages;
-  constexpr int kNT = D / 8;  // 16-row path: output n-tiles (8 dims each)
+  constexpr int kNT = D / 8;  // 16-row form: output n-tiles (8 dims each)
   constexpr int kRows = kCascadeRows;
   static_assert(C::kWarpBytes >= (kRows * D + 2 * kRows) * 4, "warp ring too small for the merge");
   static_assert(kDecodeWarps * C::kWarpBytes >= (kCascadeMaxRanges + 1) * kRows * 4,
@@ -122,6 +145,9 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
     const int4 rd = a.ranges[slot];
     const int chunk = rd.x, member = rd.y, b0 = rd.z, b1 = rd.w;
     const bool shared = member < 0;
+    // the 16-row form serves shared ranges, and own ranges of a member with
+    // more than 8 heads per kv head; other own ranges take the 8-column form
+    const bool rowform = shared || G > kMaxGroup;
     const int4 c0 = a.chunks[2 * chunk];
     const int members = c0.y, slot0 = c0.w;
     const int nranges = a.chunks[2 * chunk + 1].x;
@@ -133,6 +159,7 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
     }
     __syncthreads();
     const int own_seq = s_seq[shared ? 0 : member];
+    const int own_ctx = shared ? 0 : s_ctx[member];
     const int nblk = b1 - b0;
     const int nb_w = nblk > warp ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
     const int32_t* table = a.block_tables + static_cast<int64_t>(own_seq) * a.max_blocks;
@@ -195,26 +222,61 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
       if (!failed && i + kStages < nb_w) issue(i + kStages);
     };
 
-    if (shared) {
-      // ================= shared range: 16-row tiles =====================
+    if (rowform) {
+      // ================= 16-row tiles =====================================
+      // rows: a shared range's are the chunk's (member r / G, head r % G),
+      // an own range's the member's G heads
+      const int nrows = shared ? rows : G;
       uint32_t qa[D / 16][4];
+      float sl2r[2] = {a.sl2, a.sl2};  // softmax scale of rows g, g + 8 (log2 units)
       {
         const uint16_t* qrow[2];
+        bool okr[2];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           const int r = g + 8 * h;
-          const int rr = r < rows ? r : 0;
+          okr[h] = r < nrows;
+          const int rr = okr[h] ? r : 0;
+          const int seq = s_seq[shared ? rr / G : member];
           qrow[h] = reinterpret_cast<const uint16_t*>(a.q) +
-                    (static_cast<int64_t>(s_seq[rr / G]) * a.hq + kvh * G + rr % G) * D;
+                    (static_cast<int64_t>(seq) * a.hq + kvh * G + rr % G) * D;
         }
-        const bool ok0 = g < rows, ok1 = g + 8 < rows;
+        if constexpr (kE4M3) {
+          // k-step ks takes dims 16 ks + 4 tig .. +3 (the order ldmatrix
+          // gives 8-bit K rows): a0 / a1 the first pair, a2 / a3 the second
+          uint2 qw[2][D / 16];
+          float am[2] = {0.f, 0.f};
 #pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          const int d0 = ks * 16 + 2 * tig;
-          qa[ks][0] = ok0 ? *reinterpret_cast<const uint32_t*>(qrow[0] + d0) : 0u;
-          qa[ks][1] = ok1 ? *reinterpret_cast<const uint32_t*>(qrow[1] + d0) : 0u;
-          qa[ks][2] = ok0 ? *reinterpret_cast<const uint32_t*>(qrow[0] + d0 + 8) : 0u;
-          qa[ks][3] = ok1 ? *reinterpret_cast<const uint32_t*>(qrow[1] + d0 + 8) : 0u;
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int ks = 0; ks < D / 16; ++ks) {
+              qw[h][ks] = okr[h] ? *reinterpret_cast<const uint2*>(qrow[h] + ks * 16 + 4 * tig)
+                                 : make_uint2(0u, 0u);
+              am[h] = fmaxf(am[h], amax4<kQBF16>(qw[h][ks]));
+            }
+          int e[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            e[h] = q_row_exponent(am[h]);
+            sl2r[h] = a.sl2 * pow2f(e[h]);
+          }
+          const float dn0 = pow2f(-e[0]), dn1 = pow2f(-e[1]);
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            qa[ks][0] = pack_f16x2(to_float<kQBF16>(qw[0][ks].x & 0xffff) * dn0, to_float<kQBF16>(qw[0][ks].x >> 16) * dn0);
+            qa[ks][1] = pack_f16x2(to_float<kQBF16>(qw[1][ks].x & 0xffff) * dn1, to_float<kQBF16>(qw[1][ks].x >> 16) * dn1);
+            qa[ks][2] = pack_f16x2(to_float<kQBF16>(qw[0][ks].y & 0xffff) * dn0, to_float<kQBF16>(qw[0][ks].y >> 16) * dn0);
+            qa[ks][3] = pack_f16x2(to_float<kQBF16>(qw[1][ks].y & 0xffff) * dn1, to_float<kQBF16>(qw[1][ks].y >> 16) * dn1);
+          }
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            const int d0 = ks * 16 + 2 * tig;
+            qa[ks][0] = okr[0] ? *reinterpret_cast<const uint32_t*>(qrow[0] + d0) : 0u;
+            qa[ks][1] = okr[1] ? *reinterpret_cast<const uint32_t*>(qrow[1] + d0) : 0u;
+            qa[ks][2] = okr[0] ? *reinterpret_cast<const uint32_t*>(qrow[0] + d0 + 8) : 0u;
+            qa[ks][3] = okr[1] ? *reinterpret_cast<const uint32_t*>(qrow[1] + d0 + 8) : 0u;
+          }
         }
       }
       float acc[kNT][4];
@@ -229,9 +291,12 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
         if (consume(st)) {
           const uint32_t sK = wbase_s + st * C::kStageBytes;
           const uint32_t sV = sK + C::kTileBytes;
+          // tokens of the block inside the range: all of a shared block; an
+          // own range's last block may end early
+          const int valid = shared ? BS : min(BS, own_ctx - (b0 + warp + i * kDecodeWarps) * BS);
 #pragma unroll
           for (int kt = 0; kt < BS / 16; ++kt) {
-            // S = Q K^T for 16 keys: two n-tiles, even / odd dim steps apart
+            // S = Q K^T for 16 keys: two n-tiles of 8 keys, two accumulator chains
             float s[2][4], so[2][4];
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
@@ -240,36 +305,61 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
               const int key = kt * 16 + nt * 8 + (lane & 7);
+              if constexpr (kE4M3) {
+                // one ldmatrix.x4 = four 16-dim chunks of 8 keys; matrix j
+                // gives this thread dims 16 (c + j) + 4 tig .. +3 of key g
 #pragma unroll
-              for (int ks = 0; ks < D / 16; ks += 2) {
-                uint32_t k0, k1, k2, k3;
-                ldsm_x4(sK + tile_off<C>(key, ((ks + (li >> 1)) * 16 + (li & 1) * 8) * 2), k0, k1,
-                        k2, k3);
-                mma_16816<kBF16>(s[nt], qa[ks], k0, k1);
-                mma_16816<kBF16>(so[nt], qa[ks + 1], k2, k3);
+                for (int c = 0; c < D / 16; c += 4) {
+                  uint32_t r[4];
+                  ldsm_x4(sK + tile_off<C>(key, (c + li) * 16), r[0], r[1], r[2], r[3]);
+#pragma unroll
+                  for (int j = 0; j < 4; ++j) {
+                    const uint32_t k0 = e4m3x2_to_f16x2(r[j] & 0xffff);
+                    const uint32_t k1 = e4m3x2_to_f16x2(r[j] >> 16);
+                    if (j & 1) mma_16816<false>(so[nt], qa[c + j], k0, k1);
+                    else mma_16816<false>(s[nt], qa[c + j], k0, k1);
+                  }
+                }
+              } else {
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ks += 2) {
+                  uint32_t k0, k1, k2, k3;
+                  ldsm_x4(sK + tile_off<C>(key, ((ks + (li >> 1)) * 16 + (li & 1) * 8) * 2), k0, k1,
+                          k2, k3);
+                  mma_16816<kMmaBF16>(s[nt], qa[ks], k0, k1);
+                  mma_16816<kMmaBF16>(so[nt], qa[ks + 1], k2, k3);
+                }
               }
             }
-            // online softmax of rows g (elements 0, 1) and g + 8 (2, 3): the
-            // shared blocks are whole and every row attends them
-            float alpha[2];
+            // online softmax of rows g (elements 0, 1) and g + 8 (2, 3), the
+            // running max raised only past kRescaleLog2 (as in decode)
+            float alpha[2] = {1.f, 1.f};
+            bool resc = false;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               float x[4];
 #pragma unroll
-              for (int nt = 0; nt < 2; ++nt) {
-                x[2 * nt] = (s[nt][2 * h] + so[nt][2 * h]) * a.sl2;
-                x[2 * nt + 1] = (s[nt][2 * h + 1] + so[nt][2 * h + 1]) * a.sl2;
-              }
-              float bm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+              for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                  const int key = kt * 16 + nt * 8 + 2 * tig + c;
+                  const float v = (s[nt][2 * h + c] + so[nt][2 * h + c]) * sl2r[h];
+                  x[2 * nt + c] = key < valid ? v : -INFINITY;
+                }
+              float bm = fmax3(fmaxf(x[0], x[1]), x[2], x[3]);
               bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
               bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
-              const float mn = fmaxf(m_run[h], bm);
-              alpha[h] = fast_exp2(m_run[h] - mn);
-              m_run[h] = mn;
+              if (m_run[h] == -INFINITY) {
+                m_run[h] = bm;  // first keys: O and the sum are still zero
+              } else if (bm - m_run[h] > kRescaleLog2) {
+                alpha[h] = fast_exp2(m_run[h] - bm);
+                m_run[h] = bm;
+                resc = true;
+              }
               float ps = 0.f;
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                x[e] = fast_exp2(x[e] - mn);
+                x[e] = fast_exp2(x[e] - m_run[h]);
                 ps += x[e];
               }
               l_run[h] = l_run[h] * alpha[h] + ps;
@@ -279,37 +369,68 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
                 s[nt][2 * h + 1] = x[2 * nt + 1];
               }
             }
+            if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll
-            for (int n = 0; n < kNT; ++n) {
-              acc[n][0] *= alpha[0];
-              acc[n][1] *= alpha[0];
-              acc[n][2] *= alpha[1];
-              acc[n][3] *= alpha[1];
+              for (int n = 0; n < kNT; ++n) {
+                acc[n][0] *= alpha[0];
+                acc[n][1] *= alpha[0];
+                acc[n][2] *= alpha[1];
+                acc[n][3] *= alpha[1];
+              }
             }
             // P as the A operand (the S accumulators of two n-tiles are the A
             // fragment); bf16 keeps P as hi + lo parts (one bf16 value errs by
             // up to 2^-9 of a weight), fp16 P keeps 11 bits in one part
             uint32_t pa[4], pl[4];
-            pa[0] = pack2<kBF16>(s[0][0], s[0][1]);
-            pa[1] = pack2<kBF16>(s[0][2], s[0][3]);
-            pa[2] = pack2<kBF16>(s[1][0], s[1][1]);
-            pa[3] = pack2<kBF16>(s[1][2], s[1][3]);
-            if constexpr (kBF16) {
+            pa[0] = pack2<kMmaBF16>(s[0][0], s[0][1]);
+            pa[1] = pack2<kMmaBF16>(s[0][2], s[0][3]);
+            pa[2] = pack2<kMmaBF16>(s[1][0], s[1][1]);
+            pa[3] = pack2<kMmaBF16>(s[1][2], s[1][3]);
+            if constexpr (kPBF16) {
               pl[0] = pack_bf16x2(s[0][0] - to_float<true>(pa[0] & 0xffff), s[0][1] - to_float<true>(pa[0] >> 16));
               pl[1] = pack_bf16x2(s[0][2] - to_float<true>(pa[1] & 0xffff), s[0][3] - to_float<true>(pa[1] >> 16));
               pl[2] = pack_bf16x2(s[1][0] - to_float<true>(pa[2] & 0xffff), s[1][1] - to_float<true>(pa[2] >> 16));
               pl[3] = pack_bf16x2(s[1][2] - to_float<true>(pa[3] & 0xffff), s[1][3] - to_float<true>(pa[3] >> 16));
             }
+            // O += P V; values of keys past an own range's end are zeroed in the
+            // fragments (they may hold anything, NaN included)
+            const bool part = valid < BS;
+            const int tk = kt * 16 + 2 * tig;
+            const uint32_t m_lo = part ? pair_mask(tk < valid, tk + 1 < valid) : 0xffffffffu;
+            const uint32_t m_hi = part ? pair_mask(tk + 8 < valid, tk + 9 < valid) : 0xffffffffu;
             const int vkey = kt * 16 + (li & 1) * 8 + (lane & 7);
+            if constexpr (kE4M3) {
+              // matrices (keys 0-7 | 8-15) x (chunk c | c + 1); after the byte
+              // permute the low half holds keys 2tig, 2tig+1 of dim 2g of the
+              // chunk, the high half of dim 2g + 1: n-tile 2 chunk + parity
 #pragma unroll
-            for (int n2 = 0; n2 < D / 16; ++n2) {
-              uint32_t v0, v1, v2, v3;
-              ldsm_x4_trans(sV + tile_off<C>(vkey, (n2 * 16 + (li >> 1) * 8) * 2), v0, v1, v2, v3);
-              mma_16816<kBF16>(acc[2 * n2], pa, v0, v1);
-              mma_16816<kBF16>(acc[2 * n2 + 1], pa, v2, v3);
-              if constexpr (kBF16) {
-                mma_16816<kBF16>(acc[2 * n2], pl, v0, v1);
-                mma_16816<kBF16>(acc[2 * n2 + 1], pl, v2, v3);
+              for (int c = 0; c < D / 16; c += 2) {
+                uint32_t r0, r1, r2, r3;
+                ldsm_x4_trans(sV + tile_off<C>(vkey, (c + (li >> 1)) * 16), r0, r1, r2, r3);
+                if (part) {
+                  r0 &= m_lo; r1 &= m_hi; r2 &= m_lo; r3 &= m_hi;
+                }
+                const uint32_t p0 = __byte_perm(r0, 0, 0x3120), p1 = __byte_perm(r1, 0, 0x3120);
+                const uint32_t p2 = __byte_perm(r2, 0, 0x3120), p3 = __byte_perm(r3, 0, 0x3120);
+                mma_16816<false>(acc[2 * c], pa, e4m3x2_to_f16x2(p0 & 0xffff), e4m3x2_to_f16x2(p1 & 0xffff));
+                mma_16816<false>(acc[2 * c + 1], pa, e4m3x2_to_f16x2(p0 >> 16), e4m3x2_to_f16x2(p1 >> 16));
+                mma_16816<false>(acc[2 * c + 2], pa, e4m3x2_to_f16x2(p2 & 0xffff), e4m3x2_to_f16x2(p3 & 0xffff));
+                mma_16816<false>(acc[2 * c + 3], pa, e4m3x2_to_f16x2(p2 >> 16), e4m3x2_to_f16x2(p3 >> 16));
+              }
+            } else {
+#pragma unroll
+              for (int n2 = 0; n2 < D / 16; ++n2) {
+                uint32_t v0, v1, v2, v3;
+                ldsm_x4_trans(sV + tile_off<C>(vkey, (n2 * 16 + (li >> 1) * 8) * 2), v0, v1, v2, v3);
+                if (part) {
+                  v0 &= m_lo; v1 &= m_hi; v2 &= m_lo; v3 &= m_hi;
+                }
+                mma_16816<kMmaBF16>(acc[2 * n2], pa, v0, v1);
+                mma_16816<kMmaBF16>(acc[2 * n2 + 1], pa, v2, v3);
+                if constexpr (kPBF16) {
+                  mma_16816<kMmaBF16>(acc[2 * n2], pl, v0, v1);
+                  mma_16816<kMmaBF16>(acc[2 * n2 + 1], pl, v2, v3);
+                }
               }
             }
           }
@@ -327,9 +448,17 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
       }
 #pragma unroll
       for (int n = 0; n < kNT; ++n) {
-        const int d = n * 8 + 2 * tig;
-        *reinterpret_cast<float2*>(scr + g * D + d) = make_float2(acc[n][0], acc[n][1]);
-        *reinterpret_cast<float2*>(scr + (g + 8) * D + d) = make_float2(acc[n][2], acc[n][3]);
+        if constexpr (kE4M3) {  // n-tile n: chunk n / 2, dims of parity n % 2
+          const int d = 16 * (n >> 1) + 4 * tig + (n & 1);
+          scr[g * D + d] = acc[n][0];
+          scr[g * D + d + 2] = acc[n][1];
+          scr[(g + 8) * D + d] = acc[n][2];
+          scr[(g + 8) * D + d + 2] = acc[n][3];
+        } else {
+          const int d = n * 8 + 2 * tig;
+          *reinterpret_cast<float2*>(scr + g * D + d) = make_float2(acc[n][0], acc[n][1]);
+          *reinterpret_cast<float2*>(scr + (g + 8) * D + d) = make_float2(acc[n][2], acc[n][3]);
+        }
       }
       if (tig == 0) {
         scr[kRows * D + g] = m_run[0];
@@ -341,16 +470,35 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
       // ================= own range: the member's heads as N = 8 ==========
       // (the decode kernel's form: S^T = K Q^T, P^T by movmatrix, O^T += V^T P^T)
       constexpr int kDT = D / 16;
-      const int own_ctx = s_ctx[member];
       uint32_t qf[kDT][2];
+      float sl2c[2] = {a.sl2, a.sl2};  // softmax scale of heads 2tig, 2tig + 1
       {
         const bool hv = g < G;
         const uint16_t* qrow = reinterpret_cast<const uint16_t*>(a.q) +
                                (static_cast<int64_t>(own_seq) * a.hq + kvh * G + (hv ? g : 0)) * D;
+        if constexpr (kE4M3) {
+          uint2 qw[kDT];
+          float am = 0.f;
 #pragma unroll
-        for (int ks = 0; ks < kDT; ++ks) {
-          qf[ks][0] = hv ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * tig) : 0u;
-          qf[ks][1] = hv ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * tig) : 0u;
+          for (int ks = 0; ks < kDT; ++ks) {
+            qw[ks] = hv ? *reinterpret_cast<const uint2*>(qrow + ks * 16 + 4 * tig) : make_uint2(0u, 0u);
+            am = fmaxf(am, amax4<kQBF16>(qw[ks]));
+          }
+          const int e = q_row_exponent(am);
+          const float dn = pow2f(-e);
+#pragma unroll
+          for (int ks = 0; ks < kDT; ++ks) {
+            qf[ks][0] = pack_f16x2(to_float<kQBF16>(qw[ks].x & 0xffff) * dn, to_float<kQBF16>(qw[ks].x >> 16) * dn);
+            qf[ks][1] = pack_f16x2(to_float<kQBF16>(qw[ks].y & 0xffff) * dn, to_float<kQBF16>(qw[ks].y >> 16) * dn);
+          }
+          sl2c[0] = a.sl2 * pow2f(__shfl_sync(0xffffffffu, e, 8 * tig));
+          sl2c[1] = a.sl2 * pow2f(__shfl_sync(0xffffffffu, e, 8 * tig + 4));
+        } else {
+#pragma unroll
+          for (int ks = 0; ks < kDT; ++ks) {
+            qf[ks][0] = hv ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 2 * tig) : 0u;
+            qf[ks][1] = hv ? *reinterpret_cast<const uint32_t*>(qrow + ks * 16 + 8 + 2 * tig) : 0u;
+          }
         }
       }
       float acc[kDT][4];
@@ -373,61 +521,89 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
           for (int mt = 0; mt < BS / 16; ++mt) {
             float s0[4] = {0.f, 0.f, 0.f, 0.f}, s1[4] = {0.f, 0.f, 0.f, 0.f};
             float s2[4] = {0.f, 0.f, 0.f, 0.f}, s3[4] = {0.f, 0.f, 0.f, 0.f};
-            const int row = mt * 16 + (lane & 7) + (li & 1) * 8;
+            if constexpr (kE4M3) {
+              const int tok = mt * 16 + (lane & 7) + (li & 1) * 8;
 #pragma unroll
-            for (int ks = 0; ks < kDT; ++ks) {
-              uint32_t af[4];
-              ldsm_x4(sK + tile_off<C>(row, (ks * 16 + (li >> 1) * 8) * 2), af[0], af[1], af[2],
-                      af[3]);
-              if ((ks & 3) == 0) mma_16816<kBF16>(s0, af, qf[ks][0], qf[ks][1]);
-              else if ((ks & 3) == 1) mma_16816<kBF16>(s1, af, qf[ks][0], qf[ks][1]);
-              else if ((ks & 3) == 2) mma_16816<kBF16>(s2, af, qf[ks][0], qf[ks][1]);
-              else mma_16816<kBF16>(s3, af, qf[ks][0], qf[ks][1]);
+              for (int cp = 0; cp < kDT / 2; ++cp) {
+                uint32_t r0, r1, r2, r3;
+                ldsm_x4(sK + tile_off<C>(tok, (2 * cp + (li >> 1)) * 16), r0, r1, r2, r3);
+                const uint32_t a0[4] = {e4m3x2_to_f16x2(r0 & 0xffff), e4m3x2_to_f16x2(r1 & 0xffff),
+                                        e4m3x2_to_f16x2(r0 >> 16), e4m3x2_to_f16x2(r1 >> 16)};
+                const uint32_t a1[4] = {e4m3x2_to_f16x2(r2 & 0xffff), e4m3x2_to_f16x2(r3 & 0xffff),
+                                        e4m3x2_to_f16x2(r2 >> 16), e4m3x2_to_f16x2(r3 >> 16)};
+                if (cp & 1) {
+                  mma_16816<false>(s2, a0, qf[2 * cp][0], qf[2 * cp][1]);
+                  mma_16816<false>(s3, a1, qf[2 * cp + 1][0], qf[2 * cp + 1][1]);
+                } else {
+                  mma_16816<false>(s0, a0, qf[2 * cp][0], qf[2 * cp][1]);
+                  mma_16816<false>(s1, a1, qf[2 * cp + 1][0], qf[2 * cp + 1][1]);
+                }
+              }
+            } else {
+              const int row = mt * 16 + (lane & 7) + (li & 1) * 8;
+#pragma unroll
+              for (int ks = 0; ks < kDT; ++ks) {
+                uint32_t af[4];
+                ldsm_x4(sK + tile_off<C>(row, (ks * 16 + (li >> 1) * 8) * 2), af[0], af[1], af[2],
+                        af[3]);
+                if ((ks & 3) == 0) mma_16816<kMmaBF16>(s0, af, qf[ks][0], qf[ks][1]);
+                else if ((ks & 3) == 1) mma_16816<kMmaBF16>(s1, af, qf[ks][0], qf[ks][1]);
+                else if ((ks & 3) == 2) mma_16816<kMmaBF16>(s2, af, qf[ks][0], qf[ks][1]);
+                else mma_16816<kMmaBF16>(s3, af, qf[ks][0], qf[ks][1]);
+              }
             }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int tok = mt * 16 + g + (e >> 1) * 8;
-              const float x = ((s0[e] + s1[e]) + (s2[e] + s3[e])) * a.sl2;
+              const float x = ((s0[e] + s1[e]) + (s2[e] + s3[e])) * sl2c[e & 1];
               s[mt][e] = tok < valid ? x : -INFINITY;
             }
           }
-          // online softmax per head column (every block has a valid token)
-          float alpha[2];
+          // online softmax per head column (every block has a valid token),
+          // the running max raised only past kRescaleLog2
+          float alpha[2] = {1.f, 1.f};
+          bool resc = false;
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             float bm = -INFINITY;
 #pragma unroll
-            for (int mt = 0; mt < BS / 16; ++mt) bm = fmaxf(bm, fmaxf(s[mt][c], s[mt][2 + c]));
+            for (int mt = 0; mt < BS / 16; ++mt) bm = fmax3(bm, s[mt][c], s[mt][2 + c]);
             bm = shfl_xor_max(bm);
-            const float mn = fmaxf(m_run[c], bm);
-            alpha[c] = fast_exp2(m_run[c] - mn);
-            m_run[c] = mn;
+            if (m_run[c] == -INFINITY) {
+              m_run[c] = bm;
+            } else if (bm - m_run[c] > kRescaleLog2) {
+              alpha[c] = fast_exp2(m_run[c] - bm);
+              m_run[c] = bm;
+              resc = true;
+            }
             float ps = 0.f;
 #pragma unroll
             for (int mt = 0; mt < BS / 16; ++mt) {
-              s[mt][c] = fast_exp2(s[mt][c] - mn);
-              s[mt][2 + c] = fast_exp2(s[mt][2 + c] - mn);
+              s[mt][c] = fast_exp2(s[mt][c] - m_run[c]);
+              s[mt][2 + c] = fast_exp2(s[mt][2 + c] - m_run[c]);
               ps += s[mt][c] + s[mt][2 + c];
             }
             l_run[c] = l_run[c] * alpha[c] + ps;
           }
+          if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll
-          for (int dt = 0; dt < kDT; ++dt) {
-            acc[dt][0] *= alpha[0];
-            acc[dt][1] *= alpha[1];
-            acc[dt][2] *= alpha[0];
-            acc[dt][3] *= alpha[1];
+            for (int dt = 0; dt < kDT; ++dt) {
+              acc[dt][0] *= alpha[0];
+              acc[dt][1] *= alpha[1];
+              acc[dt][2] *= alpha[0];
+              acc[dt][3] *= alpha[1];
+            }
           }
           // P^T as the B operand (8x8 (token, head) tiles transposed in
           // registers); bf16 keeps hi + lo parts
           uint32_t pb[BS / 16][2], pl[BS / 16][2];
 #pragma unroll
           for (int mt = 0; mt < BS / 16; ++mt) {
-            const uint32_t h0 = pack2<kBF16>(s[mt][0], s[mt][1]);
-            const uint32_t h1 = pack2<kBF16>(s[mt][2], s[mt][3]);
+            const uint32_t h0 = pack2<kMmaBF16>(s[mt][0], s[mt][1]);
+            const uint32_t h1 = pack2<kMmaBF16>(s[mt][2], s[mt][3]);
             pb[mt][0] = movmatrix_trans(h0);
             pb[mt][1] = movmatrix_trans(h1);
-            if constexpr (kBF16) {
+            if constexpr (kPBF16) {
               pl[mt][0] = movmatrix_trans(pack_bf16x2(s[mt][0] - to_float<true>(h0 & 0xffff),
                                                       s[mt][1] - to_float<true>(h0 >> 16)));
               pl[mt][1] = movmatrix_trans(pack_bf16x2(s[mt][2] - to_float<true>(h1 & 0xffff),
@@ -436,23 +612,47 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
           }
           // O^T += V^T P^T; in the member's last block the value rows past its
           // length are zeroed in the fragments (they may hold anything)
+          const bool part = valid < BS;
 #pragma unroll
           for (int mt = 0; mt < BS / 16; ++mt) {
             uint32_t m_lo = 0xffffffffu, m_hi = 0xffffffffu;  // tokens 2tig(+1), 2tig+8(+9)
-            if (valid < BS) {
+            if (part) {
               const int tk = mt * 16 + 2 * tig;
               m_lo = pair_mask(tk < valid, tk + 1 < valid);
               m_hi = pair_mask(tk + 8 < valid, tk + 9 < valid);
             }
-            const int tok = mt * 16 + (lane & 7) + (li >> 1) * 8;
+            if constexpr (kE4M3) {
+              const int tok = mt * 16 + (lane & 7) + (li & 1) * 8;
 #pragma unroll
-            for (int dt = 0; dt < kDT; ++dt) {
-              uint32_t af[4];
-              ldsm_x4_trans(sV + tile_off<C>(tok, (dt * 16 + (li & 1) * 8) * 2), af[0], af[1],
-                            af[2], af[3]);
-              af[0] &= m_lo; af[1] &= m_lo; af[2] &= m_hi; af[3] &= m_hi;
-              mma_16816<kBF16>(acc[dt], af, pb[mt][0], pb[mt][1]);
-              if constexpr (kBF16) mma_16816<kBF16>(acc[dt], af, pl[mt][0], pl[mt][1]);
+              for (int cp = 0; cp < kDT / 2; ++cp) {
+                uint32_t r0, r1, r2, r3;
+                ldsm_x4_trans(sV + tile_off<C>(tok, (2 * cp + (li >> 1)) * 16), r0, r1, r2, r3);
+                if (part) {
+                  r0 &= m_lo; r1 &= m_hi; r2 &= m_lo; r3 &= m_hi;
+                }
+                // bytes (tok 2tig: dim 2g, 2g+1 | tok 2tig+1: dim 2g, 2g+1) -> pairs per dim
+                const uint32_t p0 = __byte_perm(r0, 0, 0x3120), p1 = __byte_perm(r1, 0, 0x3120);
+                const uint32_t p2 = __byte_perm(r2, 0, 0x3120), p3 = __byte_perm(r3, 0, 0x3120);
+                const uint32_t a0[4] = {e4m3x2_to_f16x2(p0 & 0xffff), e4m3x2_to_f16x2(p0 >> 16),
+                                        e4m3x2_to_f16x2(p1 & 0xffff), e4m3x2_to_f16x2(p1 >> 16)};
+                const uint32_t a1[4] = {e4m3x2_to_f16x2(p2 & 0xffff), e4m3x2_to_f16x2(p2 >> 16),
+                                        e4m3x2_to_f16x2(p3 & 0xffff), e4m3x2_to_f16x2(p3 >> 16)};
+                mma_16816<false>(acc[2 * cp], a0, pb[mt][0], pb[mt][1]);
+                mma_16816<false>(acc[2 * cp + 1], a1, pb[mt][0], pb[mt][1]);
+              }
+            } else {
+              const int tok = mt * 16 + (lane & 7) + (li >> 1) * 8;
+#pragma unroll
+              for (int dt = 0; dt < kDT; ++dt) {
+                uint32_t af[4];
+                ldsm_x4_trans(sV + tile_off<C>(tok, (dt * 16 + (li & 1) * 8) * 2), af[0], af[1],
+                              af[2], af[3]);
+                if (part) {
+                  af[0] &= m_lo; af[1] &= m_lo; af[2] &= m_hi; af[3] &= m_hi;
+                }
+                mma_16816<kMmaBF16>(acc[dt], af, pb[mt][0], pb[mt][1]);
+                if constexpr (kPBF16) mma_16816<kMmaBF16>(acc[dt], af, pl[mt][0], pl[mt][1]);
+              }
             }
           }
         }
@@ -463,7 +663,9 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
       const float lsum1 = shfl_xor_sum(l_run[1]);
 #pragma unroll
       for (int dt = 0; dt < kDT; ++dt) {
-        const int dlo = dt * 16 + g, dhi = dlo + 8;
+        // C fragment rows: 16-bit path dims 16dt + g (+8); 8-bit path 16dt + 2g (+1)
+        const int dlo = kE4M3 ? dt * 16 + 2 * g : dt * 16 + g;
+        const int dhi = kE4M3 ? dlo + 1 : dlo + 8;
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           const int h = 2 * tig + c;
@@ -480,11 +682,12 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
     }
     __syncthreads();
     {
-      // combine the 4 warps; a shared range covers the chunk's rows 0..rows-1
-      // (scratch: O [16][D], max at 16 D, sums at 16 D + 16), an own range the
-      // member's G rows (scratch: O [8][D], max at 8 D, sums at 8 D + 8)
+      // combine the 4 warps; the 16-row form covers rows 0..nrow-1 of its
+      // tile (scratch: O [16][D], max at 16 D, sums at 16 D + 16), the
+      // 8-column form the member's G rows (scratch: O [8][D], max at 8 D,
+      // sums at 8 D + 8)
       const int nrow = shared ? rows : G;
-      const int mrow = shared ? kRows : 8;
+      const int mrow = rowform ? kRows : 8;
       constexpr int kVec = 8;
       const int units = nrow * (D / kVec);
       for (int u = threadIdx.x; u < units; u += kDecodeThreads) {
@@ -513,7 +716,7 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
             o[0] += f * x0.x; o[1] += f * x0.y; o[2] += f * x0.z; o[3] += f * x0.w;
             o[4] += f * x1.x; o[5] += f * x1.y; o[6] += f * x1.z; o[7] += f * x1.w;
           }
-          const float inv = 1.f / L;
+          const float inv = a.out_scale / L;
 #pragma unroll
           for (int v = 0; v < kVec; ++v) o[v] *= inv;
         }
@@ -521,10 +724,10 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
         if (nranges == 1) {
           const int64_t qh = static_cast<int64_t>(s_seq[r / G]) * a.hq + kvh * G + r % G;
           uint4 pk;
-          pk.x = pack2<kBF16>(o[0], o[1]);
-          pk.y = pack2<kBF16>(o[2], o[3]);
-          pk.z = pack2<kBF16>(o[4], o[5]);
-          pk.w = pack2<kBF16>(o[6], o[7]);
+          pk.x = pack2<kQBF16>(o[0], o[1]);
+          pk.y = pack2<kQBF16>(o[2], o[3]);
+          pk.z = pack2<kQBF16>(o[4], o[5]);
+          pk.w = pack2<kQBF16>(o[6], o[7]);
           *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.out) + qh * D + d0) = pk;
         } else {
           const int64_t pi = (static_cast<int64_t>(slot) * a.hkv + kvh) * kRows + r;
@@ -598,8 +801,8 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
           const float inv = W > 0.f ? 1.f / W : 0.f;
           const int64_t qh = static_cast<int64_t>(s_seq[r / G]) * a.hq + kvh * G + r % G;
           uint2 pk;
-          pk.x = pack2<kBF16>(o0 * inv, o1 * inv);
-          pk.y = pack2<kBF16>(o2 * inv, o3 * inv);
+          pk.x = pack2<kQBF16>(o0 * inv, o1 * inv);
+          pk.y = pack2<kQBF16>(o2 * inv, o3 * inv);
           *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.out) + qh * D + d0) = pk;
         }
       }

@@ -22,8 +22,21 @@ __device__ __forceinline__ void record_error(int code) {
   atomicCAS(&g_device_error, 0, code);
 }
 
-// A wait on an asynchronous copy gives up after this many nanoseconds.
-constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;
+// A wait on an asynchronous copy gives up after this many nanoseconds (one
+// second; a test build may shorten it).
+#ifndef PA_WAIT_LIMIT_NS
+#define PA_WAIT_LIMIT_NS (1000ull * 1000ull * 1000ull)
+#endif
+constexpr unsigned long long kWaitLimitNs = PA_WAIT_LIMIT_NS;
+
+// Test builds only: extra bytes every decode stage barrier expects beyond
+// its two tile copies.  With a non-zero value no stage ever completes while
+// every copy stays a valid, in-bounds load that lands, so the decode
+// kernel's bounded waits run out and its give-up path (record the timeout,
+// stop issuing, drain) runs.  The library build leaves it 0.
+#ifndef PA_TEST_STAGE_EXTRA_TX
+#define PA_TEST_STAGE_EXTRA_TX 0
+#endif
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

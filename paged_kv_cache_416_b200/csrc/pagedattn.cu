@@ -13,6 +13,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "prefill.cuh"
+#include "prefill_pp.cuh"
 #include "cascade.cuh"
 
 namespace {
@@ -280,11 +281,11 @@ pa_status dispatch_shape(const pa::DecodeArgs& a, int D, int BS, int64_t items, 
   return fail(PA_ERR_SHAPE, "head_dim %d / block_size %d not supported", D, BS);
 }
 
-template <bool kBF16, int D, int BS>
+template <int CK, bool kQBF16, int D, int BS>
 pa_status launch_cascade(const pa::CascadeArgs& args, int64_t items_upper, int dev,
                          cudaStream_t stream) {
-  using C = pa::DecodeCfg<kBF16 ? pa::kCacheBF16 : pa::kCacheF16, D, BS>;
-  auto kern = pa::cascade_kernel<kBF16, D, BS>;
+  using C = pa::DecodeCfg<CK, D, BS>;
+  auto kern = pa::cascade_kernel<CK, kQBF16, D, BS>;
   static std::atomic<int> occ[kMaxDevices] = {};
   int per_sm = 0;
   const pa_status os = resident_ctas(occ, dev, kern, pa::kDecodeThreads, C::kSmemBytes,
@@ -298,13 +299,13 @@ pa_status launch_cascade(const pa::CascadeArgs& args, int64_t items_upper, int d
   return PA_OK;
 }
 
-template <bool kBF16>
+template <int CK, bool kQBF16>
 pa_status dispatch_cascade(const pa::CascadeArgs& a, int D, int BS, int64_t items, int dev,
                            cudaStream_t st) {
-  if (D == 128 && BS == 16) return launch_cascade<kBF16, 128, 16>(a, items, dev, st);
-  if (D == 128 && BS == 32) return launch_cascade<kBF16, 128, 32>(a, items, dev, st);
-  if (D == 64 && BS == 16) return launch_cascade<kBF16, 64, 16>(a, items, dev, st);
-  if (D == 64 && BS == 32) return launch_cascade<kBF16, 64, 32>(a, items, dev, st);
+  if (D == 128 && BS == 16) return launch_cascade<CK, kQBF16, 128, 16>(a, items, dev, st);
+  if (D == 128 && BS == 32) return launch_cascade<CK, kQBF16, 128, 32>(a, items, dev, st);
+  if (D == 64 && BS == 16) return launch_cascade<CK, kQBF16, 64, 16>(a, items, dev, st);
+  if (D == 64 && BS == 32) return launch_cascade<CK, kQBF16, 64, 32>(a, items, dev, st);
   return fail(PA_ERR_SHAPE, "head_dim %d / block_size %d not supported", D, BS);
 }
 
@@ -583,12 +584,14 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype q_dtype, co
                                   const int32_t* group_start, const int32_t* group_seqs,
                                   int32_t num_groups, int32_t num_seqs, int32_t num_q_heads,
                                   int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
-                                  int32_t num_blocks, float scale, int32_t split_tokens,
-                                  void* workspace, size_t workspace_bytes, pa_stream_t stream) {
+                                  int32_t num_blocks, float scale, float k_scale, float v_scale,
+                                  int32_t split_tokens, void* workspace, size_t workspace_bytes,
+                                  pa_stream_t stream) {
   if (!valid_dtype(q_dtype) || !valid_dtype(cache_dtype))
     return fail(PA_ERR_DTYPE, "pa_decode_shared_prefix: unknown dtype");
-  if (cache_dtype == PA_FP8_E4M3 || q_dtype != cache_dtype)
-    return fail(PA_ERR_DTYPE, "pa_decode_shared_prefix: q and cache must both be f16 or both bf16");
+  const bool fp8 = cache_dtype == PA_FP8_E4M3;
+  if (q_dtype == PA_FP8_E4M3 || (!fp8 && q_dtype != cache_dtype))
+    return fail(PA_ERR_DTYPE, "pa_decode_shared_prefix: q must be f16/bf16 and match a 16-bit cache");
   if (num_seqs < 0 || num_groups < 0 || max_blocks_per_seq <= 0 || max_context_len < 0 ||
       split_tokens < 0 || !cache_shape_ok(num_blocks, block_size, num_kv_heads, head_dim))
     return fail(PA_ERR_SHAPE, "pa_decode_shared_prefix: unsupported sizes (seqs %d, groups %d, "
@@ -599,11 +602,13 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype q_dtype, co
     return fail(PA_ERR_SHAPE, "pa_decode_shared_prefix: max_context_len %d exceeds "
                 "max_blocks_per_seq * bs", max_context_len);
   if (num_q_heads <= 0 || num_q_heads % num_kv_heads != 0 ||
-      num_q_heads / num_kv_heads > pa::kMaxGroup)
+      num_q_heads / num_kv_heads > pa::kCascadeRows)
     return fail(PA_ERR_HEADS, "pa_decode_shared_prefix: num_q_heads %d must be a multiple of "
                 "num_kv_heads %d with at most %d query heads per kv head", num_q_heads,
-                num_kv_heads, pa::kMaxGroup);
-  if (!std::isfinite(scale)) return fail(PA_ERR_SHAPE, "pa_decode_shared_prefix: scale must be finite");
+                num_kv_heads, pa::kCascadeRows);
+  if (!std::isfinite(scale) || (fp8 && !(std::isfinite(k_scale) && k_scale > 0.f &&
+                                         std::isfinite(v_scale) && v_scale > 0.f)))
+    return fail(PA_ERR_SHAPE, "pa_decode_shared_prefix: scales must be finite (and positive for e4m3)");
   if (num_seqs == 0) return ok();
   if (!out || !q || !k_pool || !v_pool || !block_tables || !context_lens ||
       (num_groups > 0 && (!group_start || !group_seqs)))
@@ -644,7 +649,8 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype q_dtype, co
   a.group = num_q_heads / num_kv_heads;
   a.max_blocks = max_blocks_per_seq;
   a.num_blocks = num_blocks;
-  a.sl2 = scale * 1.4426950408889634f;
+  a.sl2 = scale * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
+  a.out_scale = fp8 ? v_scale : 1.f;
 
   pa::cascade_plan_kernel<<<1, 1024, 0, st>>>(
       context_lens, block_tables, group_start, group_seqs, num_groups, num_seqs, max_context_len,
@@ -653,9 +659,15 @@ pa_status pa_decode_shared_prefix(void* out, const void* q, pa_dtype q_dtype, co
       reinterpret_cast<int4*>(ws + w.chunks), reinterpret_cast<int4*>(ws + w.ranges),
       reinterpret_cast<int32_t*>(ws + w.total), a.counter, a.arrived);
   const int64_t items_upper = w.slots * num_kv_heads;
-  const pa_status s = cache_dtype == PA_BF16
-                          ? dispatch_cascade<true>(a, head_dim, block_size, items_upper, dev, st)
-                          : dispatch_cascade<false>(a, head_dim, block_size, items_upper, dev, st);
+  pa_status s;
+  if (cache_dtype == PA_F16)
+    s = dispatch_cascade<pa::kCacheF16, false>(a, head_dim, block_size, items_upper, dev, st);
+  else if (cache_dtype == PA_BF16)
+    s = dispatch_cascade<pa::kCacheBF16, true>(a, head_dim, block_size, items_upper, dev, st);
+  else if (q_dtype == PA_BF16)
+    s = dispatch_cascade<pa::kCacheE4M3, true>(a, head_dim, block_size, items_upper, dev, st);
+  else
+    s = dispatch_cascade<pa::kCacheE4M3, false>(a, head_dim, block_size, items_upper, dev, st);
   if (s != PA_OK) return s;
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "pa_decode_shared_prefix launch");
@@ -710,8 +722,9 @@ pa_status pa_prefill(void* out, const void* q, pa_dtype q_dtype, const void* k_p
   a.num_blocks = num_blocks;
   a.max_ctx = max_context_len;
   a.sl2 = scale * 1.4426950408889634f;
+  // a CTA takes two query tiles of T = 128 / G tokens each
   const int T = pa::kPfRows / a.group;
-  dim3 grid(static_cast<unsigned>(cdiv(max_query_len, T)), static_cast<unsigned>(num_kv_heads),
+  dim3 grid(static_cast<unsigned>(cdiv(max_query_len, 2 * T)), static_cast<unsigned>(num_kv_heads),
             static_cast<unsigned>(num_seqs));
   if (grid.y > 65535 || grid.z > 65535)
     return fail(PA_ERR_SHAPE, "pa_prefill: too many kv heads or sequences for one launch");
@@ -719,14 +732,14 @@ pa_status pa_prefill(void* out, const void* q, pa_dtype q_dtype, const void* k_p
   auto launch = [&](auto kern, int smem_bytes) -> pa_status {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill)");
-    kern<<<grid, pa::kPfThreads, smem_bytes, st>>>(a);
+    kern<<<grid, pa::kPpThreads, smem_bytes, st>>>(a);
     return PA_OK;
   };
   pa_status ls;
   const bool bf = q_dtype == PA_BF16;
-#define PA_PF_LAUNCH(BS_, D_)                                                              \
-  (bf ? launch(pa::prefill_kernel<true, BS_, D_>, pa::PrefillCfg<BS_, D_>::kSmemBytes)     \
-      : launch(pa::prefill_kernel<false, BS_, D_>, pa::PrefillCfg<BS_, D_>::kSmemBytes))
+#define PA_PF_LAUNCH(BS_, D_)                                                                 \
+  (bf ? launch(pa::prefill_pp_kernel<true, BS_, D_>, pa::PrefillPpCfg<BS_, D_>::kSmemBytes)   \
+      : launch(pa::prefill_pp_kernel<false, BS_, D_>, pa::PrefillPpCfg<BS_, D_>::kSmemBytes))
   if (head_dim == 64)
     ls = block_size == 16 ? PA_PF_LAUNCH(16, 64) : PA_PF_LAUNCH(32, 64);
   else

@@ -58,7 +58,7 @@ def declare(lib: ctypes.CDLL) -> ctypes.CDLL:
                             F, F, F, I32, P, SZ, P]),
         "pa_decode_shared_prefix_workspace_size": (SZ, [I32, I32, I32, I32, I32, I32, I32]),
         "pa_decode_shared_prefix": (I32, [P, P, I32, P, P, I32, P, I32, P, I32, P, P, I32, I32,
-                                          I32, I32, I32, I32, I32, F, I32, P, SZ, P]),
+                                          I32, I32, I32, I32, I32, F, F, F, I32, P, SZ, P]),
         "pa_sync_status": (I32, [P]),
         "pa_last_error": (ctypes.c_char_p, []),
         "pa_validate_slot_mapping": (I32, [P, I32, I32, I32, P]),
@@ -275,11 +275,12 @@ def shared_prefix_workspace_size(num_seqs, hq, hkv, head_dim, bs, max_context_le
 
 
 def decode_shared_prefix(q, k_pool, v_pool, block_tables, context_lens, group_start, group_seqs,
-                         scale: float, max_context_len: int, split_tokens: int = 0, out=None,
+                         scale: float, max_context_len: int, k_scale: float = 1.0,
+                         v_scale: float = 1.0, split_tokens: int = 0, out=None,
                          workspace=None, stream=None) -> torch.Tensor:
     """pa_decode_shared_prefix on tensors: pa_decode's arguments plus the
-    groups (group_start int32 [G + 1], group_seqs int32 [group_start[G]]),
-    16-bit caches.  Returns out [B, Hq, D]."""
+    groups (group_start int32 [G + 1], group_seqs int32 [group_start[G]]).
+    Returns out [B, Hq, D]."""
     _contig(q, k_pool, v_pool, block_tables, context_lens, group_start, group_seqs)
     for t in (block_tables, context_lens, group_start, group_seqs):
         if t.dtype != torch.int32:
@@ -295,7 +296,8 @@ def decode_shared_prefix(q, k_pool, v_pool, block_tables, context_lens, group_st
         _ptr(out), _ptr(q), _dtype(q), _ptr(k_pool), _ptr(v_pool), _dtype(k_pool),
         _ptr(block_tables), block_tables.shape[1], _ptr(context_lens), int(max_context_len),
         _ptr(group_start), _ptr(group_seqs), group_start.shape[0] - 1, B, hq, hkv, d, bs, N,
-        float(scale), int(split_tokens), _ptr(workspace), workspace.numel(), _stream(stream)))
+        float(scale), float(k_scale), float(v_scale), int(split_tokens), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
     return out
 
 

@@ -274,8 +274,10 @@ def _lens_shared_prefix(phase, seed, prompts=32, samples=4, prefix=1024, max_tai
 
 
 def _shared_prefix(phase, seed, device, prompts=32, samples=4, prefix=1024,
-                   max_tail=512, hq=32, hkv=8, d=128, bs=16) -> Workload:
-    """Parallel sampling over a shared prompt (see the module docstring)."""
+                   max_tail=512, hq=32, hkv=8, d=128, bs=16, cache="bf16") -> Workload:
+    """Parallel sampling over a shared prompt (see the module docstring);
+    queries and new tokens bf16, the cache bf16 or e4m3 (per-tensor scales
+    from the prompt's values, later tokens quantised with the same scales)."""
     rng, plen, tails = _shared_prefix_draws(seed, prompts, samples, prefix, max_tail, bs)
     B = prompts * samples
     # pool: shared prompt blocks once, plus every sample's own blocks
@@ -304,8 +306,8 @@ def _shared_prefix(phase, seed, device, prompts=32, samples=4, prefix=1024,
             if cow is not None:
                 pairs.append(cow)
     pairs = np.asarray(pairs, dtype=np.int64).reshape(-1, 2)
-    k_pool, k_scale = _fill_pool(num_blocks, bs, hkv, d, "bf16", prompt_valid, gen, device)
-    v_pool, v_scale = _fill_pool(num_blocks, bs, hkv, d, "bf16", prompt_valid, gen, device)
+    k_pool, k_scale = _fill_pool(num_blocks, bs, hkv, d, cache, prompt_valid, gen, device)
+    v_pool, v_scale = _fill_pool(num_blocks, bs, hkv, d, cache, prompt_valid, gen, device)
     q = _to_storage(_randn((B, hq, d), gen, device), "bf16")
     first_k = _to_storage(_randn((B, hkv, d), gen, device), "bf16")
     first_v = _to_storage(_randn((B, hkv, d), gen, device), "bf16")
@@ -315,8 +317,8 @@ def _shared_prefix(phase, seed, device, prompts=32, samples=4, prefix=1024,
         tables = alloc.table_array(list(range(B)))
         return Workload(
             name="shared_prefix_fork", num_seqs=B, num_q_heads=hq, num_kv_heads=hkv, head_dim=d,
-            block_size=bs, q_dtype="bf16", cache_dtype="bf16", num_blocks=num_blocks,
-            scale=1.0 / math.sqrt(d), k_scale=1.0, v_scale=1.0, context_lens=lens,
+            block_size=bs, q_dtype="bf16", cache_dtype=cache, num_blocks=num_blocks,
+            scale=1.0 / math.sqrt(d), k_scale=k_scale, v_scale=v_scale, context_lens=lens,
             block_tables=tables, q=q, k_pool=k_pool, v_pool=v_pool, new_k=first_k, new_v=first_v,
             slot_mapping=np.asarray(first_slots, dtype=np.int64), cow_pairs=pairs,
             meta={"seed": int(seed), "allocator": alloc, "prompt_lens": plen, "samples": samples,
@@ -331,8 +333,8 @@ def _shared_prefix(phase, seed, device, prompts=32, samples=4, prefix=1024,
         k_pool[dst] = k_pool[src]
         v_pool[dst] = v_pool[src]
     fs = torch.from_numpy(np.asarray(first_slots, dtype=np.int64)).to(device)
-    k_pool.view(-1, hkv, d)[fs] = first_k
-    v_pool.view(-1, hkv, d)[fs] = first_v
+    k_pool.view(-1, hkv, d)[fs] = _to_storage(first_k.float(), cache, k_scale)
+    v_pool.view(-1, hkv, d)[fs] = _to_storage(first_v.float(), cache, v_scale)
     tail_slots = []
     for p in range(prompts):
         for i in range(samples):
@@ -343,8 +345,8 @@ def _shared_prefix(phase, seed, device, prompts=32, samples=4, prefix=1024,
     if tail_slots:
         ts = torch.from_numpy(np.asarray(tail_slots, dtype=np.int64)).to(device)
         n = len(tail_slots)
-        k_pool.view(-1, hkv, d)[ts] = _to_storage(_randn((n, hkv, d), gen, device), "bf16")
-        v_pool.view(-1, hkv, d)[ts] = _to_storage(_randn((n, hkv, d), gen, device), "bf16")
+        k_pool.view(-1, hkv, d)[ts] = _to_storage(_randn((n, hkv, d), gen, device), cache, k_scale)
+        v_pool.view(-1, hkv, d)[ts] = _to_storage(_randn((n, hkv, d), gen, device), cache, v_scale)
     step_slots = []
     for p in range(prompts):
         for i in range(samples):
@@ -358,8 +360,8 @@ def _shared_prefix(phase, seed, device, prompts=32, samples=4, prefix=1024,
     new_v = _to_storage(_randn((B, hkv, d), gen, device), "bf16")
     return Workload(
         name="shared_prefix_tails", num_seqs=B, num_q_heads=hq, num_kv_heads=hkv, head_dim=d,
-        block_size=bs, q_dtype="bf16", cache_dtype="bf16", num_blocks=num_blocks,
-        scale=1.0 / math.sqrt(d), k_scale=1.0, v_scale=1.0, context_lens=lens,
+        block_size=bs, q_dtype="bf16", cache_dtype=cache, num_blocks=num_blocks,
+        scale=1.0 / math.sqrt(d), k_scale=k_scale, v_scale=v_scale, context_lens=lens,
         block_tables=tables, q=q, k_pool=k_pool, v_pool=v_pool, new_k=new_k, new_v=new_v,
         slot_mapping=np.asarray(step_slots, dtype=np.int64), cow_pairs=np.zeros((0, 2), np.int64),
         meta={"seed": int(seed), "allocator": alloc, "prompt_lens": plen, "tails": tails,
@@ -418,6 +420,11 @@ _SHAPES = {"tiny": (4, 64, 2), "llama13b_mha": (40, 128, 2), "llama70b_gqa": (8,
            "fp8_longtail_bs16": (8, 128, 1), "fp8_longtail_bs32": (8, 128, 1)}
 _DEFAULT_SEEDS = {"tiny": 1, "llama13b_mha": 2, "llama70b_gqa": 3, "shared_prefix_fork": 4,
                   "shared_prefix_tails": 4, "fp8_longtail_bs16": 5, "fp8_longtail_bs32": 5}
+
+
+def default_seed(name: str) -> int:
+    """The seed of a workload's configuration (1..5, by configuration)."""
+    return _DEFAULT_SEEDS[name]
 
 
 def context_lens(name: str, seed: Optional[int] = None, **kw) -> np.ndarray:

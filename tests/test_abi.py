@@ -115,14 +115,17 @@ def _shared(pa, **kw):
     args = dict(out=None, q=None, q_dtype=1, k_pool=None, v_pool=None, cache_dtype=1,
                 block_tables=None, max_blocks=4, context_lens=None, max_ctx=64, group_start=None,
                 group_seqs=None, num_groups=1, B=2, hq=8, hkv=2, D=128, bs=16, N=32, scale=0.1,
-                split=0, ws=None, ws_bytes=0, stream=None)
+                k_scale=1.0, v_scale=1.0, split=0, ws=None, ws_bytes=0, stream=None)
     args.update(kw)
     return pa.pa_decode_shared_prefix(*args.values())
 
 
 @pytest.mark.parametrize("kw,status", [
-    (dict(q_dtype=2, cache_dtype=2), 2),         # no e4m3 cache on this path
+    (dict(q_dtype=2, cache_dtype=2), 2),         # an e4m3 query
     (dict(q_dtype=0, cache_dtype=1), 2),
+    (dict(cache_dtype=2, k_scale=0.0), 3),       # e4m3 cache with a bad scale
+    (dict(hq=34), 4),                            # 17 query heads per kv head
+    (dict(hq=32, cache_dtype=2), 1),             # 16 per kv head, e4m3: valid, nulls
     (dict(D=96), 3),
     (dict(num_groups=-1), 3),
     (dict(max_ctx=65), 3),

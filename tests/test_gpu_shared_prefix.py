@@ -25,7 +25,7 @@ def step_inputs(pa, w):
     if len(w.cow_pairs):
         pa.copy_blocks(kp, vp, torch.from_numpy(w.cow_pairs).cuda())
     pa.write_kv(w.new_k.cuda().contiguous(), w.new_v.cuda().contiguous(),
-                torch.from_numpy(w.slot_mapping).cuda(), kp, vp)
+                torch.from_numpy(w.slot_mapping).cuda(), kp, vp, w.k_scale, w.v_scale)
     return kp, vp
 
 
@@ -35,19 +35,20 @@ def run_shared(pa, w, kp, vp, group_start, group_seqs, split_tokens=0):
         torch.from_numpy(w.context_lens).cuda(),
         torch.from_numpy(np.asarray(group_start, np.int32)).cuda(),
         torch.from_numpy(np.asarray(group_seqs, np.int32)).cuda(), w.scale, w.max_context_len,
-        split_tokens=split_tokens)
+        k_scale=w.k_scale, v_scale=w.v_scale, split_tokens=split_tokens)
     return out
 
 
 def run_plain(pa, w, kp, vp, split_tokens=0):
     return pa.decode(w.q.cuda().contiguous(), kp, vp, torch.from_numpy(w.block_tables).cuda(),
                      torch.from_numpy(w.context_lens).cuda(), w.scale, w.max_context_len,
-                     split_tokens=split_tokens)
+                     k_scale=w.k_scale, v_scale=w.v_scale, split_tokens=split_tokens)
 
 
 def oracle_out(w, kp, vp, seqs=None):
     return oracle.decode(raw(w.q), w.q_dtype, raw(kp), raw(vp), w.cache_dtype, w.block_tables,
-                         w.context_lens, w.scale, w.num_kv_heads, seqs=seqs)
+                         w.context_lens, w.scale, w.num_kv_heads, w.k_scale, w.v_scale,
+                         seqs=seqs)
 
 
 def groups(w):
@@ -85,6 +86,39 @@ def test_shared_prefix_shapes(pa, hq, hkv, d, bs, dtype):
     out = run_shared(pa, w, kp, vp, *groups(w), split_tokens=96)
     pa.sync_status()
     assert_attention_close(as_f64(out), oracle_out(w, kp, vp), f"shared prefix {hq}/{hkv} D{d} bs{bs}")
+
+
+@pytest.mark.parametrize("phase", ["fork", "tails"])
+@pytest.mark.parametrize("hq,hkv,d,bs,split", [(32, 8, 128, 16, 0), (32, 8, 128, 16, 64),
+                                               (16, 4, 64, 32, 96), (64, 8, 128, 32, 0)])
+def test_shared_prefix_e4m3_cache(pa, phase, hq, hkv, d, bs, split):
+    """e4m3 caches (q bf16, per-tensor scales): the 16-row tiles and the
+    8-column form dequantise on load, against the oracle on the dequantised
+    cache and against plain decode."""
+    w = W._shared_prefix(phase, 12, "cpu", prompts=4, samples=4, prefix=288, max_tail=150,
+                         hq=hq, hkv=hkv, d=d, bs=bs, cache="e4m3")
+    kp, vp = step_inputs(pa, w)
+    out = run_shared(pa, w, kp, vp, *groups(w), split_tokens=split)
+    plain = run_plain(pa, w, kp, vp, split_tokens=split)
+    pa.sync_status()
+    ref = oracle_out(w, kp, vp)
+    assert_attention_close(as_f64(out), ref, f"e4m3 shared prefix {phase} {hq}/{hkv} D{d} bs{bs}")
+    assert_attention_close(as_f64(out), as_f64(plain), "e4m3 shared prefix vs plain decode")
+
+
+@pytest.mark.parametrize("hq,hkv,cache,split", [(64, 4, "bf16", 0), (64, 4, "bf16", 64),
+                                                (48, 4, "bf16", 0), (64, 4, "e4m3", 64),
+                                                (96, 8, "e4m3", 0)])
+def test_shared_prefix_more_than_eight_heads_per_kv_head(pa, hq, hkv, cache, split):
+    """12 and 16 query heads per kv head: a chunk is one member whose heads
+    fill the 16-row tile, for its shared and its own ranges."""
+    w = W._shared_prefix("tails", 13, "cpu", prompts=3, samples=3, prefix=200, max_tail=120,
+                         hq=hq, hkv=hkv, cache=cache)
+    kp, vp = step_inputs(pa, w)
+    out = run_shared(pa, w, kp, vp, *groups(w), split_tokens=split)
+    pa.sync_status()
+    assert_attention_close(as_f64(out), oracle_out(w, kp, vp),
+                           f"shared prefix {hq}/{hkv} {cache} split {split}")
 
 
 def test_ungrouped_and_unrelated_sequences_decode_plainly(pa):
