@@ -87,6 +87,12 @@ def parse_args(argv=None):
     ap.add_argument("--ingest-kernel", default="decode_kernel", choices=sorted(KERNEL_SOURCES))
     ap.add_argument("--ingest-command", default="",
                     help="the command line that produced the capture (recorded)")
+    ap.add_argument("--ingest-source-sha16", default=None,
+                    help="source hash of the kernel when it was captured (bench.py "
+                         "--print-source-sha16 on the capturing machine); must match the "
+                         "sources here, else nothing is recorded")
+    ap.add_argument("--print-source-sha16", action="store_true",
+                    help="print the decode and cascade kernels' source hashes and exit")
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--num-seqs", type=int, default=None,
                     help="override the workload's batch (smaller cases for profiling only)")
@@ -261,7 +267,8 @@ def profiled_traffic(workload: str, kernel: str = "decode_kernel"):
 
 
 _NCU_UNITS = {"byte": 1, "kbyte": 1e3, "mbyte": 1e6, "gbyte": 1e9, "tbyte": 1e12,
-              "nsecond": 1e-9, "usecond": 1e-6, "msecond": 1e-3, "second": 1.0}
+              "nsecond": 1e-9, "usecond": 1e-6, "msecond": 1e-3, "second": 1.0,
+              "ns": 1e-9, "us": 1e-6, "ms": 1e-3, "s": 1.0}
 
 
 def parse_ncu_csv(path: str, kernel: str):
@@ -284,6 +291,10 @@ def parse_ncu_csv(path: str, kernel: str):
 def ingest_ncu(args):
     """Record the DRAM traffic of one captured kernel launch per workload."""
     from paged_kv_cache_416_b200 import workloads as W
+    here = source_hash(args.ingest_kernel)
+    if args.ingest_source_sha16 is not None and args.ingest_source_sha16 != here:
+        raise SystemExit(f"the capture is of {args.ingest_kernel} source {args.ingest_source_sha16}, "
+                         f"the sources here hash {here}: not recorded")
     launches = parse_ncu_csv(args.ingest_ncu, args.ingest_kernel)
     if not launches:
         raise SystemExit(f"no {args.ingest_kernel} launch in {args.ingest_ncu}")
@@ -636,12 +647,19 @@ def measure_configs(args, pa, W, device, head_w, head_dec_ms, peak, peak_kind):
     (plan + attention kernel) and the whole step (copy-on-write copies, cache
     write, decode) timed per iteration by CUDA events on the launching stream,
     median / min / mean over the iterations.  A configuration whose distinct
-    K/V bytes are under 4x the L2 size gets L2 flushed (a 4x-L2 buffer
-    written) before every timed iteration, outside the events."""
+    K/V bytes are under 4x the L2 size gets L2 flushed before every timed
+    iteration, outside the events: a 4x-L2 buffer is written, then a second
+    one read, so the L2 holds none of the inputs and no dirty lines whose
+    write-back would land inside the timed kernel."""
     import numpy as np
     import torch
     l2 = int(torch.cuda.get_device_properties(device).L2_cache_size)
     flush_buf = torch.empty(4 * l2, dtype=torch.uint8, device=device)
+    flush_rd = torch.zeros(4 * l2, dtype=torch.uint8, device=device)
+
+    def flush_l2():
+        flush_buf.zero_()
+        flush_rd.sum(dtype=torch.int64)
     stream = torch.cuda.current_stream()
     iters = max(3, args.config_iters)
     results = {}
@@ -684,7 +702,7 @@ def measure_configs(args, pa, W, device, head_w, head_dec_ms, peak, peak_kind):
         clocks.start()
         for i in range(iters):
             if flush:
-                flush_buf.zero_()
+                flush_l2()
             step(evs[i])
         torch.cuda.synchronize()
         clocks.stop()
@@ -708,7 +726,8 @@ def measure_configs(args, pa, W, device, head_w, head_dec_ms, peak, peak_kind):
                          "frac": round(gbs / peak, 4), "peak_kind": peak_kind,
                          "bytes": "algorithmic (logical) K/V bytes, median pa_decode time",
                          "traffic": traffic, "traffic_source": _traffic_note(rec, traffic)},
-            "l2": (f"flushed before every timed iteration ({4 * l2 / 2**20:.0f} MiB written): "
+            "l2": (f"flushed before every timed iteration ({4 * l2 / 2**20:.0f} MiB written, "
+                   f"then another {4 * l2 / 2**20:.0f} MiB read): "
                    f"{unique / 2**20:.1f} MiB of distinct K/V < 4x L2" if flush else
                    f"no flush: {unique / 2**30:.2f} GiB of distinct K/V >= 4x L2"),
             "memory": config_memory(w, name),
@@ -736,7 +755,7 @@ def measure_configs(args, pa, W, device, head_w, head_dec_ms, peak, peak_kind):
                    for _ in range(iters)]
             for i in range(iters):
                 if flush:
-                    flush_buf.zero_()
+                    flush_l2()
                 sev[i][0].record(stream)
                 shared()
                 sev[i][1].record(stream)
@@ -755,7 +774,7 @@ def measure_configs(args, pa, W, device, head_w, head_dec_ms, peak, peak_kind):
         if own:
             del w
         torch.cuda.empty_cache()
-    del flush_buf
+    del flush_buf, flush_rd
     torch.cuda.empty_cache()
     return results
 
@@ -1036,6 +1055,9 @@ def run_shared_prefix(args):
 
 def main(argv=None):
     args = parse_args(argv)
+    if args.print_source_sha16:
+        print(json.dumps({k: source_hash(k) for k in KERNEL_SOURCES}))
+        return 0
     if args.ingest_ncu:
         ingest_ncu(args)
         return 0

@@ -331,35 +331,33 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
                 }
               }
             }
-            // online softmax of rows g (elements 0, 1) and g + 8 (2, 3), the
-            // running max raised only past kRescaleLog2 (as in decode)
-            float alpha[2] = {1.f, 1.f};
-            bool resc = false;
+            // online softmax of rows g (elements 0, 1) and g + 8 (2, 3); keys
+            // past an own range's end (only in its last block) get -inf
+            const bool part = valid < BS;
+            float alpha[2];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               float x[4];
 #pragma unroll
               for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                  const int key = kt * 16 + nt * 8 + 2 * tig + c;
-                  const float v = (s[nt][2 * h + c] + so[nt][2 * h + c]) * sl2r[h];
-                  x[2 * nt + c] = key < valid ? v : -INFINITY;
-                }
-              float bm = fmax3(fmaxf(x[0], x[1]), x[2], x[3]);
+                for (int c = 0; c < 2; ++c)
+                  x[2 * nt + c] = (s[nt][2 * h + c] + so[nt][2 * h + c]) * sl2r[h];
+              if (part) {
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  if (kt * 16 + (e >> 1) * 8 + 2 * tig + (e & 1) >= valid) x[e] = -INFINITY;
+              }
+              float bm = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
               bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
               bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
-              if (m_run[h] == -INFINITY) {
-                m_run[h] = bm;  // first keys: O and the sum are still zero
-              } else if (bm - m_run[h] > kRescaleLog2) {
-                alpha[h] = fast_exp2(m_run[h] - bm);
-                m_run[h] = bm;
-                resc = true;
-              }
+              const float mn = fmaxf(m_run[h], bm);
+              alpha[h] = fast_exp2(m_run[h] - mn);
+              m_run[h] = mn;
               float ps = 0.f;
 #pragma unroll
               for (int e = 0; e < 4; ++e) {
-                x[e] = fast_exp2(x[e] - m_run[h]);
+                x[e] = fast_exp2(x[e] - mn);
                 ps += x[e];
               }
               l_run[h] = l_run[h] * alpha[h] + ps;
@@ -369,14 +367,12 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
                 s[nt][2 * h + 1] = x[2 * nt + 1];
               }
             }
-            if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll
-              for (int n = 0; n < kNT; ++n) {
-                acc[n][0] *= alpha[0];
-                acc[n][1] *= alpha[0];
-                acc[n][2] *= alpha[1];
-                acc[n][3] *= alpha[1];
-              }
+            for (int n = 0; n < kNT; ++n) {
+              acc[n][0] *= alpha[0];
+              acc[n][1] *= alpha[0];
+              acc[n][2] *= alpha[1];
+              acc[n][3] *= alpha[1];
             }
             // P as the A operand (the S accumulators of two n-tiles are the A
             // fragment); bf16 keeps P as hi + lo parts (one bf16 value errs by
@@ -394,7 +390,6 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
             }
             // O += P V; values of keys past an own range's end are zeroed in the
             // fragments (they may hold anything, NaN included)
-            const bool part = valid < BS;
             const int tk = kt * 16 + 2 * tig;
             const uint32_t m_lo = part ? pair_mask(tk < valid, tk + 1 < valid) : 0xffffffffu;
             const uint32_t m_hi = part ? pair_mask(tk + 8 < valid, tk + 9 < valid) : 0xffffffffu;
@@ -559,40 +554,32 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
               s[mt][e] = tok < valid ? x : -INFINITY;
             }
           }
-          // online softmax per head column (every block has a valid token),
-          // the running max raised only past kRescaleLog2
-          float alpha[2] = {1.f, 1.f};
-          bool resc = false;
+          // online softmax per head column (every block has a valid token)
+          float alpha[2];
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             float bm = -INFINITY;
 #pragma unroll
-            for (int mt = 0; mt < BS / 16; ++mt) bm = fmax3(bm, s[mt][c], s[mt][2 + c]);
+            for (int mt = 0; mt < BS / 16; ++mt) bm = fmaxf(bm, fmaxf(s[mt][c], s[mt][2 + c]));
             bm = shfl_xor_max(bm);
-            if (m_run[c] == -INFINITY) {
-              m_run[c] = bm;
-            } else if (bm - m_run[c] > kRescaleLog2) {
-              alpha[c] = fast_exp2(m_run[c] - bm);
-              m_run[c] = bm;
-              resc = true;
-            }
+            const float mn = fmaxf(m_run[c], bm);
+            alpha[c] = fast_exp2(m_run[c] - mn);
+            m_run[c] = mn;
             float ps = 0.f;
 #pragma unroll
             for (int mt = 0; mt < BS / 16; ++mt) {
-              s[mt][c] = fast_exp2(s[mt][c] - m_run[c]);
-              s[mt][2 + c] = fast_exp2(s[mt][2 + c] - m_run[c]);
+              s[mt][c] = fast_exp2(s[mt][c] - mn);
+              s[mt][2 + c] = fast_exp2(s[mt][2 + c] - mn);
               ps += s[mt][c] + s[mt][2 + c];
             }
             l_run[c] = l_run[c] * alpha[c] + ps;
           }
-          if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll
-            for (int dt = 0; dt < kDT; ++dt) {
-              acc[dt][0] *= alpha[0];
-              acc[dt][1] *= alpha[1];
-              acc[dt][2] *= alpha[0];
-              acc[dt][3] *= alpha[1];
-            }
+          for (int dt = 0; dt < kDT; ++dt) {
+            acc[dt][0] *= alpha[0];
+            acc[dt][1] *= alpha[1];
+            acc[dt][2] *= alpha[0];
+            acc[dt][3] *= alpha[1];
           }
           // P^T as the B operand (8x8 (token, head) tiles transposed in
           // registers); bf16 keeps hi + lo parts

@@ -46,7 +46,6 @@ constexpr int kMaxGroup = 8;          // packed query heads per work item (MMA N
 constexpr int kBarrierBytes = 256;    // mbarrier area at the start of smem
 constexpr int kTileAlign = 1024;      // swizzled tiles start on this boundary
 constexpr int kMaxRanges = 1024;      // context ranges per sequence (fused merge uses smem)
-constexpr float kRescaleLog2 = 8.f;   // raise a head's running max only past this (log2 units)
 
 template <int CK, int D, int BS>
 struct DecodeCfg {
@@ -298,80 +297,49 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
   uint32_t skip_stage = 0;                // stages holding a block with a bad table entry
   bool failed = false;                    // a wait timed out: stop issuing / computing
 
-  // ---- work items: item -> (sequence, range, kv head, column group); kv
-  // heads innermost, so the heads of one range run side by side and share
-  // the table's cache lines.  The kv head's query heads are cut into column
-  // groups of at most 8 (the MMA's N); each group is its own item over the
-  // same blocks.  desc = a.order entry: (sequence, range, end token, ranges).
-  // The warp's blocks of an item are the range's blocks warp, warp + 4, ...
-  auto blocks_of_warp = [&](int4 d) {
-    const int t0 = d.y * a.split_tokens;
-    const int nblk = d.z > t0 ? (d.z + BS - 1) / BS - t0 / BS : 0;
-    return nblk > warp ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
-  };
-  // block-table entries of the warp's blocks, prefetched in registers: lane
-  // l of chunk c holds the entry of the warp's block 32 c + l
-  auto table_chunk = [&](int4 d, int c) -> int {
-    const int i = c * 32 + lane;
-    return i < blocks_of_warp(d)
-               ? a.block_tables[static_cast<int64_t>(d.x) * a.max_blocks +
-                                (d.y * a.split_tokens) / BS + warp + i * kDecodeWarps]
-               : -1;
-  };
-
-  // the CTA's first item, fetched by thread 0; every later one is fetched
-  // by thread 0 while warp 0 works on its last blocks of the current item,
-  // and its first table entries are read while the CTA merges the current
-  // item, so a new item's tile loads go out as soon as the ring is free
-  if (threadIdx.x == 0) {
+  // the next item and its descriptor, fetched by thread 0
+  auto fetch_next = [&]() {
     const int it = atomicAdd(a.counter, 1);
     s_item = it;
     if (it < total) s_desc = a.order[it / (a.hkv * a.ncg)];
-  }
+  };
+  if (threadIdx.x == 0) fetch_next();
   __syncthreads();
-  int item = s_item;
-  int4 desc = item < total ? s_desc : make_int4(0, 0, 0, 1);
-  int tab_cur = item < total ? table_chunk(desc, 0) : -1;
-  int tab_nxt = item < total ? table_chunk(desc, 1) : -1;
 
   for (;;) {
+    const int item = s_item;
     if (item >= total) break;
+
+    // ---- item -> (sequence, range, kv head); kv heads innermost, so the
+    // heads of one range run side by side and share the table's cache lines
+    // the kv head's query heads are cut into column groups of at most 8 (the
+    // MMA's N); each group is its own item over the same blocks
     const int kvh_cg = item % (a.hkv * a.ncg);
     const int kvh = kvh_cg / a.ncg, cg = kvh_cg % a.ncg;
     const int ncols = min(kMaxGroup, a.group - cg * kMaxGroup);  // heads of this item
+    const int4 desc = s_desc;
     const int seq = desc.x;
     const int split = desc.y;
     const int t1 = desc.z;  // end token of the range (validated by plan_kernel)
     const int nsplit = desc.w;
     const int t0 = split * a.split_tokens;
     const int jb0 = t0 / BS;
-    const int nb_w = blocks_of_warp(desc);
+    const int nblk = t1 > t0 ? (t1 + BS - 1) / BS - jb0 : 0;
+    const int nb_w = nblk > warp ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
+    const int32_t* table = a.block_tables + static_cast<int64_t>(seq) * a.max_blocks;
     const int h0 = kvh * a.group + cg * kMaxGroup;
 
-    // tab_cur is the table chunk the issue cursor is in, tab_nxt the one
-    // after it, so the table read never sits on the path from one block to
-    // the next
+    // ---- block-table entries of the warp's blocks, prefetched in registers:
+    // lane l holds the entry of the warp's block (32 * chunk + l); tab_cur is
+    // the chunk the issue cursor is in, tab_nxt the one after it, so the
+    // table read never sits on the path from one block to the next
+    auto load_chunk = [&](int c) -> int {
+      const int i = c * 32 + lane;
+      return i < nb_w ? table[jb0 + warp + i * kDecodeWarps] : -1;
+    };
     int tab_chunk = 0;
-    auto load_chunk = [&](int c) -> int { return table_chunk(desc, c); };
-
-    // thread 0: the next item's id (two blocks before warp 0's last) and
-    // descriptor (at its last block), consumed after the block loop
-    int next_item = -1;
-    int4 next_desc = make_int4(0, 0, 0, 1);
-    bool got_id = false, got_desc = false;
-    auto fetch_id = [&]() {
-      if (!got_id) {
-        next_item = atomicAdd(a.counter, 1);
-        got_id = true;
-      }
-    };
-    auto fetch_desc = [&]() {
-      fetch_id();
-      if (!got_desc) {
-        if (next_item < total) next_desc = a.order[next_item / (a.hkv * a.ncg)];
-        got_desc = true;
-      }
-    };
+    int tab_cur = load_chunk(0);
+    int tab_nxt = load_chunk(1);
 
     // ---- issue the two tile loads of the warp's i-th block of this item
     // (i increases by at most one chunk between calls)
@@ -468,10 +436,6 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
 
     const int li = lane >> 3;  // which 8x8 matrix of an ldmatrix.x4 this lane addresses
     for (int i = 0; i < nb_w; ++i) {
-      if (threadIdx.x == 0) {
-        if (i + 2 == nb_w) fetch_id();
-        if (i + 1 == nb_w) fetch_desc();
-      }
       const int st = n_consumed % kStages;
       const uint32_t par = (n_consumed / kStages) & 1u;
       if (!failed) {
@@ -533,43 +497,32 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
           }
         }
 
-        // ---- online softmax per head column.  The weights are taken against
-        // the running max m_run, which is raised (and O and the sum rescaled)
-        // only when a block's max exceeds it by more than kRescaleLog2: the
-        // weights then stay below 2^kRescaleLog2 and the normalised result is
-        // unchanged, while most blocks skip the rescale
-        bool resc = false;
-        float alpha[2] = {1.f, 1.f};
+        // ---- online softmax per head column
+        float alpha[2];
 #pragma unroll
         for (int c = 0; c < 2; ++c) {
           float bm = -INFINITY;
 #pragma unroll
-          for (int mt = 0; mt < C::kTokTiles; ++mt) bm = fmax3(bm, s[mt][c], s[mt][2 + c]);
+          for (int mt = 0; mt < C::kTokTiles; ++mt) bm = fmaxf(bm, fmaxf(s[mt][c], s[mt][2 + c]));
           bm = shfl_xor_max(bm);
-          if (m_run[c] == -INFINITY) {
-            m_run[c] = bm;  // first block: O and the sum are still zero
-          } else if (bm - m_run[c] > kRescaleLog2) {
-            alpha[c] = fast_exp2(m_run[c] - bm);
-            m_run[c] = bm;
-            resc = true;
-          }
+          const float mn = fmaxf(m_run[c], bm);
+          alpha[c] = fast_exp2(m_run[c] - mn);
+          m_run[c] = mn;
           float ps = 0.f;
 #pragma unroll
           for (int mt = 0; mt < C::kTokTiles; ++mt) {
-            s[mt][c] = fast_exp2(s[mt][c] - m_run[c]);
-            s[mt][2 + c] = fast_exp2(s[mt][2 + c] - m_run[c]);
+            s[mt][c] = fast_exp2(s[mt][c] - mn);
+            s[mt][2 + c] = fast_exp2(s[mt][2 + c] - mn);
             ps += s[mt][c] + s[mt][2 + c];
           }
           l_run[c] = l_run[c] * alpha[c] + ps;
         }
-        if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll
-          for (int dt = 0; dt < C::kDimTiles; ++dt) {
-            acc[dt][0] *= alpha[0];
-            acc[dt][1] *= alpha[1];
-            acc[dt][2] *= alpha[0];
-            acc[dt][3] *= alpha[1];
-          }
+        for (int dt = 0; dt < C::kDimTiles; ++dt) {
+          acc[dt][0] *= alpha[0];
+          acc[dt][1] *= alpha[1];
+          acc[dt][2] *= alpha[0];
+          acc[dt][3] *= alpha[1];
         }
 
         // ---- P^T as the B operand: transpose the 8x8 (token, head) tiles
@@ -644,14 +597,6 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
       if (!failed && i + kStages < nb_w) issue(i + kStages);
     }
 
-    // ---- hand the next item to the CTA (thread 0 fetched it above, or now
-    // when warp 0 had fewer than two blocks)
-    if (threadIdx.x == 0) {
-      fetch_desc();
-      s_item = next_item;
-      s_desc = next_desc;
-    }
-
     // ---- merge the warps' partial states through shared memory
     {
       float* scr = reinterpret_cast<float*>(wbase);
@@ -677,11 +622,6 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
       }
     }
     __syncthreads();
-    // the next item's first table entries, read while this one is merged
-    const int nitem = s_item;
-    const int4 ndesc = s_desc;
-    const int ntab_cur = nitem < total ? table_chunk(ndesc, 0) : -1;
-    const int ntab_nxt = nitem < total ? table_chunk(ndesc, 1) : -1;
     {
       constexpr int kVec = 8;
       const int units = ncols * (D / kVec);
@@ -798,12 +738,11 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
         }
       }
     }
+    // the next item is taken only now, when this CTA can start it at once,
+    // so no CTA holds an item it cannot start while others run dry
+    if (threadIdx.x == 0) fetch_next();
     __syncthreads();           // scratch (= stage memory) is free again ...
     fence_proxy_async_smem();  // ... and the next item's tile loads come after these accesses
-    item = nitem;
-    desc = ndesc;
-    tab_cur = ntab_cur;
-    tab_nxt = ntab_nxt;
   }
 
   // drain copies still in flight after a timeout (bounded again)

@@ -13,7 +13,6 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "prefill.cuh"
-#include "prefill_pp.cuh"
 #include "cascade.cuh"
 
 namespace {
@@ -722,9 +721,8 @@ pa_status pa_prefill(void* out, const void* q, pa_dtype q_dtype, const void* k_p
   a.num_blocks = num_blocks;
   a.max_ctx = max_context_len;
   a.sl2 = scale * 1.4426950408889634f;
-  // a CTA takes two query tiles of T = 128 / G tokens each
   const int T = pa::kPfRows / a.group;
-  dim3 grid(static_cast<unsigned>(cdiv(max_query_len, 2 * T)), static_cast<unsigned>(num_kv_heads),
+  dim3 grid(static_cast<unsigned>(cdiv(max_query_len, T)), static_cast<unsigned>(num_kv_heads),
             static_cast<unsigned>(num_seqs));
   if (grid.y > 65535 || grid.z > 65535)
     return fail(PA_ERR_SHAPE, "pa_prefill: too many kv heads or sequences for one launch");
@@ -732,14 +730,14 @@ pa_status pa_prefill(void* out, const void* q, pa_dtype q_dtype, const void* k_p
   auto launch = [&](auto kern, int smem_bytes) -> pa_status {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes);
     if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(prefill)");
-    kern<<<grid, pa::kPpThreads, smem_bytes, st>>>(a);
+    kern<<<grid, pa::kPfThreads, smem_bytes, st>>>(a);
     return PA_OK;
   };
   pa_status ls;
   const bool bf = q_dtype == PA_BF16;
-#define PA_PF_LAUNCH(BS_, D_)                                                                 \
-  (bf ? launch(pa::prefill_pp_kernel<true, BS_, D_>, pa::PrefillPpCfg<BS_, D_>::kSmemBytes)   \
-      : launch(pa::prefill_pp_kernel<false, BS_, D_>, pa::PrefillPpCfg<BS_, D_>::kSmemBytes))
+#define PA_PF_LAUNCH(BS_, D_)                                                              \
+  (bf ? launch(pa::prefill_kernel<true, BS_, D_>, pa::PrefillCfg<BS_, D_>::kSmemBytes)     \
+      : launch(pa::prefill_kernel<false, BS_, D_>, pa::PrefillCfg<BS_, D_>::kSmemBytes))
   if (head_dim == 64)
     ls = block_size == 16 ? PA_PF_LAUNCH(16, 64) : PA_PF_LAUNCH(32, 64);
   else

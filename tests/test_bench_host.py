@@ -91,7 +91,7 @@ NCU_CSV = '''==PROF== Connected to process 4242
 "3","4242","python3","127.0.0.1","void pa::plan_kernel(const int *, int)","1","7","(1024, 1, 1)","(1, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","byte","4,096"
 "4","4242","python3","127.0.0.1","void pa::decode_kernel<1, true, 128, 16>(pa::DecodeArgs)","1","7","(128, 1, 1)","(444, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_read.sum","Mbyte","1,077.45"
 "4","4242","python3","127.0.0.1","void pa::decode_kernel<1, true, 128, 16>(pa::DecodeArgs)","1","7","(128, 1, 1)","(444, 1, 1)","0","10.0","Command line profiler metrics","dram__bytes_write.sum","byte","7,160,000"
-"4","4242","python3","127.0.0.1","void pa::decode_kernel<1, true, 128, 16>(pa::DecodeArgs)","1","7","(128, 1, 1)","(444, 1, 1)","0","10.0","Command line profiler metrics","gpu__time_duration.sum","usecond","183.90"
+"4","4242","python3","127.0.0.1","void pa::decode_kernel<1, true, 128, 16>(pa::DecodeArgs)","1","7","(128, 1, 1)","(444, 1, 1)","0","10.0","Command line profiler metrics","gpu__time_duration.sum","ns","183900"
 '''
 
 
