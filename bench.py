@@ -390,11 +390,12 @@ def workload_seed(name: str, seed=None) -> int:
 def _full_seqs(name):
     return {"llama70b_gqa": 256, "llama13b_mha": 64, "fp8_longtail_bs16": 128,
             "fp8_longtail_bs32": 128, "shared_prefix_tails": 128, "shared_prefix_fork": 128,
-            "tiny": 4}[name]
+            "tiny": 4, "e4m3_uniform": 128}[name]
 
 
 def _sample_kw(name, n):
-    if name in ("llama70b_gqa", "llama13b_mha", "fp8_longtail_bs16", "fp8_longtail_bs32"):
+    if name in ("llama70b_gqa", "llama13b_mha", "fp8_longtail_bs16", "fp8_longtail_bs32",
+                "e4m3_uniform"):
         return {"num_seqs": n}
     if name.startswith("shared_prefix"):
         return {"prompts": max(1, n // 4)}

@@ -247,6 +247,16 @@ def fp8_longtail(seed=5, device="cpu", num_seqs=128, block_size=16, max_len=3276
     return w
 
 
+def e4m3_uniform(seed=5, device="cpu", num_seqs=128, context_len=4096, **kw) -> Workload:
+    """Diagnostic companion of the fp8 long-tail batch: the same layer shape
+    and cache format (32/8 heads, D 128, e4m3 cache, bf16 q, bs 16) with every
+    sequence ``context_len`` tokens, so the per-byte cost of the e4m3 path
+    can be told apart from the cost of a long-tailed length mix."""
+    lens = _lens_llama70b(num_seqs, context_len)
+    return _generic("e4m3_uniform", lens, 32, 8, 128, kw.pop("block_size", 16), "bf16", "e4m3",
+                    seed, device, **kw)
+
+
 def _sample_groups(prompts: int, samples: int) -> Dict:
     """The samples of one prompt form a group: group_seqs lists sequences
     p * samples + i group by group, group_start[g] is where group g starts."""
@@ -417,9 +427,11 @@ def prefill(seed=6, device="cpu", ctxs=(200, 300, 1, 77), nqs=(200, 77, 1, 50), 
 # workload, for sizes without building pools
 _SHAPES = {"tiny": (4, 64, 2), "llama13b_mha": (40, 128, 2), "llama70b_gqa": (8, 128, 2),
            "shared_prefix_fork": (8, 128, 2), "shared_prefix_tails": (8, 128, 2),
-           "fp8_longtail_bs16": (8, 128, 1), "fp8_longtail_bs32": (8, 128, 1)}
+           "fp8_longtail_bs16": (8, 128, 1), "fp8_longtail_bs32": (8, 128, 1),
+           "e4m3_uniform": (8, 128, 1)}
 _DEFAULT_SEEDS = {"tiny": 1, "llama13b_mha": 2, "llama70b_gqa": 3, "shared_prefix_fork": 4,
-                  "shared_prefix_tails": 4, "fp8_longtail_bs16": 5, "fp8_longtail_bs32": 5}
+                  "shared_prefix_tails": 4, "fp8_longtail_bs16": 5, "fp8_longtail_bs32": 5,
+                  "e4m3_uniform": 5}
 
 
 def default_seed(name: str) -> int:
@@ -437,6 +449,8 @@ def context_lens(name: str, seed: Optional[int] = None, **kw) -> np.ndarray:
         return _lens_llama13b(seed, **{k: kw[k] for k in ("num_seqs", "max_len", "min_len") if k in kw})
     if name == "llama70b_gqa":
         return _lens_llama70b(**{k: kw[k] for k in ("num_seqs", "context_len") if k in kw})
+    if name == "e4m3_uniform":
+        return _lens_llama70b(kw.get("num_seqs", 128), kw.get("context_len", 4096))
     if name.startswith("fp8_longtail"):
         return _lens_fp8(seed, **{k: kw[k] for k in ("num_seqs", "max_len") if k in kw})
     return _lens_shared_prefix(name.split("_")[-1], seed, **kw)
@@ -457,6 +471,7 @@ REGISTRY = {
     "shared_prefix_tails": shared_prefix_tails,
     "fp8_longtail_bs16": lambda seed=5, device="cpu", **kw: fp8_longtail(seed, device, block_size=16, **kw),
     "fp8_longtail_bs32": lambda seed=5, device="cpu", **kw: fp8_longtail(seed, device, block_size=32, **kw),
+    "e4m3_uniform": e4m3_uniform,
 }
 
 
