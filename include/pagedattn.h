@@ -175,12 +175,19 @@ pa_status pa_hash_blocks(const int32_t* token_ids, int64_t token_stride,
                          int32_t max_blocks, pa_stream_t stream);
 
 /*
- * pa_decode_split_tokens -- the context-split length pa_decode uses for these
- * sizes: the automatic choice when split_tokens == 0, else split_tokens
- * rounded up to a multiple of block_size and raised, if needed, so that no
- * sequence has more than 1024 ranges.  A value >= max_context_len means every
- * (sequence, kv head) is one work item and nothing is merged.  Returns 0 on
- * invalid arguments.
+ * pa_decode_split_tokens -- the context-split length that sizes pa_decode's
+ * workspace for these sizes: the automatic choice when split_tokens == 0,
+ * else split_tokens rounded up to a multiple of block_size and raised, if
+ * needed, so that no sequence has more than 1024 ranges.  A value >=
+ * max_context_len means every (sequence, kv head) is one work item and
+ * nothing is merged.  With split_tokens == 0 and a value below
+ * max_context_len, pa_decode's planning kernel may lengthen the ranges on
+ * the device, from the lengths it reads, to about
+ *   (sum of the valid context_lens) * num_kv_heads * ceil(G / 8) / 704
+ * tokens (G = query heads per kv head), in whole blocks and never below this
+ * value, so that a batch of a few long and many short contexts is cut by its
+ * total rather than by its longest context; the length used is left in the
+ * workspace (see pa_decode).  Returns 0 on invalid arguments.
  */
 int32_t pa_decode_split_tokens(int32_t num_seqs, int32_t num_kv_heads,
                                int32_t block_size, int32_t max_context_len,
@@ -231,7 +238,10 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
  * skipped (its tokens left out) and reported the same way.  The pools must be
  * 16-byte aligned (they are read through TMA tensor maps).
  * workspace: device memory of at least pa_decode_workspace_size(...) bytes,
- * 256-byte aligned, used only during the call (stream-ordered).
+ * 256-byte aligned, used only during the call (stream-ordered).  When the
+ * call has completed, the int32 at byte offset 8 of the workspace holds the
+ * range length it used; passing that value as split_tokens reproduces the
+ * output bit for bit.
  * The call enqueues two kernels on `stream`: a one-block planning kernel,
  * then the attention kernel, launched with programmatic stream
  * serialization so that its blocks set up while the plan runs and read the

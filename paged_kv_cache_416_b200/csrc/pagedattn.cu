@@ -124,18 +124,19 @@ int32_t choose_split(int32_t B, int32_t hkv, int32_t bs, int32_t max_ctx, int32_
 // are split, arrival counters [B * Hkv], fp32 lse [ranges * Hq] and fp32
 // partial outputs [ranges * Hq * D].
 struct WsLayout {
-  size_t counter = 0, total = 4, seq_off = 256, order = 0, arrived = 0, lse = 0, o = 0, bytes = 0;
-  bool split = false;
-  int64_t ranges = 0;  // upper bound on (sequence, range) pairs
+  size_t counter = 0, total = 4, split = 8, seq_off = 256, order = 0, arrived = 0, lse = 0, o = 0,
+         bytes = 0;
+  bool is_split = false;  // contexts may be cut into ranges (partials allocated)
+  int64_t ranges = 0;     // upper bound on (sequence, range) pairs
 };
 
 WsLayout ws_layout(int32_t B, int32_t hq, int32_t hkv, int32_t D, int32_t max_ctx, int32_t S) {
   WsLayout w;
-  w.split = S < max_ctx;
-  w.ranges = w.split ? static_cast<int64_t>(B) * cdiv(max_ctx, S) : B;
+  w.is_split = S < max_ctx;
+  w.ranges = w.is_split ? static_cast<int64_t>(B) * cdiv(max_ctx, S) : B;
   w.order = w.seq_off + static_cast<size_t>(round_up(static_cast<int64_t>(B + 1) * 4, 256));
   w.arrived = w.order + static_cast<size_t>(round_up(w.ranges * 16, 256));
-  if (!w.split) {
+  if (!w.is_split) {
     w.lse = w.o = w.arrived;
     w.bytes = w.arrived;
     return w;
@@ -536,18 +537,23 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_po
   a.max_blocks = max_blocks_per_seq;
   a.num_blocks = num_blocks;
   a.max_ctx = max_context_len;
-  a.split_tokens = w.split ? S : std::max(S, max_context_len);
+  const bool adapt = split_tokens == 0 && w.is_split;
+  a.split_tokens = w.is_split ? S : std::max(S, max_context_len);
+  a.split = adapt ? reinterpret_cast<const int32_t*>(ws + w.split) : nullptr;
   a.sl2 = scale * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
   a.out_scale = fp8 ? v_scale : 1.f;
   a.ncg = ncg;
 
+  // the automatic split may be lengthened on the device from the actual
+  // lengths (never shortened: the workspace holds the ranges of S)
   pa::plan_kernel<<<1, 1024, 0, st>>>(context_lens, num_seqs, max_context_len, max_blocks_per_seq,
-                                      block_size, a.split_tokens, num_kv_heads * ncg,
+                                      block_size, a.split_tokens, adapt, num_kv_heads * ncg,
                                       reinterpret_cast<int32_t*>(ws + w.counter),
                                       reinterpret_cast<int32_t*>(ws + w.total),
+                                      reinterpret_cast<int32_t*>(ws + w.split),
                                       reinterpret_cast<int32_t*>(ws + w.seq_off),
                                       reinterpret_cast<int4*>(ws + w.order),
-                                      w.split ? reinterpret_cast<int32_t*>(ws + w.arrived) : nullptr);
+                                      w.is_split ? reinterpret_cast<int32_t*>(ws + w.arrived) : nullptr);
   const int64_t items_upper = w.ranges * num_kv_heads * ncg;
   const bool qbf = q_dtype == PA_BF16;
   pa_status s;

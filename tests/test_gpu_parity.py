@@ -362,6 +362,43 @@ def test_full_size_workloads_against_oracle(pa, name):
     assert_attention_close(as_f64(out)[seqs], ref, f"{name} full size")
 
 
+def test_automatic_split_follows_the_batch_total(pa):
+    """With split_tokens == 0 the planning kernel lengthens the ranges to
+    about (sum of the lengths) x kv heads / 704 tokens, in whole blocks and
+    never below pa_decode_split_tokens (which sizes the workspace): on the
+    FP8 long-tail batch (177,982 tokens, longest 7,305) that is 2,032 tokens
+    instead of 1,024.  The length used, left in the workspace, reproduces the
+    output bit for bit when passed explicitly."""
+    w = W.make("fp8_longtail_bs16", device="cuda")
+    dev = "cuda"
+    kp, vp = w.k_pool.to(dev).clone(), w.v_pool.to(dev).clone()
+    pa.write_kv(w.new_k.to(dev).contiguous(), w.new_v.to(dev).contiguous(),
+                torch.from_numpy(w.slot_mapping).to(dev), kp, vp, w.k_scale, w.v_scale)
+    q = w.q.to(dev).contiguous()
+    bt = torch.from_numpy(w.block_tables).to(dev)
+    cl = torch.from_numpy(w.context_lens).to(dev)
+    bs = w.block_size
+    floor = pa.decode_split_tokens(w.num_seqs, w.num_kv_heads, bs, w.max_context_len)
+    nbytes = pa.decode_workspace_size(w.num_seqs, w.num_q_heads, w.num_kv_heads, w.head_dim, bs,
+                                      w.max_context_len)
+    ws = torch.zeros(nbytes, dtype=torch.uint8, device=dev)
+    out = pa.decode(q, kp, vp, bt, cl, w.scale, w.max_context_len, k_scale=w.k_scale,
+                    v_scale=w.v_scale, workspace=ws)
+    pa.sync_status()
+    used = int(ws[8:12].view(torch.int32).item())
+    units = w.num_kv_heads * -(-(w.num_q_heads // w.num_kv_heads) // 8)
+    want = -(-int(w.context_lens.sum()) * units // 704)
+    assert used == max(floor, min(-(-want // bs), -(-w.max_context_len // bs)) * bs)
+    assert (floor, used) == (1024, 2032)
+    again = pa.decode(q, kp, vp, bt, cl, w.scale, w.max_context_len, k_scale=w.k_scale,
+                      v_scale=w.v_scale, split_tokens=used)
+    pa.sync_status()
+    assert torch.equal(again, out)
+    seqs = [int(np.argmax(w.context_lens)), 0, 5, 77]
+    ref = compact_oracle_step(w, seqs)
+    assert_attention_close(as_f64(out)[seqs], ref, "fp8 long tail, lengthened split")
+
+
 @pytest.mark.parametrize("cache", ["bf16", "e4m3"])
 def test_decode_short_contexts_many_sequences(pa, cache):
     """2-8 keys per sequence concentrate the softmax weights, so outputs are
