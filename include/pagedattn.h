@@ -183,11 +183,13 @@ pa_status pa_hash_blocks(const int32_t* token_ids, int64_t token_stride,
  * nothing is merged.  With split_tokens == 0 and a value below
  * max_context_len, pa_decode's planning kernel may lengthen the ranges on
  * the device, from the lengths it reads, to about
- *   (sum of the valid context_lens) * num_kv_heads * ceil(G / 8) / 704
- * tokens (G = query heads per kv head), in whole blocks and never below this
- * value, so that a batch of a few long and many short contexts is cut by its
- * total rather than by its longest context; the length used is left in the
- * workspace (see pa_decode).  Returns 0 on invalid arguments.
+ *   (sum of the valid context_lens) * num_kv_heads * ceil(G / 8) / I
+ * tokens (G = query heads per kv head; I = 15/16 of 148 SMs times the decode
+ * kernel's resident blocks per SM), in whole blocks, never below this value
+ * and never past max_context_len, so that a batch of a few long and many
+ * short contexts is cut by its total rather than by its longest context; the
+ * length used is left in the workspace (see pa_decode).  Returns 0 on
+ * invalid arguments.
  */
 int32_t pa_decode_split_tokens(int32_t num_seqs, int32_t num_kv_heads,
                                int32_t block_size, int32_t max_context_len,
@@ -225,10 +227,13 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
  * (k_scale = v_scale = 1 for 16-bit caches), accumulated in fp32 and
  * rounded to q's dtype (round to nearest even).  n == 0 gives zeros.
  *
- * Contexts longer than the split length are cut into ranges of split_tokens
- * tokens (0 = automatic, see pa_decode_split_tokens); each range writes a
- * partial (log-sum-exp, normalised vector) into the workspace; the kernel
- * that finishes a sequence's last range combines them (log-sum-exp merge).
+ * A context longer than the split length S (split_tokens, or the automatic
+ * choice when it is 0, see pa_decode_split_tokens) is cut into
+ * n = ceil(len / S) ranges of whole blocks, as equal as blocks allow (the
+ * first ceil-share ranges one block longer), none longer than S; each range
+ * writes a partial (log-sum-exp, normalised vector) into the workspace, and
+ * the kernel that finishes a sequence's last range combines them
+ * (log-sum-exp merge).
  * Results depend only on the arguments (not on the grid or on timing): the
  * same call gives bit-identical outputs.
  *

@@ -119,15 +119,12 @@ struct DecodeArgs {
   int32_t* counter;        // workspace: work-queue counter (zeroed by plan_kernel)
   const int32_t* total;    // workspace: number of items (written by plan_kernel)
   const int32_t* seq_off;  // workspace: [B + 1] first range index of each sequence
-  const int4* order;       // workspace: [ranges] (sequence, range, end token, ranges of
-                           // the sequence), longest range first
+  const int4* order;       // workspace: [ranges] (sequence, range | ranges of the
+                           // sequence << 16, first token, end token), longest range first
   int32_t* arrived;        // workspace: [B * Hkv] ranges finished per (sequence, kv head)
   float* lse_part;         // workspace: [ranges * Hq]
   float* o_part;           // workspace: [ranges * Hq * D]
-  const int32_t* split;    // workspace: range length in tokens when plan_kernel may
-                           // lengthen it (the automatic split), else nullptr
   int num_seqs, hq, hkv, group, max_blocks, num_blocks, max_ctx;
-  int split_tokens;        // range length in tokens when `split` is nullptr
   int ncg;                 // column groups per kv head: ceil(group / 8) items read its blocks
   float sl2;               // scale * k_scale * log2(e)
   float out_scale;         // v_scale
@@ -135,31 +132,30 @@ struct DecodeArgs {
 
 // ---------------------------------------------------------------- planning
 constexpr int kPlanBuckets = 256;  // range-length classes of the longest-first order
-// work items the automatic range length aims at when the planning kernel
-// lengthens it from the batch's actual lengths: on the lognormal long-tail
-// batch (128 sequences, 32/8 heads, e4m3, 177,982 tokens) ranges of 768 /
-// 1024 / 1536 / 2048 / 4096 tokens ran 85.0 / 82.9 / 78.9 / 74.7 / 91.2 us,
-// i.e. about 700 items of (range, kv head) was best
-constexpr int64_t kAdaptItems = 704;
 
 // One CTA of 1024 threads, once per decode call:
-//  0. with `adapt` (the automatic split), lengthens the range length S to
-//     about (sum of the valid lengths) x units / kAdaptItems tokens, rounded
-//     up to whole blocks (never below S, whose ranges the workspace holds),
-//     and writes the length used to *split_out;
+//  0. with adapt_items > 0 (the automatic split), lengthens the range
+//     length S to about (sum of the valid lengths) x units / adapt_items
+//     tokens, rounded up to whole blocks (never below S, whose ranges the
+//     workspace holds, never past one range per sequence); writes the length
+//     used to *split_out;
 //  1. validates the context lengths (an out-of-range length counts as 0 and
-//     is reported), counts each sequence's ranges max(1, ceil(len / S)) and
-//     writes their exclusive prefix sum seq_off (where a sequence's partials
-//     go) and the item total (ranges * Hkv); zeroes the work counter;
+//     is reported), counts each sequence's ranges n = max(1, ceil(len / S))
+//     and writes their exclusive prefix sum seq_off (where a sequence's
+//     partials go) and the item total (ranges * Hkv); zeroes the work
+//     counter.  A sequence's nb blocks are dealt out evenly: its first
+//     nb % n ranges take floor(nb / n) + 1 blocks, the others floor(nb / n)
+//     (never more than S tokens), so no short remnant range of a split
+//     sequence, with the merge it triggers, is left for the end of the queue;
 //  2. writes the work order: every (sequence, range) pair with the range's
-//     end token and the sequence's range count, longest range first
+//     first and end token and the sequence's range count, longest range first
 //     (counting sort over kPlanBuckets length classes), so that the
 //     short ranges fill the end of the persistent grid's queue.  The order
 //     inside a class is whatever the atomics give: outputs do not depend on
 //     it, because every item writes its own output or partial slot.
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ ctx_lens, int B,
                                                     int max_ctx, int max_blocks, int bs, int S,
-                                                    bool adapt, int hkv, int32_t* counter,
+                                                    int adapt_items, int hkv, int32_t* counter,
                                                     int32_t* total, int32_t* split_out,
                                                     int32_t* seq_off, int4* order,
                                                     int32_t* arrived) {
@@ -174,9 +170,12 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
     const int c = ctx_lens[s];
     return (c < 0 || c > max_ctx || c > max_blocks * bs) ? -1 : c;
   };
-  if (adapt) {
+  // the thread's first sequence (s = tid) is read once and kept for every pass
+  const int c_own = tid < B ? valid_len(tid) : 0;
+  auto len_of = [&](int s) { return s == tid ? c_own : valid_len(s); };
+  if (adapt_items > 0) {
     long long sum = 0;
-    for (int s = tid; s < B; s += 1024) sum += max(0, valid_len(s));
+    for (int s = tid; s < B; s += 1024) sum += max(0, len_of(s));
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     if (lane == 0) warp_sum[warp] = sum;
@@ -186,7 +185,7 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
       if (lane == 0) {
-        const long long want = (sum * hkv + kAdaptItems - 1) / kAdaptItems;
+        const long long want = (sum * hkv + adapt_items - 1) / adapt_items;
         const long long blocks = (want + bs - 1) / bs;
         const long long cap = (static_cast<long long>(max_ctx) + bs - 1) / bs;  // one range
         s_split = static_cast<int>(max(static_cast<long long>(S), min(blocks, cap) * bs));
@@ -212,15 +211,16 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
     const int s = base + tid;
     int n = 0;
     if (s < B) {
-      int c = valid_len(s);
+      int c = len_of(s);
       if (c < 0) {
         record_error(PA_ERR_DEVICE_BOUNDS);
         c = 0;
       }
       n = c > 0 ? (c + S - 1) / S : 1;
-      const int last = c - (n - 1) * S;  // tokens of the last range (0 when c == 0)
-      if (n > 1) atomicAdd(&hist[bucket((S + bs - 1) / bs)], n - 1);
-      atomicAdd(&hist[bucket((last + bs - 1) / bs)], 1);
+      const int nb = (c + bs - 1) / bs;
+      const int q = nb / n, ex = nb % n;  // ex ranges of q + 1 blocks, n - ex of q
+      if (ex > 0) atomicAdd(&hist[bucket(q + 1)], ex);
+      atomicAdd(&hist[bucket(q)], n - ex);
     }
     int x = n;  // inclusive warp scan
 #pragma unroll
@@ -274,16 +274,18 @@ __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ 
   }
   __syncthreads();
   for (int s = tid; s < B; s += 1024) {
-    int c = valid_len(s);
+    int c = len_of(s);
     if (c < 0) c = 0;
     const int n = c > 0 ? (c + S - 1) / S : 1;
-    const int last = c - (n - 1) * S;
-    const int bf = bucket((S + bs - 1) / bs);
-    if (n > 1) {
-      const int p = atomicAdd(&hist[bf], n - 1);
-      for (int r = 0; r < n - 1; ++r) order[p + r] = make_int4(s, r, (r + 1) * S, n);
+    const int nb = (c + bs - 1) / bs;
+    const int q = nb / n, ex = nb % n;
+    const int p1 = ex > 0 ? atomicAdd(&hist[bucket(q + 1)], ex) : 0;
+    const int p0 = atomicAdd(&hist[bucket(q)], n - ex);
+    for (int r = 0; r < n; ++r) {
+      const int b0 = r * q + min(r, ex);     // first block of range r
+      const int b1 = b0 + q + (r < ex ? 1 : 0);
+      order[r < ex ? p1 + r : p0 + r - ex] = make_int4(s, r | (n << 16), b0 * bs, min(c, b1 * bs));
     }
-    order[atomicAdd(&hist[bucket((last + bs - 1) / bs)], 1)] = make_int4(s, n - 1, c, n);
   }
 }
 
@@ -331,7 +333,6 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
   __syncthreads();
 
   const int total = *a.total;
-  const int S = a.split != nullptr ? *a.split : a.split_tokens;  // range length in tokens
   uint32_t n_issued = 0, n_consumed = 0;  // warp-uniform ring counters
   uint32_t skip_stage = 0;                // stages holding a block with a bad table entry
   bool failed = false;                    // a wait timed out: stop issuing / computing
@@ -358,10 +359,10 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
     const int ncols = min(kMaxGroup, a.group - cg * kMaxGroup);  // heads of this item
     const int4 desc = s_desc;
     const int seq = desc.x;
-    const int split = desc.y;
-    const int t1 = desc.z;  // end token of the range (validated by plan_kernel)
-    const int nsplit = desc.w;
-    const int t0 = split * S;
+    const int split = desc.y & 0xffff;  // range index ...
+    const int nsplit = desc.y >> 16;    // ... of this many
+    const int t0 = desc.z;  // first token of the range (a block boundary) ...
+    const int t1 = desc.w;  // ... and its end (both validated by plan_kernel)
     const int jb0 = t0 / BS;
     const int nblk = t1 > t0 ? (t1 + BS - 1) / BS - jb0 : 0;
     const int nb_w = nblk > warp ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;

@@ -100,6 +100,15 @@ constexpr int kMaxQHeadsPerKv = 64;
 int32_t col_groups(int32_t hq, int32_t hkv) {
   return hkv > 0 ? std::max<int32_t>(1, static_cast<int32_t>(cdiv(hq / hkv, pa::kMaxGroup))) : 1;
 }
+// SMs the device-side lengthening of the automatic split plans for (a
+// B200's 148), fixed for the same reason as kPlanCtas; with the instance's
+// resident CTAs per SM it sets the work items the planning kernel aims at:
+// 15/16 of the persistent grid.  On the FP8 long-tail batch (128 sequences,
+// 177,982 tokens, 32/8 heads, e4m3) the best range lengths were 2,560 tokens
+// at bs 16 (592 CTAs: 74.1 us, against 76.5 at 2,048 and 75.6 at 3,072) and
+// 3,584 at bs 32 (444 CTAs: 70.2 us, against 74.5 at 2,048), i.e. about 0.93
+// of the grid's CTAs in (range, kv head) items.
+constexpr int64_t kPlanSms = 148;
 constexpr int64_t kMinSplit = 256;        // shortest range worth its partial
 constexpr int64_t kLongContext = 4096;    // above this, cap ranges ...
 constexpr int64_t kLongSplit = 1024;      // ... at this many tokens
@@ -253,15 +262,22 @@ cudaError_t launch_behind_plan(void (*kern)(Args), unsigned grid, int threads, i
   return cudaLaunchKernelEx(&cfg, kern, args);
 }
 
+// Resident CTAs per SM of one decode kernel instance (cached per device).
+template <int CK, bool kQBF16, int D, int BS>
+pa_status decode_occupancy(int dev, int* per_sm) {
+  using C = pa::DecodeCfg<CK, D, BS>;
+  static std::atomic<int> occ[kMaxDevices] = {};
+  return resident_ctas(occ, dev, pa::decode_kernel<CK, kQBF16, D, BS>, pa::kDecodeThreads,
+                       C::kSmemBytes, "pa_decode: kernel set-up", per_sm);
+}
+
 template <int CK, bool kQBF16, int D, int BS>
 pa_status launch_decode_main(const pa::DecodeArgs& args, int64_t items_upper, int dev,
                              cudaStream_t stream) {
   using C = pa::DecodeCfg<CK, D, BS>;
   auto kern = pa::decode_kernel<CK, kQBF16, D, BS>;
-  static std::atomic<int> occ[kMaxDevices] = {};
   int per_sm = 0;
-  const pa_status os = resident_ctas(occ, dev, kern, pa::kDecodeThreads, C::kSmemBytes,
-                                     "pa_decode: kernel set-up", &per_sm);
+  const pa_status os = decode_occupancy<CK, kQBF16, D, BS>(dev, &per_sm);
   if (os != PA_OK) return os;
   const int64_t grid = std::max<int64_t>(
       1, std::min<int64_t>(items_upper, static_cast<int64_t>(device_sms(dev)) * per_sm));
@@ -269,6 +285,15 @@ pa_status launch_decode_main(const pa::DecodeArgs& args, int64_t items_upper, in
                                            C::kSmemBytes, stream, args);
   if (e != cudaSuccess) return cuda_fail(e, "pa_decode launch");
   return PA_OK;
+}
+
+template <int CK, bool kQBF16>
+pa_status occupancy_shape(int D, int BS, int dev, int* per_sm) {
+  if (D == 128 && BS == 16) return decode_occupancy<CK, kQBF16, 128, 16>(dev, per_sm);
+  if (D == 128 && BS == 32) return decode_occupancy<CK, kQBF16, 128, 32>(dev, per_sm);
+  if (D == 64 && BS == 16) return decode_occupancy<CK, kQBF16, 64, 16>(dev, per_sm);
+  if (D == 64 && BS == 32) return decode_occupancy<CK, kQBF16, 64, 32>(dev, per_sm);
+  return fail(PA_ERR_SHAPE, "head_dim %d / block_size %d not supported", D, BS);
 }
 
 template <int CK, bool kQBF16>
@@ -537,17 +562,32 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_po
   a.max_blocks = max_blocks_per_seq;
   a.num_blocks = num_blocks;
   a.max_ctx = max_context_len;
-  const bool adapt = split_tokens == 0 && w.is_split;
-  a.split_tokens = w.is_split ? S : std::max(S, max_context_len);
-  a.split = adapt ? reinterpret_cast<const int32_t*>(ws + w.split) : nullptr;
   a.sl2 = scale * (fp8 ? k_scale : 1.f) * 1.4426950408889634f;
   a.out_scale = fp8 ? v_scale : 1.f;
   a.ncg = ncg;
+  const bool qbf = q_dtype == PA_BF16;
 
   // the automatic split may be lengthened on the device from the actual
-  // lengths (never shortened: the workspace holds the ranges of S)
+  // lengths (never shortened: the workspace holds the ranges of S), aiming
+  // at 15/16 of a kPlanSms-SM persistent grid of this instance in items
+  int adapt_items = 0;
+  if (split_tokens == 0 && w.is_split) {
+    int per_sm = 0;
+    pa_status os;
+    if (cache_dtype == PA_F16)
+      os = occupancy_shape<pa::kCacheF16, false>(head_dim, block_size, dev, &per_sm);
+    else if (cache_dtype == PA_BF16)
+      os = occupancy_shape<pa::kCacheBF16, true>(head_dim, block_size, dev, &per_sm);
+    else if (qbf)
+      os = occupancy_shape<pa::kCacheE4M3, true>(head_dim, block_size, dev, &per_sm);
+    else
+      os = occupancy_shape<pa::kCacheE4M3, false>(head_dim, block_size, dev, &per_sm);
+    if (os != PA_OK) return os;
+    adapt_items = static_cast<int>(std::max<int64_t>(1, kPlanSms * per_sm * 15 / 16));
+  }
   pa::plan_kernel<<<1, 1024, 0, st>>>(context_lens, num_seqs, max_context_len, max_blocks_per_seq,
-                                      block_size, a.split_tokens, adapt, num_kv_heads * ncg,
+                                      block_size, w.is_split ? S : std::max(S, max_context_len),
+                                      adapt_items, num_kv_heads * ncg,
                                       reinterpret_cast<int32_t*>(ws + w.counter),
                                       reinterpret_cast<int32_t*>(ws + w.total),
                                       reinterpret_cast<int32_t*>(ws + w.split),
@@ -555,7 +595,6 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_po
                                       reinterpret_cast<int4*>(ws + w.order),
                                       w.is_split ? reinterpret_cast<int32_t*>(ws + w.arrived) : nullptr);
   const int64_t items_upper = w.ranges * num_kv_heads * ncg;
-  const bool qbf = q_dtype == PA_BF16;
   pa_status s;
   if (cache_dtype == PA_F16)
     s = dispatch_shape<pa::kCacheF16, false>(a, head_dim, block_size, items_upper, dev, st);

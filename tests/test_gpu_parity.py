@@ -364,11 +364,12 @@ def test_full_size_workloads_against_oracle(pa, name):
 
 def test_automatic_split_follows_the_batch_total(pa):
     """With split_tokens == 0 the planning kernel lengthens the ranges to
-    about (sum of the lengths) x kv heads / 704 tokens, in whole blocks and
-    never below pa_decode_split_tokens (which sizes the workspace): on the
-    FP8 long-tail batch (177,982 tokens, longest 7,305) that is 2,032 tokens
-    instead of 1,024.  The length used, left in the workspace, reproduces the
-    output bit for bit when passed explicitly."""
+    about (sum of the lengths) x kv heads / I tokens, I = 15/16 of 148 SMs
+    times the kernel's resident blocks per SM, in whole blocks and never
+    below pa_decode_split_tokens (which sizes the workspace): on the FP8
+    long-tail batch (177,982 tokens, longest 7,305) well above the host's
+    1,024.  The length used, left in the workspace, reproduces the output
+    bit for bit when passed explicitly."""
     w = W.make("fp8_longtail_bs16", device="cuda")
     dev = "cuda"
     kp, vp = w.k_pool.to(dev).clone(), w.v_pool.to(dev).clone()
@@ -387,9 +388,34 @@ def test_automatic_split_follows_the_batch_total(pa):
     pa.sync_status()
     used = int(ws[8:12].view(torch.int32).item())
     units = w.num_kv_heads * -(-(w.num_q_heads // w.num_kv_heads) // 8)
-    want = -(-int(w.context_lens.sum()) * units // 704)
-    assert used == max(floor, min(-(-want // bs), -(-w.max_context_len // bs)) * bs)
-    assert (floor, used) == (1024, 2032)
+    total = int(w.context_lens.sum())
+
+    def rule(per_sm):
+        items = 148 * per_sm * 15 // 16
+        want = -(-total * units // items)
+        return max(floor, min(-(-want // bs), -(-w.max_context_len // bs)) * bs)
+
+    assert floor == 1024 and used > floor
+    assert used in {rule(k) for k in range(1, 9)}
+    # the work order in the workspace: every sequence cut into
+    # n = ceil(len / used) ranges of whole blocks differing by at most one
+    # block, none longer than `used`, listed longest first
+    B = w.num_seqs
+    nranges = int(ws[4:8].view(torch.int32).item()) // units
+    off = 256 + -(-(B + 1) * 4 // 256) * 256
+    order = ws[off:off + 16 * nranges].view(torch.int32).reshape(-1, 4).cpu().numpy()
+    nblk = (order[:, 3] - order[:, 2] + bs - 1) // bs
+    assert (np.diff(nblk) <= 0).all()
+    for sq in range(B):
+        rows = order[order[:, 0] == sq]
+        rows = rows[np.argsort(rows[:, 1] & 0xFFFF)]
+        n = max(1, -(-int(w.context_lens[sq]) // used))
+        assert len(rows) == n and ((rows[:, 1] >> 16) == n).all()
+        assert ((rows[:, 1] & 0xFFFF) == np.arange(n)).all()
+        assert rows[0, 2] == 0 and rows[-1, 3] == w.context_lens[sq]
+        assert (rows[1:, 2] == rows[:-1, 3]).all() and (rows[:, 2] % bs == 0).all()
+        nb = (rows[:, 3] - rows[:, 2] + bs - 1) // bs
+        assert nb.max() - nb.min() <= 1 and (rows[:, 3] - rows[:, 2] <= used).all()
     again = pa.decode(q, kp, vp, bt, cl, w.scale, w.max_context_len, k_scale=w.k_scale,
                       v_scale=w.v_scale, split_tokens=used)
     pa.sync_status()
