@@ -87,7 +87,9 @@ __device__ __forceinline__ float amax4(uint2 w) {
 }
 
 template <int CK, bool kQBF16, int D, int BS>
-__global__ void __launch_bounds__(kDecodeThreads)
+// at most 170 registers a thread (65,536 / (3 x 128)), so that three CTAs
+// share an SM in every instance (the bf16 bs-32 one needed 171)
+__global__ void __launch_bounds__(kDecodeThreads, 3)
 cascade_kernel(const __grid_constant__ CascadeArgs a) {
   using C = DecodeCfg<CK, D, BS>;
   constexpr bool kE4M3 = CK == kCacheE4M3;
