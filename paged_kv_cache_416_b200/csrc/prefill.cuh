@@ -20,7 +20,8 @@
 //           empty per stage), never a CTA-wide barrier inside the key loop.
 //   TMEM  = two S/P buffers [0, 64) and [64, 128) | O [128, 128 + D): S(kt)
 //           in buffer kt & 1 (fp32), then P(kt) over it (P_hi in its first
-//           32 columns, P_lo in the next 32, two 16-bit values per column)
+//           32 columns, P_lo (bf16 caches) in the next 32, two 16-bit values
+//           per column)
 //   per 64-key tile kt (K and V by TMA into two stages each, one box per
 //   (block, dim half); K(kt+2) is loaded once S(kt) is done, V(kt+2) once
 //   O(kt) is done; the load warp reads the block ids one tile ahead):
@@ -31,8 +32,9 @@
 //                               done, so it runs under the softmax of tile kt
 //     softmax      thread r: tcgen05.ld of its S row, causal and block masks
 //                  (only on tiles that need them), online max / sum in packed
-//                  fp32 pairs; P = P_hi + P_lo (two 16-bit parts, so P keeps
-//                  ~16 significant bits) by tcgen05.st into TMEM
+//                  fp32 pairs; with a bf16 cache P = P_hi + P_lo (two bf16
+//                  parts, so P keeps ~16 significant bits), with fp16 one
+//                  fp16 part, by tcgen05.st into TMEM
 //     O           += P V        tcgen05.mma, A = P from TMEM, B = V from shared
 //                               memory read MN-major (no transpose), M128 N=D,
 //                               2 x 4 x K16, accumulated in TMEM across tiles
@@ -292,7 +294,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
         fence_proxy_async_smem();
         __syncwarp();
       }
-      if (lane == 0 && !failed) {  // O += (P_hi + P_lo) V(kt): 2 x 4 MMAs of K = 16
+      if (lane == 0 && !failed) {  // O += (P_hi [+ P_lo]) V(kt): (2 x) 4 MMAs of K = 16
         tc_fence_after_sync();
         const uint32_t v_st = sV + st * C::kKBytes;
         const uint32_t tP = tbuf(kt);
@@ -300,10 +302,12 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
         for (int k = 0; k < kPfKeys / 16; ++k)
           umma_f16_ts(tO, tP + 8 * k, umma_desc_mn128(v_st + k * 2048, kPfKeys * 128), kIdescO,
                       (kt > 0 || k > 0) ? 1u : 0u);
+        if constexpr (kBF16) {
 #pragma unroll
-        for (int k = 0; k < kPfKeys / 16; ++k)
-          umma_f16_ts(tO, tP + 32 + 8 * k, umma_desc_mn128(v_st + k * 2048, kPfKeys * 128),
-                      kIdescO, 1u);
+          for (int k = 0; k < kPfKeys / 16; ++k)
+            umma_f16_ts(tO, tP + 32 + 8 * k, umma_desc_mn128(v_st + k * 2048, kPfKeys * 128),
+                        kIdescO, 1u);
+        }
         umma_commit(bar_o);
         umma_commit(v_empty + 8 * st);
       }
@@ -403,9 +407,9 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
       }
       const float nm = m_run == -INFINITY ? 0.f : -m_run * a.sl2;
       const uint64_t nm2 = f2(nm, nm);
-      // P = P_hi + P_lo, both in the operands' 16-bit type: rounding P to one
-      // 16-bit value alone (8 significant bits for bf16) errs by up to 2^-9 of
-      // each weight, which outputs formed by cancellation cannot absorb
+      // bf16: P = P_hi + P_lo, both bf16: rounding P to one bf16 value alone
+      // (8 significant bits) errs by up to 2^-9 of each weight, which outputs
+      // formed by cancellation cannot absorb.  fp16 keeps 11 bits: one part
       uint32_t ph[kPfKeys / 2], pl[kPfKeys / 2];
       uint64_t sum2 = f2(0.f, 0.f);
 #pragma unroll
@@ -416,11 +420,11 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
         sum2 = f2_add(sum2, pp);
         const uint32_t h = pack2<kBF16>(p0, p1);
         ph[c / 2] = h;
-        uint64_t hf;
-        if constexpr (kBF16) hf = f2(__uint_as_float(h << 16), __uint_as_float(h & 0xffff0000u));
-        else hf = f2(to_float<false>(h & 0xffff), to_float<false>(h >> 16));
-        const float2 d = f2_split(f2_sub(pp, hf));
-        pl[c / 2] = pack2<kBF16>(d.x, d.y);
+        if constexpr (kBF16) {
+          const uint64_t hf = f2(__uint_as_float(h << 16), __uint_as_float(h & 0xffff0000u));
+          const float2 d = f2_split(f2_sub(pp, hf));
+          pl[c / 2] = pack2<true>(d.x, d.y);
+        }
       }
       const float2 ss = f2_split(sum2);
       l_run = l_run * alpha + (ss.x + ss.y);
@@ -450,7 +454,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
       // P(kt) over S(kt) in its buffer: the buffer's previous reader O(kt-2)
       // finished before S(kt) did
       tmem_st32(tb, ph);
-      tmem_st32(tb + 32, pl);
+      if constexpr (kBF16) tmem_st32(tb + 32, pl);
       tmem_wait_st();
       tc_fence_before_sync();
       __syncwarp();
