@@ -23,7 +23,10 @@
 // O += P V (A = P straight from the S accumulators, B = V by ldmatrix.trans).
 // An own range runs the decode kernel's form with the member's heads as the
 // MMA's N = 8 columns: S^T = K Q^T, P^T by movmatrix, O^T += V^T P^T, half the
-// MMAs of a 16-row tile.  bf16 keeps P as hi + lo parts in both.
+// MMAs of a 16-row tile.  When every member's own part is short (a fork,
+// where each sample owns only its copied partial block), one own-group range
+// takes them all, warp w walking member w's blocks, so the chunk pays one
+// range start and one partial instead of one per member.  bf16 keeps P as hi + lo parts in both.
 // The warps' states merge through shared memory; a chunk of one range writes
 // the output, otherwise every range writes (log-sum-exp, normalised output)
 // per row (-inf for rows it does not attend) and the CTA that finishes the
@@ -38,6 +41,12 @@
 namespace pa {
 
 constexpr int kCascadeRows = 16;        // query rows per chunk (members x heads)
+constexpr int kRangeShared = -1;        // range member field: the shared blocks
+constexpr int kRangeOwnGroup = -2;      // ... every member's own blocks, one warp each
+// a chunk of at most 4 members with at most 8 heads per kv head whose own
+// parts are all this short runs them as one own-group range, not one range
+// (four warps, a merge) per member
+constexpr int kOwnGroupMaxBlocks = 8;
 constexpr int kCascadeMaxRanges = 512;  // ranges per chunk (their weights sit in smem)
 // work items (x Hkv) the range length aims at: ~1.5 waves of 444 persistent
 // CTAs (on the shared-prefix workload 666 ran 74.9 us, 555: 75.0, 888: 74.8,
@@ -55,8 +64,9 @@ struct CascadeArgs {
   const int32_t* chunk_seqs;   // members, chunk by chunk
   const int4* chunks;          // [2 * chunks]: (member offset, members, shared blocks, first
                                // slot), (ranges, -, -, -)
-  const int4* ranges;          // [slots]: (chunk, member or -1 for shared, first block, end
-                               // block): table entries of the leader (shared) or the member
+  const int4* ranges;          // [slots]: (chunk, member, or -1 for shared, -2 for every
+                               // member's own, first block, end block): table entries of the
+                               // leader (shared) or the member(s)
   const int32_t* total;        // number of ranges
   int32_t* counter;            // work counter (zeroed by the planning kernel)
   int32_t* arrived;            // [chunks * Hkv] ranges finished
@@ -146,7 +156,9 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
     const int slot = item / a.hkv;
     const int4 rd = a.ranges[slot];
     const int chunk = rd.x, member = rd.y, b0 = rd.z, b1 = rd.w;
-    const bool shared = member < 0;
+    const bool shared = member == kRangeShared;
+    // every member's own blocks at once, warp w walking member w's
+    const bool group = member == kRangeOwnGroup;
     // the 16-row form serves shared ranges, and own ranges of a member with
     // more than 8 heads per kv head; other own ranges take the 8-column form
     const bool rowform = shared || G > kMaxGroup;
@@ -160,17 +172,24 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
       s_ctx[threadIdx.x] = a.context_lens[seq];  // validated by the planning kernel
     }
     __syncthreads();
-    const int own_seq = s_seq[shared ? 0 : member];
-    const int own_ctx = shared ? 0 : s_ctx[member];
+    // this warp's member (idle warps of an own-group range take the last
+    // member's sequence and walk no block)
+    const int wm = shared ? 0 : (group ? min(warp, members - 1) : member);
+    const int own_seq = s_seq[wm];
+    const int own_ctx = shared ? 0 : s_ctx[wm];
     const int nblk = b1 - b0;
-    const int nb_w = nblk > warp ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0;
+    const int nb_w = group ? (warp < members ? max(0, (own_ctx + BS - 1) / BS - b0) : 0)
+                           : (nblk > warp ? (nblk - warp + kDecodeWarps - 1) / kDecodeWarps : 0);
     const int32_t* table = a.block_tables + static_cast<int64_t>(own_seq) * a.max_blocks;
+    // table index of the warp's i-th block: every 4th block of the range,
+    // or, in an own-group range, every block of its member from b0 on
+    auto jblk = [&](int i) { return group ? b0 + i : b0 + warp + i * kDecodeWarps; };
 
     // ---- table entries of the warp's blocks, 32 ahead in registers (lane l
     // holds the warp's block 32 * chunk + l)
     auto load_chunk = [&](int c) -> int {
       const int i = c * 32 + lane;
-      return i < nb_w ? table[b0 + warp + i * kDecodeWarps] : -1;
+      return i < nb_w ? table[jblk(i)] : -1;
     };
     int tab_chunk = 0;
     int tab_cur = load_chunk(0);
@@ -510,7 +529,7 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
         if (consume(st)) {
           const uint32_t sK = wbase_s + st * C::kStageBytes;
           const uint32_t sV = sK + C::kTileBytes;
-          const int j = b0 + warp + i * kDecodeWarps;       // the block's table entry
+          const int j = jblk(i);                            // the block's table entry
           const int valid = min(BS, own_ctx - j * BS);      // its tokens inside the context
           // S^T = K Q^T (rows: tokens, cols: the member's heads), four chains
           float s[BS / 16][4];
@@ -674,20 +693,22 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
       // combine the 4 warps; the 16-row form covers rows 0..nrow-1 of its
       // tile (scratch: O [16][D], max at 16 D, sums at 16 D + 16), the
       // 8-column form the member's G rows (scratch: O [8][D], max at 8 D,
-      // sums at 8 D + 8)
-      const int nrow = shared ? rows : G;
+      // sums at 8 D + 8); in an own-group range row r is member r / G's
+      // head r % G, held by warp r / G alone
+      const int nrow = (shared || group) ? rows : G;
       const int mrow = rowform ? kRows : 8;
       constexpr int kVec = 8;
       const int units = nrow * (D / kVec);
       for (int u = threadIdx.x; u < units; u += kDecodeThreads) {
         const int rl = u / (D / kVec);
         const int d0 = (u % (D / kVec)) * kVec;
+        const int hl = group ? rl % G : rl;  // the row in the warps' scratch
         float mw[kDecodeWarps];
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kDecodeWarps; ++w) {
           const float* sw = reinterpret_cast<const float*>(ring + w * C::kWarpBytes);
-          mw[w] = sw[mrow * D + rl];
+          mw[w] = (!group || w == rl / G) ? sw[mrow * D + hl] : -INFINITY;
           M = fmaxf(M, mw[w]);
         }
         float o[kVec];
@@ -697,11 +718,12 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
         if (M != -INFINITY) {
 #pragma unroll
           for (int w = 0; w < kDecodeWarps; ++w) {
+            if (group && w != rl / G) continue;
             const float* sw = reinterpret_cast<const float*>(ring + w * C::kWarpBytes);
             const float f = fast_exp2(mw[w] - M);
-            L += f * sw[mrow * D + mrow + rl];
-            const float4 x0 = *reinterpret_cast<const float4*>(sw + rl * D + d0);
-            const float4 x1 = *reinterpret_cast<const float4*>(sw + rl * D + d0 + 4);
+            L += f * sw[mrow * D + mrow + hl];
+            const float4 x0 = *reinterpret_cast<const float4*>(sw + hl * D + d0);
+            const float4 x1 = *reinterpret_cast<const float4*>(sw + hl * D + d0 + 4);
             o[0] += f * x0.x; o[1] += f * x0.y; o[2] += f * x0.z; o[3] += f * x0.w;
             o[4] += f * x1.x; o[5] += f * x1.y; o[6] += f * x1.z; o[7] += f * x1.w;
           }
@@ -709,7 +731,7 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
 #pragma unroll
           for (int v = 0; v < kVec; ++v) o[v] *= inv;
         }
-        const int r = shared ? rl : member * G + rl;  // the chunk's row
+        const int r = (shared || group) ? rl : member * G + rl;  // the chunk's row
         if (nranges == 1) {
           const int64_t qh = static_cast<int64_t>(s_seq[r / G]) * a.hq + kvh * G + r % G;
           uint4 pk;
@@ -727,7 +749,7 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
         }
       }
       // the rows an own range does not attend carry no weight
-      if (!shared && nranges > 1)
+      if (!shared && !group && nranges > 1)
         for (int r = threadIdx.x; r < rows; r += kDecodeThreads)
           if (r / G != member)
             a.lse_part[(static_cast<int64_t>(slot) * a.hkv + kvh) * kRows + r] = -INFINITY;
@@ -826,9 +848,12 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
 //     what keeps a chunk under kCascadeMaxRanges ranges;
 //  5. each chunk's shared blocks are cut into ceil(P / R) equal ranges and
 //     each member's own blocks into max(1, ceil(n / R)) (an empty range
-//     still writes a zero output), every range with its partial slot; the
-//     work list holds one (chunk, member or -1, first block, end block) per
-//     slot, and the arrival counters and the work counter are zeroed.
+//     still writes a zero output), every range with its partial slot; in a
+//     chunk of up to 4 members and 8 heads per kv head whose own parts are
+//     all at most kOwnGroupMaxBlocks (and R) blocks, one own-group range
+//     covers every member's own blocks instead; the work list holds one
+//     (chunk, member / -1 / -2, first block, end block) per slot, and the
+//     arrival counters and the work counter are zeroed.
 // Chunk and slot numbers come from atomics (their order varies), but every
 // output depends only on its chunk's ranges, merged in range order: results
 // are the same from call to call.
@@ -943,22 +968,34 @@ __global__ void __launch_bounds__(1024) cascade_plan_kernel(
     const int4 d = chunks[2 * c];
     const int P = d.z;
     const int nsh = P > 0 ? (P + R - 1) / R : 0;
+    // short own parts of a shared chunk: one own-group range
+    int own_max = 0;
+    for (int i = 0; i < d.y; ++i) own_max = max(own_max, own_blocks(chunk_seqs[d.x + i], P));
+    const bool own_group = P > 0 && d.y <= kDecodeWarps && group <= kMaxGroup &&
+                           own_max <= min(kOwnGroupMaxBlocks, R);
     int nr = nsh;
-    for (int i = 0; i < d.y; ++i) nr += max(1, (own_blocks(chunk_seqs[d.x + i], P) + R - 1) / R);
+    if (own_group) nr += 1;
+    else
+      for (int i = 0; i < d.y; ++i) nr += max(1, (own_blocks(chunk_seqs[d.x + i], P) + R - 1) / R);
     const int slot0 = atomicAdd(&n_slots, nr);
     chunks[2 * c] = make_int4(d.x, d.y, P, slot0);
     chunks[2 * c + 1] = make_int4(nr, 0, 0, 0);
     int sl = slot0;
     if (nsh > 0) {
       const int len = (P + nsh - 1) / nsh;  // equal shared ranges
-      for (int k = 0; k < nsh; ++k) ranges[sl++] = make_int4(c, -1, k * len, min(P, (k + 1) * len));
+      for (int k = 0; k < nsh; ++k)
+        ranges[sl++] = make_int4(c, kRangeShared, k * len, min(P, (k + 1) * len));
     }
-    for (int i = 0; i < d.y; ++i) {
-      const int n = own_blocks(chunk_seqs[d.x + i], P);
-      const int no = max(1, (n + R - 1) / R);
-      const int len = n > 0 ? (n + no - 1) / no : 0;  // equal own ranges
-      for (int k = 0; k < no; ++k)
-        ranges[sl++] = make_int4(c, i, P + min(n, k * len), P + min(n, (k + 1) * len));
+    if (own_group) {
+      ranges[sl++] = make_int4(c, kRangeOwnGroup, P, P + own_max);
+    } else {
+      for (int i = 0; i < d.y; ++i) {
+        const int n = own_blocks(chunk_seqs[d.x + i], P);
+        const int no = max(1, (n + R - 1) / R);
+        const int len = n > 0 ? (n + no - 1) / no : 0;  // equal own ranges
+        for (int k = 0; k < no; ++k)
+          ranges[sl++] = make_int4(c, i, P + min(n, k * len), P + min(n, (k + 1) * len));
+      }
     }
     for (int h = 0; h < hkv; ++h) arrived[c * hkv + h] = 0;
   }
