@@ -794,27 +794,54 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
           if (lane == 0) wsum_s[r] = W;
         }
         __syncthreads();
-        constexpr int kVec = 4;
+        // one unit = 16 dims of one row; four ranges per pass, their loads
+        // issued together (a weightless range loads nothing)
+        constexpr int kVec = 16;
         const int units = rows * (D / kVec);
         for (int u = threadIdx.x; u < units; u += kDecodeThreads) {
           const int r = u / (D / kVec);
           const int d0 = (u % (D / kVec)) * kVec;
-          float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+          float o[kVec];
+#pragma unroll
+          for (int v = 0; v < kVec; ++v) o[v] = 0.f;
           const float* op = a.o_part + (base + r) * D + d0;
-          for (int i = 0; i < nranges; ++i) {
-            const float w = w_s[i * kRows + r];
-            if (w > 0.f) {
-              const float4 x = __ldcg(reinterpret_cast<const float4*>(op + i * rstride * D));
-              o0 += w * x.x; o1 += w * x.y; o2 += w * x.z; o3 += w * x.w;
+          for (int i0 = 0; i0 < nranges; i0 += 4) {
+            float w[4];
+            float4 x[4][kVec / 4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              w[k] = i0 + k < nranges ? w_s[(i0 + k) * kRows + r] : 0.f;
+#pragma unroll
+              for (int q4 = 0; q4 < kVec / 4; ++q4)
+                x[k][q4] = w[k] > 0.f ? __ldcg(reinterpret_cast<const float4*>(
+                                            op + (i0 + k) * rstride * D + 4 * q4))
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
             }
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+#pragma unroll
+              for (int q4 = 0; q4 < kVec / 4; ++q4) {
+                o[4 * q4] += w[k] * x[k][q4].x;
+                o[4 * q4 + 1] += w[k] * x[k][q4].y;
+                o[4 * q4 + 2] += w[k] * x[k][q4].z;
+                o[4 * q4 + 3] += w[k] * x[k][q4].w;
+              }
           }
           const float W = wsum_s[r];
           const float inv = W > 0.f ? 1.f / W : 0.f;
           const int64_t qh = static_cast<int64_t>(s_seq[r / G]) * a.hq + kvh * G + r % G;
-          uint2 pk;
-          pk.x = pack2<kQBF16>(o0 * inv, o1 * inv);
-          pk.y = pack2<kQBF16>(o2 * inv, o3 * inv);
-          *reinterpret_cast<uint2*>(reinterpret_cast<uint16_t*>(a.out) + qh * D + d0) = pk;
+          uint4 pk0, pk1;
+          pk0.x = pack2<kQBF16>(o[0] * inv, o[1] * inv);
+          pk0.y = pack2<kQBF16>(o[2] * inv, o[3] * inv);
+          pk0.z = pack2<kQBF16>(o[4] * inv, o[5] * inv);
+          pk0.w = pack2<kQBF16>(o[6] * inv, o[7] * inv);
+          pk1.x = pack2<kQBF16>(o[8] * inv, o[9] * inv);
+          pk1.y = pack2<kQBF16>(o[10] * inv, o[11] * inv);
+          pk1.z = pack2<kQBF16>(o[12] * inv, o[13] * inv);
+          pk1.w = pack2<kQBF16>(o[14] * inv, o[15] * inv);
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(a.out) + qh * D + d0);
+          dst[0] = pk0;
+          dst[1] = pk1;
         }
       }
     }

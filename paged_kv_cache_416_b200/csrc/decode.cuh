@@ -729,7 +729,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
         // (1) every range's lse of every head into shared memory (the ring is
         // free: the warps' scratch was consumed above), (2) per head the max
         // and the weights w_i = 2^(lse_i - max), (3) the weighted sum of the
-        // partial outputs with independent (unrolled) loads
+        // partial outputs, four ranges' loads at a time
         float* lse_s = reinterpret_cast<float*>(ring);           // [nsplit][group]
         float* wsum_s = lse_s + nsplit * ncols;                  // [ncols]
         const int64_t base = static_cast<int64_t>(a.seq_off[seq]) * a.hq + h0;
@@ -762,11 +762,21 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
           const int d0 = (u % (D / kVec)) * kVec;
           float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
           const float* op = a.o_part + (base + h) * D + d0;
-#pragma unroll 8
-          for (int i = 0; i < nsplit; ++i) {
-            const float w = lse_s[i * ncols + h];
-            const float4 x = __ldcg(reinterpret_cast<const float4*>(op + static_cast<int64_t>(i) * a.hq * D));
-            o0 += w * x.x; o1 += w * x.y; o2 += w * x.z; o3 += w * x.w;
+          // four ranges per pass, their loads issued together
+          for (int i0 = 0; i0 < nsplit; i0 += 4) {
+            float w[4];
+            float4 x[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const bool in = i0 + k < nsplit;
+              w[k] = in ? lse_s[(i0 + k) * ncols + h] : 0.f;
+              x[k] = in ? __ldcg(reinterpret_cast<const float4*>(op + static_cast<int64_t>(i0 + k) * a.hq * D))
+                        : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              o0 += w[k] * x[k].x; o1 += w[k] * x[k].y; o2 += w[k] * x[k].z; o3 += w[k] * x[k].w;
+            }
           }
           const float W = wsum_s[h];
           const float inv = W > 0.f ? 1.f / W : 0.f;
