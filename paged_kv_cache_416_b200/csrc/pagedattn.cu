@@ -218,7 +218,7 @@ EncodeTiledFn encode_tiled_fn() {
 // one block, landing in shared memory as [half][token][R] with the R-byte
 // swizzle (128B or 64B).  Must match DecodeCfg / tile_off in decode.cuh.
 // With one_half the box is a single dim half (the prefill kernel places the
-// halves of consecutive blocks in separate K-major tiles).
+// halves of consecutive blocks of K in separate K-major tiles).
 pa_status encode_pool_map(CUtensorMap* map, const void* pool, int32_t num_blocks, int32_t bs,
                           int32_t hkv, int32_t head_dim, int32_t elem, bool one_half = false) {
   EncodeTiledFn fn = encode_tiled_fn();
@@ -752,7 +752,7 @@ pa_status pa_prefill(void* out, const void* q, pa_dtype q_dtype, const void* k_p
   pa_status ms = encode_pool_map(&a.tmap_k, k_pool, num_blocks, block_size, num_kv_heads,
                                  head_dim, 2, true);
   if (ms == PA_OK)
-    ms = encode_pool_map(&a.tmap_v, v_pool, num_blocks, block_size, num_kv_heads, head_dim, 2, true);
+    ms = encode_pool_map(&a.tmap_v, v_pool, num_blocks, block_size, num_kv_heads, head_dim, 2);
   if (ms != PA_OK) return ms;
   a.out = out;
   a.q = q;

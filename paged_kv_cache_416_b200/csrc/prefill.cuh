@@ -22,9 +22,10 @@
 //           in buffer kt & 1 (fp32), then P(kt) over it (P_hi in its first
 //           32 columns, P_lo (bf16 caches) in the next 32, two 16-bit values
 //           per column)
-//   per 64-key tile kt (K and V by TMA into two stages each, one box per
-//   (block, dim half); K(kt+2) is loaded once S(kt) is done, V(kt+2) once
-//   O(kt) is done; the load warp reads the block ids one tile ahead):
+//   per 64-key tile kt (K and V by TMA into two stages each, K one box per
+//   (block, dim half), V one box per block; K(kt+2) is loaded once S(kt) is
+//   done, V(kt+2) once O(kt) is done; the load warp reads the block ids 32 at
+//   a time, a chunk ahead, and polls the stages without sleeping on either):
 //     S            = Q K^T      tcgen05.mma, A = Q and B = K from shared memory
 //                               (K-major), M128 N64, D/16 x K16; S(kt+1) is
 //                               issued once the rows have read S(kt) and
@@ -67,8 +68,9 @@ template <int BS, int D>
 struct PrefillCfg {
   static constexpr int kHalves = D / 64;                  // 128-byte dim halves of a row
   static constexpr int kQBytes = kPfRows * D * 2;         // [halves][128 rows][128 B]
-  static constexpr int kKBytes = kPfKeys * D * 2;         // [halves][64 keys][128 B]
+  static constexpr int kKBytes = kPfKeys * D * 2;         // K: [halves][64 keys][128 B]
   static constexpr int kBlocksPerTile = kPfKeys / BS;
+  static constexpr int kVBlockBytes = kHalves * BS * 128; // V: [blocks][halves][bs keys][128 B]
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQBytes;           // 2 stages
   static constexpr int kOffV = kOffK + 2 * kKBytes;       // 2 stages
@@ -80,7 +82,8 @@ struct PrefillCfg {
 
 struct PrefillArgs {
   // Pools viewed as 5-D bytes (x, token, half, kv head, block) =
-  // (128, bs, D / 64, Hkv, N); box (128, bs, 1, 1, 1): one dim half of one block.
+  // (128, bs, D / 64, Hkv, N); a K box (128, bs, 1, 1, 1) is one dim half of
+  // one block, a V box (128, bs, D / 64, 1, 1) the whole block
   CUtensorMap tmap_k;
   CUtensorMap tmap_v;
   void* out;                   // [total_q, Hq, D], q's dtype
@@ -161,9 +164,10 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     const int p = table[j];
     return (p >= 0 && p < a.num_blocks) ? p : -2;
   };
-  // loader lane 0: TMA loads of one K or V tile into its stage (one box per
-  // block and dim half); blocks past the context or with a bad entry
-  // (phys < 0) are not loaded
+  // loader lane 0: TMA loads of one K or V tile into its stage (K: one box
+  // per block and dim half, so that each half is one K-major tile; V: one
+  // box per block, both halves); blocks past the context or with a bad
+  // entry (phys < 0) are not loaded
   auto issue_tile = [&](int kt, bool is_v, const int* phys) {
     const int st = kt & 1;
     uint32_t bytes = 0;
@@ -177,9 +181,13 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
 #pragma unroll
     for (int b = 0; b < C::kBlocksPerTile; ++b) {
       if (phys[b] < 0) continue;
+      if (is_v) {
+        tma_load_5d(dst + b * C::kVBlockBytes, map, 0, 0, 0, kvh, phys[b], bar);
+      } else {
 #pragma unroll
-      for (int hf = 0; hf < C::kHalves; ++hf)
-        tma_load_5d(dst + hf * (kPfKeys * 128) + b * BS * 128, map, 0, 0, hf, kvh, phys[b], bar);
+        for (int hf = 0; hf < C::kHalves; ++hf)
+          tma_load_5d(dst + hf * (kPfKeys * 128) + b * BS * 128, map, 0, 0, hf, kvh, phys[b], bar);
+      }
     }
   };
 
@@ -286,7 +294,8 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
           const int row = lane + 32 * i, key = row & (kPfKeys - 1), hf = row >> 6;
           if (kt * kPfKeys + key >= ctx || ((bad >> (key / BS)) & 1)) {
             uint4* dst = reinterpret_cast<uint4*>(base + C::kOffV + st * C::kKBytes +
-                                                  hf * (kPfKeys * 128) + key * 128);
+                                                  (key / BS) * C::kVBlockBytes + hf * (BS * 128) +
+                                                  (key % BS) * 128);
 #pragma unroll
             for (int c = 0; c < 8; ++c) dst[c] = make_uint4(0, 0, 0, 0);
           }
@@ -298,15 +307,20 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
         tc_fence_after_sync();
         const uint32_t v_st = sV + st * C::kKBytes;
         const uint32_t tP = tbuf(kt);
+        // keys 16k .. 16k+15 lie in one block: rows of 128 bytes from
+        // v_koff(k), the next dim half bs * 128 bytes further
+        auto v_koff = [&](int k) {
+          return static_cast<uint32_t>((k * 16 / BS) * C::kVBlockBytes + (k * 16 % BS) * 128);
+        };
 #pragma unroll
         for (int k = 0; k < kPfKeys / 16; ++k)
-          umma_f16_ts(tO, tP + 8 * k, umma_desc_mn128(v_st + k * 2048, kPfKeys * 128), kIdescO,
+          umma_f16_ts(tO, tP + 8 * k, umma_desc_mn128(v_st + v_koff(k), BS * 128), kIdescO,
                       (kt > 0 || k > 0) ? 1u : 0u);
         if constexpr (kBF16) {
 #pragma unroll
           for (int k = 0; k < kPfKeys / 16; ++k)
-            umma_f16_ts(tO, tP + 32 + 8 * k, umma_desc_mn128(v_st + k * 2048, kPfKeys * 128),
-                        kIdescO, 1u);
+            umma_f16_ts(tO, tP + 32 + 8 * k, umma_desc_mn128(v_st + v_koff(k), BS * 128), kIdescO,
+                        1u);
         }
         umma_commit(bar_o);
         umma_commit(v_empty + 8 * st);
@@ -320,15 +334,23 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     // done); whichever is ready goes first.  The block ids of the next K
     // tile are read ahead, while the loader waits.
     int nk = min(2, nkt), nv = min(2, nkt);  // tiles 0 and 1 went out above
-    int nphys[C::kBlocksPerTile];
-#pragma unroll
-    for (int b = 0; b < C::kBlocksPerTile; ++b) nphys[b] = nk < nkt ? tile_block(nk, b) : -1;
+    // block ids in chunks of 32 (lane i holds entry 32 c + i of the table,
+    // or -1 past the context), the next chunk loaded while the current one
+    // is used, so no table read stands between two tile loads
+    auto fetch_ids = [&](int c) {
+      const int j = c * 32 + lane;
+      int p = -1;
+      if (j * BS < ctx) p = table[j];
+      return p;
+    };
+    int tab_c = (nk * C::kBlocksPerTile) >> 5;
+    int tab_cur = fetch_ids(tab_c), tab_nxt = fetch_ids(tab_c + 1);
     unsigned long long t_idle = global_timer_ns();
     while ((nk < nkt || nv < nkt) && !failed) {
       bool did = false;
       if (nv < nk && nv < nkt) {
         const int ready = __shfl_sync(
-            0xffffffffu, lane == 0 ? (int)mbar_try_wait(v_empty + 8 * (nv & 1), ((nv >> 1) - 1) & 1) : 0, 0);
+            0xffffffffu, lane == 0 ? (int)mbar_test_wait(v_empty + 8 * (nv & 1), ((nv >> 1) - 1) & 1) : 0, 0);
         if (ready) {
           if (lane == 0) issue_tile(nv, true, s_phys + (nv & 3) * C::kBlocksPerTile);
           ++nv;
@@ -337,17 +359,27 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
       }
       if (nk < nkt) {
         const int ready = __shfl_sync(
-            0xffffffffu, lane == 0 ? (int)mbar_try_wait(k_empty + 8 * (nk & 1), ((nk >> 1) - 1) & 1) : 0, 0);
+            0xffffffffu, lane == 0 ? (int)mbar_test_wait(k_empty + 8 * (nk & 1), ((nk >> 1) - 1) & 1) : 0, 0);
         if (ready) {
+          const int j0 = nk * C::kBlocksPerTile;  // a tile never straddles two chunks
+          if ((j0 >> 5) != tab_c) {
+            ++tab_c;
+            tab_cur = tab_nxt;
+            tab_nxt = fetch_ids(tab_c + 1);
+          }
+          int phys[C::kBlocksPerTile];
+#pragma unroll
+          for (int b = 0; b < C::kBlocksPerTile; ++b) {  // as tile_block(nk, b)
+            const int p = __shfl_sync(0xffffffffu, tab_cur, (j0 + b) & 31);
+            phys[b] = (j0 + b) * BS >= ctx ? -1 : ((p >= 0 && p < a.num_blocks) ? p : -2);
+          }
           if (lane == 0) {
 #pragma unroll
             for (int b = 0; b < C::kBlocksPerTile; ++b)
-              s_phys[(nk & 3) * C::kBlocksPerTile + b] = nphys[b];
-            issue_tile(nk, false, nphys);
+              s_phys[(nk & 3) * C::kBlocksPerTile + b] = phys[b];
+            issue_tile(nk, false, phys);
           }
           ++nk;
-#pragma unroll
-          for (int b = 0; b < C::kBlocksPerTile; ++b) nphys[b] = nk < nkt ? tile_block(nk, b) : -1;
           did = true;
         }
       }
