@@ -18,19 +18,20 @@
 //           reach O; warp 5 issues the TMA loads.  They hand over through
 //           mbarriers only (S done, S read, P ready, O done, K / V full and
 //           empty per stage), never a CTA-wide barrier inside the key loop.
-//   TMEM  = two S/P buffers [0, 64) and [64, 128) | O [128, 128 + D): S(kt)
-//           in buffer kt & 1 (fp32), then P(kt) over it (P_hi in its first
-//           32 columns, P_lo (bf16 caches) in the next 32, two 16-bit values
-//           per column)
+//   TMEM  = S [0, 64) | P [64, 128) | O [128, 128 + D): S(kt) in fp32; P(kt)
+//           with P_hi in the first 32 columns of P, P_lo (bf16 caches) in
+//           the next 32, two 16-bit values per column.  S and P have
+//           buffers of their own, so S(kt+1) waits only for the rows to have
+//           read S(kt), never for O(kt-1): the MMA queue need not drain
+//           between the products of consecutive tiles
 //   per 64-key tile kt (K and V by TMA into two stages each, K one box per
 //   (block, dim half), V one box per block; K(kt+2) is loaded once S(kt) is
 //   done, V(kt+2) once O(kt) is done; the load warp reads the block ids 32 at
 //   a time, a chunk ahead, and polls the stages without sleeping on either):
 //     S            = Q K^T      tcgen05.mma, A = Q and B = K from shared memory
 //                               (K-major), M128 N64, D/16 x K16; S(kt+1) is
-//                               issued once the rows have read S(kt) and
-//                               O(kt-1), the last reader of its buffer, is
-//                               done, so it runs under the softmax of tile kt
+//                               issued once the rows have read S(kt), so it
+//                               runs under the softmax of tile kt
 //     softmax      thread r: tcgen05.ld of its S row, causal and block masks
 //                  (only on tiles that need them), online max / sum in packed
 //                  fp32 pairs; with a bf16 cache P = P_hi + P_lo (two bf16
@@ -61,7 +62,7 @@ constexpr int kPfThreads = 192;     // + warp 4: MMA issue, warp 5: TMA loads
 constexpr int kPfRows = 128;      // MMA M: (token, head) rows per CTA
 constexpr int kPfKeys = 64;       // keys per tile
 constexpr int kPfMaxD = 128;      // head_dim 64 or 128: one or two 64-dim (128-byte) halves
-constexpr int kPfTmemCols = 256;  // S/P buffers [0, 64) and [64, 128), O [128, 256)
+constexpr int kPfTmemCols = 256;  // S [0, 64), P [64, 128), O [128, 256)
 constexpr float kPfRescaleLog2 = 8.f;  // rescale O when the max grows by more than this
 
 template <int BS, int D>
@@ -223,11 +224,13 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     }
     fence_proxy_async_smem();
   }
-  // any bad table entry among the blocks this CTA reads?  (then every tile
-  // takes the masked path; otherwise only the tiles that cross the diagonal
-  // or the end of the context)
+  // any bad table entry among the blocks this CTA loads (every block of its
+  // key tiles inside the context, visible to its rows or not)?  (then every
+  // tile takes the masked path and the bad blocks' values are zeroed;
+  // otherwise only the tiles that cross the diagonal or the end of the
+  // context are masked)
   int my_bad = 0;
-  for (int j = tid; j * BS < kend; j += kPfThreads) {
+  for (int j = tid; j * BS < min(nkt * kPfKeys, ctx); j += kPfThreads) {
     const int p = table[j];
     my_bad |= (p < 0 || p >= a.num_blocks);
   }
@@ -236,10 +239,9 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
   tc_fence_after_sync();
   if (any_bad && tid == 0) record_error(PA_ERR_DEVICE_BOUNDS);
   const uint32_t tmem = *tmem_slot;
-  // S(kt) and then P(kt) (hi in the first 32 columns, lo in the next 32) live
-  // in buffer kt & 1; O in [128, 256)
-  const uint32_t tO = tmem + 128;
-  auto tbuf = [&](int kt) { return tmem + 64u * static_cast<uint32_t>(kt & 1); };
+  // S(kt) in [0, 64); P(kt) in [64, 128), hi in its first 32 columns, lo in
+  // the next 32; O in [128, 256)
+  const uint32_t tS = tmem, tP = tmem + 64, tO = tmem + 128;
   bool failed = false;
   auto wait = [&](uint32_t bar, int parity) {
     if (!failed && !mbar_wait_bounded(bar, parity)) {
@@ -267,7 +269,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
       const uint32_t k_st = sK + (kt & 1) * C::kKBytes;
 #pragma unroll
       for (int k = 0; k < D / 16; ++k)
-        umma_f16(tbuf(kt), umma_desc_k128(sQ + (k >> 2) * (kPfRows * 128) + (k & 3) * 32),
+        umma_f16(tS, umma_desc_k128(sQ + (k >> 2) * (kPfRows * 128) + (k & 3) * 32),
                  umma_desc_k128(k_st + (k >> 2) * (kPfKeys * 128) + (k & 3) * 32), kIdescS,
                  k > 0 ? 1u : 0u);
       umma_commit(bar_s);
@@ -277,13 +279,10 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     for (int kt = 0; kt < nkt; ++kt) {
       const int st = kt & 1;
       if (kt + 1 < nkt) {
-        wait(s_free, kt & 1);  // every row has read S(kt)
-        // S(kt+1) overwrites buffer (kt+1) & 1, whose P(kt-1) O(kt-1) reads:
-        // wait for O(kt-1) (these waits go in order, one per product)
-        if (kt >= 1) wait(bar_o, (kt - 1) & 1);
+        wait(s_free, kt & 1);  // every row has read S(kt): S(kt+1) may overwrite it
         issue_s(kt + 1);
       }
-      wait(p_ready, kt & 1);  // P(kt) in TMEM, O(kt-1) done (the rows waited for it)
+      wait(p_ready, kt & 1);  // P(kt) in TMEM (the rows waited for O(kt-1) to write it)
       wait(full_v + 8 * st, (kt >> 1) & 1);
       // values of keys past the context or in bad blocks may hold anything
       // (0 * NaN would reach O): zero their rows of V(kt)
@@ -306,7 +305,6 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
       if (lane == 0 && !failed) {  // O += (P_hi [+ P_lo]) V(kt): (2 x) 4 MMAs of K = 16
         tc_fence_after_sync();
         const uint32_t v_st = sV + st * C::kKBytes;
-        const uint32_t tP = tbuf(kt);
         // keys 16k .. 16k+15 lie in one block: rows of 128 bytes from
         // v_koff(k), the next dim half bs * 128 bytes further
         auto v_koff = [&](int k) {
@@ -401,7 +399,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
       wait(bar_s, kt & 1);
       tc_fence_after_sync();
       uint32_t sv[kPfKeys];
-      const uint32_t tb = tbuf(kt) + lane_off;
+      const uint32_t tb = tS + lane_off;
       {
         uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[0]);
         uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sv[32]);
@@ -460,11 +458,14 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
       }
       const float2 ss = f2_split(sum2);
       l_run = l_run * alpha + (ss.x + ss.y);
-      // O is touched only to rescale it: then wait for O(kt-1) (S(kt) done
-      // means O(kt-2) is, so this wait cannot fall two phases behind)
-      if (kt > 0 && __any_sync(0xffffffffu, resc)) {
+      // P(kt) takes the P buffer and a rescale touches O: wait for O(kt-1),
+      // the last reader of both (O(kt) needs P(kt), so this wait cannot fall
+      // two phases behind); by now it has long finished
+      if (kt > 0) {
         wait(bar_o, (kt - 1) & 1);
         tc_fence_after_sync();
+      }
+      if (kt > 0 && __any_sync(0xffffffffu, resc)) {
         {  // tcgen05.ld / st are warp-wide
           const uint64_t al2 = f2(alpha, alpha);
 #pragma unroll
@@ -483,10 +484,8 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
           }
         }
       }
-      // P(kt) over S(kt) in its buffer: the buffer's previous reader O(kt-2)
-      // finished before S(kt) did
-      tmem_st32(tb, ph);
-      if constexpr (kBF16) tmem_st32(tb + 32, pl);
+      tmem_st32(tP + lane_off, ph);
+      if constexpr (kBF16) tmem_st32(tP + lane_off + 32, pl);
       tmem_wait_st();
       tc_fence_before_sync();
       __syncwarp();

@@ -110,6 +110,14 @@ def test_prefill_bad_table_entry_masks_its_block(pa):
     # over the remaining keys
     pw = W.prefill(seed=12, ctxs=(160,), nqs=(160,), hq=32, hkv=8, bs=16, dtype="bf16")
     b = pw.base
+    # first a call whose values are all NaN, so that shared memory left over
+    # from it holds NaN: a CTA whose first key tile holds the bad block (rows
+    # 0-31 here, which never see it) must still zero that block's values
+    nan_v = torch.full_like(b.v_pool, float("nan")).cuda()
+    pa.prefill(pw.q.cuda(), b.k_pool.cuda(), nan_v, torch.from_numpy(b.block_tables).cuda(),
+               torch.from_numpy(b.context_lens).cuda(), torch.from_numpy(pw.query_start).cuda(),
+               b.scale, pw.max_query_len, b.max_context_len)
+    pa.sync_status()
     b.block_tables = b.block_tables.copy()
     b.block_tables[0, 3] = b.k_pool.shape[0] + 5
     bt = torch.from_numpy(b.block_tables).cuda()
