@@ -139,7 +139,7 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
   if (threadIdx.x == 0) {
     prefetch_tensormap(&a.tmap_k);
     prefetch_tensormap(&a.tmap_v);
-    s_item = atomicAdd(a.counter, 1);
+    s_item = blockIdx.x;  // CTA c starts on item c; later ones come from the counter
   }
   __syncthreads();
 
@@ -845,7 +845,7 @@ cascade_kernel(const __grid_constant__ CascadeArgs a) {
         }
       }
     }
-    if (threadIdx.x == 0) s_item = atomicAdd(a.counter, 1);
+    if (threadIdx.x == 0) s_item = static_cast<int>(gridDim.x) + atomicAdd(a.counter, 1);
     __syncthreads();           // scratch (= stage memory) and s_seq free again ...
     fence_proxy_async_smem();  // ... before the next item's tile loads
   }

@@ -337,13 +337,16 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
   uint32_t skip_stage = 0;                // stages holding a block with a bad table entry
   bool failed = false;                    // a wait timed out: stop issuing / computing
 
-  // the next item and its descriptor, fetched by thread 0
-  auto fetch_next = [&]() {
-    const int it = atomicAdd(a.counter, 1);
+  // the next item and its descriptor, fetched by thread 0: CTA c starts on
+  // item c (no atomic on the path to the first tile); later items come from
+  // the counter, past the grid's first ones
+  auto fetch_next = [&](bool first) {
+    const int it = first ? static_cast<int>(blockIdx.x)
+                         : static_cast<int>(gridDim.x) + atomicAdd(a.counter, 1);
     s_item = it;
     if (it < total) s_desc = a.order[it / (a.hkv * a.ncg)];
   };
-  if (threadIdx.x == 0) fetch_next();
+  if (threadIdx.x == 0) fetch_next(true);
   __syncthreads();
 
   for (;;) {
@@ -790,7 +793,7 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
     }
     // the next item is taken only now, when this CTA can start it at once,
     // so no CTA holds an item it cannot start while others run dry
-    if (threadIdx.x == 0) fetch_next();
+    if (threadIdx.x == 0) fetch_next(false);
     __syncthreads();           // scratch (= stage memory) is free again ...
     fence_proxy_async_smem();  // ... and the next item's tile loads come after these accesses
   }
