@@ -16,8 +16,9 @@
 //           head r % G) lives in TMEM lane r and thread r runs its softmax.
 //           Warp 4 issues the MMAs (one lane) and zeroes values that must not
 //           reach O; warp 5 issues the TMA loads.  They hand over through
-//           mbarriers only (S done, S read, P ready, O done, K / V full and
-//           empty per stage), never a CTA-wide barrier inside the key loop.
+//           mbarriers only (S done and O done, four of each, which also
+//           free K and V stages; S read, P ready; K / V full per stage),
+//           never a CTA-wide barrier inside the key loop.
 //   TMEM  = S [0, 64) | P [64, 128) | O [128, 128 + D): S(kt) in fp32; P(kt)
 //           with P_hi in the first 32 columns of P, P_lo (bf16 caches) in
 //           the next 32, two 16-bit values per column.  S and P have
@@ -76,7 +77,7 @@ struct PrefillCfg {
   static constexpr int kOffK = kOffQ + kQBytes;           // 2 stages
   static constexpr int kOffV = kOffK + 2 * kKBytes;       // 2 stages
   static constexpr int kTiles = kOffV + 2 * kKBytes;      // 96 KiB at D 128: two CTAs per SM
-  static constexpr int kHead = 256;                       // 12 mbarriers, TMEM slot, block ids
+  static constexpr int kHead = 256;                       // 15 mbarriers, TMEM slot, block ids
   static constexpr int kSmemBytes = kTiles + kHead;
   static_assert(kPfKeys % BS == 0, "a key tile holds whole blocks");
 };
@@ -143,12 +144,17 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
   uint8_t* const base = pf_smem;
   const uint32_t head_s = base_s + C::kTiles;
   const uint32_t full_k = head_s, full_v = head_s + 16;  // + 8 * stage, TMA
-  const uint32_t bar_s = head_s + 32, bar_o = head_s + 40;  // MMA commits
-  const uint32_t s_free = head_s + 48, p_ready = head_s + 56;  // one arrival per row warp
-  const uint32_t k_empty = head_s + 64, v_empty = head_s + 80;  // + 8 * stage, MMA commits
-  const uint32_t bar_done = head_s + 96;                           // the last O product
-  const uint32_t tmem_slot_s = head_s + 104;  // tcgen05.alloc writes the TMEM address here
-  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(base + C::kTiles + 104);
+  // S(kt) done and O(kt) done: MMA commits to one of four barriers each, kt & 3,
+  // waited with parity (kt >> 2) & 1.  The row warps wait on them, and so
+  // does the load warp before it refills a stage (K(kt+2) after S(kt),
+  // V(kt+2) after O(kt)): a barrier cannot run a phase ahead of the loader,
+  // since its next phase, S(kt+4) or O(kt+4), needs the tile the loader has
+  // yet to load, so no separate "stage empty" commits are needed
+  const uint32_t bar_s = head_s + 32, bar_o = head_s + 64;  // + 8 * (kt & 3)
+  const uint32_t s_free = head_s + 96, p_ready = head_s + 104;  // one arrival per row warp
+  const uint32_t bar_done = head_s + 112;                        // the last O product
+  const uint32_t tmem_slot_s = head_s + 120;  // tcgen05.alloc writes the TMEM address here
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(base + C::kTiles + 120);
   // the loader's block ids of key tile kt (K issue writes, V issue reads)
   int* const s_phys = reinterpret_cast<int*>(base + C::kTiles + 128);  // [4][kBlocksPerTile]
   const uint32_t sQ = base_s + C::kOffQ, sK = base_s + C::kOffK, sV = base_s + C::kOffV;
@@ -193,10 +199,10 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
   };
 
   if (producer && !mma_warp && lane == 0) {
-    for (int i = 0; i < 6; ++i) mbar_init(head_s + 8 * i, 1);
+    for (int i = 0; i < 12; ++i) mbar_init(head_s + 8 * i, 1);  // full_k/v[2], bar_s[4], bar_o[4]
     mbar_init(s_free, kPfRowThreads / 32);
     mbar_init(p_ready, kPfRowThreads / 32);
-    for (int i = 0; i < 5; ++i) mbar_init(k_empty + 8 * i, 1);  // k/v_empty[2], done
+    mbar_init(bar_done, 1);
     mbar_init_fence();
     prefetch_tensormap(&a.tmap_k);
     prefetch_tensormap(&a.tmap_v);
@@ -272,8 +278,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
         umma_f16(tS, umma_desc_k128(sQ + (k >> 2) * (kPfRows * 128) + (k & 3) * 32),
                  umma_desc_k128(k_st + (k >> 2) * (kPfKeys * 128) + (k & 3) * 32), kIdescS,
                  k > 0 ? 1u : 0u);
-      umma_commit(bar_s);
-      umma_commit(k_empty + 8 * (kt & 1));
+      umma_commit(bar_s + 8 * (kt & 3));  // S(kt) done: the rows read it, K(kt)'s stage is free
     };
     issue_s(0);
     for (int kt = 0; kt < nkt; ++kt) {
@@ -320,8 +325,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
             umma_f16_ts(tO, tP + 32 + 8 * k, umma_desc_mn128(v_st + v_koff(k), BS * 128), kIdescO,
                         1u);
         }
-        umma_commit(bar_o);
-        umma_commit(v_empty + 8 * st);
+        umma_commit(bar_o + 8 * (kt & 3));  // O(kt) done: P and V(kt)'s stage are free
       }
       __syncwarp();
     }
@@ -348,7 +352,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
       bool did = false;
       if (nv < nk && nv < nkt) {
         const int ready = __shfl_sync(
-            0xffffffffu, lane == 0 ? (int)mbar_test_wait(v_empty + 8 * (nv & 1), ((nv >> 1) - 1) & 1) : 0, 0);
+            0xffffffffu, lane == 0 ? (int)mbar_test_wait(bar_o + 8 * ((nv - 2) & 3), ((nv - 2) >> 2) & 1) : 0, 0);
         if (ready) {
           if (lane == 0) issue_tile(nv, true, s_phys + (nv & 3) * C::kBlocksPerTile);
           ++nv;
@@ -357,7 +361,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
       }
       if (nk < nkt) {
         const int ready = __shfl_sync(
-            0xffffffffu, lane == 0 ? (int)mbar_test_wait(k_empty + 8 * (nk & 1), ((nk >> 1) - 1) & 1) : 0, 0);
+            0xffffffffu, lane == 0 ? (int)mbar_test_wait(bar_s + 8 * ((nk - 2) & 3), ((nk - 2) >> 2) & 1) : 0, 0);
         if (ready) {
           const int j0 = nk * C::kBlocksPerTile;  // a tile never straddles two chunks
           if ((j0 >> 5) != tab_c) {
@@ -396,7 +400,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
     float m_run = -INFINITY;  // running max of the raw scores
     float l_run = 0.f;        // sum of weights, relative to m_run
     for (int kt = 0; kt < nkt; ++kt) {
-      wait(bar_s, kt & 1);
+      wait(bar_s + 8 * (kt & 3), (kt >> 2) & 1);
       tc_fence_after_sync();
       uint32_t sv[kPfKeys];
       const uint32_t tb = tS + lane_off;
@@ -462,7 +466,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
       // the last reader of both (O(kt) needs P(kt), so this wait cannot fall
       // two phases behind); by now it has long finished
       if (kt > 0) {
-        wait(bar_o, (kt - 1) & 1);
+        wait(bar_o + 8 * ((kt - 1) & 3), ((kt - 1) >> 2) & 1);
         tc_fence_after_sync();
       }
       if (kt > 0 && __any_sync(0xffffffffu, resc)) {
