@@ -24,7 +24,8 @@
 //           the next 32, two 16-bit values per column.  S and P have
 //           buffers of their own, so S(kt+1) waits only for the rows to have
 //           read S(kt), never for O(kt-1): the MMA queue need not drain
-//           between the products of consecutive tiles
+//           between the products of consecutive tiles (the rows write P(kt)
+//           once O(kt-1), the P buffer's last reader, is done)
 //   per 64-key tile kt (K and V by TMA into two stages each, K one box per
 //   (block, dim half), V one box per block; K(kt+2) is loaded once S(kt) is
 //   done, V(kt+2) once O(kt) is done; the load warp reads the block ids 32 at
