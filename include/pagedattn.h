@@ -250,8 +250,12 @@ size_t pa_decode_workspace_size(int32_t num_seqs, int32_t num_q_heads,
  * The call enqueues two kernels on `stream`: a one-block planning kernel,
  * then the attention kernel, launched with programmatic stream
  * serialization so that its blocks set up while the plan runs and read the
- * plan only once it has completed.  Work before and after the call on the
- * stream is ordered as usual; the pair can be captured in a CUDA graph.
+ * plan only once it has completed.  When no context is split and the work
+ * items (sequences x kv heads x groups of up to 8 query heads) fit the
+ * GPU's resident attention blocks at once, there is no queue to plan: the
+ * attention kernel runs alone, block c on item c.  Work before and after
+ * the call on the stream is ordered as usual; the call can be captured in
+ * a CUDA graph.
  */
 pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype,
                     const void* k_pool, const void* v_pool, pa_dtype cache_dtype,

@@ -128,6 +128,12 @@ struct DecodeArgs {
   int ncg;                 // column groups per kv head: ceil(group / 8) items read its blocks
   float sl2;               // scale * k_scale * log2(e)
   float out_scale;         // v_scale
+  // direct = 1: no planning kernel ran (unsplit contexts, one item per CTA):
+  // CTA c takes item c, whose descriptor it forms from the context length,
+  // and CTA 0 writes split_len to *split_out as the plan would
+  int direct;
+  int split_len;
+  int32_t* split_out;
 };
 
 // ---------------------------------------------------------------- planning
@@ -328,11 +334,12 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
     prefetch_tensormap(&a.tmap_k);
     prefetch_tensormap(&a.tmap_v);
   }
-  // launched behind plan_kernel: nothing from global memory before it is done
+  // launched behind plan_kernel (or, direct, behind whatever wrote the cache):
+  // nothing from global memory before it is done
   grid_dependency_wait();
   __syncthreads();
 
-  const int total = *a.total;
+  const int total = a.direct ? a.num_seqs * a.hkv * a.ncg : *a.total;
   uint32_t n_issued = 0, n_consumed = 0;  // warp-uniform ring counters
   uint32_t skip_stage = 0;                // stages holding a block with a bad table entry
   bool failed = false;                    // a wait timed out: stop issuing / computing
@@ -342,9 +349,23 @@ decode_kernel(const __grid_constant__ DecodeArgs a) {
   // the counter, past the grid's first ones
   auto fetch_next = [&](bool first) {
     const int it = first ? static_cast<int>(blockIdx.x)
-                         : static_cast<int>(gridDim.x) + atomicAdd(a.counter, 1);
+                   : a.direct ? total  // one item per CTA
+                              : static_cast<int>(gridDim.x) + atomicAdd(a.counter, 1);
     s_item = it;
-    if (it < total) s_desc = a.order[it / (a.hkv * a.ncg)];
+    if (it < total) {
+      if (a.direct) {  // the whole context as one range, validated as the plan does
+        const int seq = it / (a.hkv * a.ncg);
+        int c = a.context_lens[seq];
+        if (c < 0 || c > a.max_ctx || c > a.max_blocks * BS) {
+          if (it % (a.hkv * a.ncg) == 0) record_error(PA_ERR_DEVICE_BOUNDS);
+          c = 0;
+        }
+        s_desc = make_int4(seq, 1 << 16, 0, c);
+      } else {
+        s_desc = a.order[it / (a.hkv * a.ncg)];
+      }
+    }
+    if (a.direct && first && blockIdx.x == 0) *a.split_out = a.split_len;
   };
   if (threadIdx.x == 0) fetch_next(true);
   __syncthreads();

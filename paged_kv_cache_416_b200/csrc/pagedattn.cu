@@ -567,12 +567,8 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_po
   a.ncg = ncg;
   const bool qbf = q_dtype == PA_BF16;
 
-  // the automatic split may be lengthened on the device from the actual
-  // lengths (never shortened: the workspace holds the ranges of S), aiming
-  // at 15/16 of a kPlanSms-SM persistent grid of this instance in items
-  int adapt_items = 0;
-  if (split_tokens == 0 && w.is_split) {
-    int per_sm = 0;
+  int per_sm = 0;  // resident CTAs of this instance (cached per device)
+  {
     pa_status os;
     if (cache_dtype == PA_F16)
       os = occupancy_shape<pa::kCacheF16, false>(head_dim, block_size, dev, &per_sm);
@@ -583,18 +579,31 @@ pa_status pa_decode(void* out, const void* q, pa_dtype q_dtype, const void* k_po
     else
       os = occupancy_shape<pa::kCacheE4M3, false>(head_dim, block_size, dev, &per_sm);
     if (os != PA_OK) return os;
-    adapt_items = static_cast<int>(std::max<int64_t>(1, kPlanSms * per_sm * 15 / 16));
   }
-  pa::plan_kernel<<<1, 1024, 0, st>>>(context_lens, num_seqs, max_context_len, max_blocks_per_seq,
-                                      block_size, w.is_split ? S : std::max(S, max_context_len),
-                                      adapt_items, num_kv_heads * ncg,
-                                      reinterpret_cast<int32_t*>(ws + w.counter),
-                                      reinterpret_cast<int32_t*>(ws + w.total),
-                                      reinterpret_cast<int32_t*>(ws + w.split),
-                                      reinterpret_cast<int32_t*>(ws + w.seq_off),
-                                      reinterpret_cast<int4*>(ws + w.order),
-                                      w.is_split ? reinterpret_cast<int32_t*>(ws + w.arrived) : nullptr);
   const int64_t items_upper = w.ranges * num_kv_heads * ncg;
+  // unsplit contexts and no more items than resident CTAs: no planning
+  // kernel (CTA c forms item c itself; there is no queue to order)
+  const bool direct = !w.is_split && items_upper <= static_cast<int64_t>(device_sms(dev)) * per_sm;
+  a.direct = direct ? 1 : 0;
+  a.split_len = w.is_split ? S : std::max(S, max_context_len);
+  a.split_out = reinterpret_cast<int32_t*>(ws + w.split);
+  // the automatic split may be lengthened on the device from the actual
+  // lengths (never shortened: the workspace holds the ranges of S), aiming
+  // at 15/16 of a kPlanSms-SM persistent grid of this instance in items
+  int adapt_items = 0;
+  if (split_tokens == 0 && w.is_split)
+    adapt_items = static_cast<int>(std::max<int64_t>(1, kPlanSms * per_sm * 15 / 16));
+  if (!direct) {
+    pa::plan_kernel<<<1, 1024, 0, st>>>(context_lens, num_seqs, max_context_len, max_blocks_per_seq,
+                                        block_size, w.is_split ? S : std::max(S, max_context_len),
+                                        adapt_items, num_kv_heads * ncg,
+                                        reinterpret_cast<int32_t*>(ws + w.counter),
+                                        reinterpret_cast<int32_t*>(ws + w.total),
+                                        reinterpret_cast<int32_t*>(ws + w.split),
+                                        reinterpret_cast<int32_t*>(ws + w.seq_off),
+                                        reinterpret_cast<int4*>(ws + w.order),
+                                        w.is_split ? reinterpret_cast<int32_t*>(ws + w.arrived) : nullptr);
+  }
   pa_status s;
   if (cache_dtype == PA_F16)
     s = dispatch_shape<pa::kCacheF16, false>(a, head_dim, block_size, items_upper, dev, st);
