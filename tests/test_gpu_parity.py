@@ -438,6 +438,42 @@ def test_decode_short_contexts_many_sequences(pa, cache):
     assert_attention_close(as_f64(out), ref, f"short contexts {cache}")
 
 
+def test_unplanned_small_batch_equals_the_planned_large_one(pa):
+    """A batch whose unsplit items fit the resident CTAs runs without the
+    planning kernel (each CTA forms its item from the context length); the
+    same sequences inside a batch too large for that go through the plan and
+    its work queue.  Both compute each (sequence, kv head) item the same way,
+    so the outputs agree bit for bit; the small batch also matches the oracle."""
+    rng = np.random.default_rng(43)
+    lens = rng.integers(1, 200, size=1000)
+    w = W._generic("planned", lens, 32, 8, 128, 16, "bf16", "bf16", seed=43, device="cpu")
+    kp, vp = w.k_pool.cuda().clone(), w.v_pool.cuda().clone()
+    pa.write_kv(w.new_k.cuda().contiguous(), w.new_v.cuda().contiguous(),
+                torch.from_numpy(w.slot_mapping).cuda(), kp, vp, w.k_scale, w.v_scale)
+    q = w.q.cuda().contiguous()
+    bt = torch.from_numpy(w.block_tables).cuda()
+    cl = torch.from_numpy(w.context_lens).cuda()
+    B, hq, d = q.shape
+    ws_big = torch.zeros(pa.decode_workspace_size(B, hq, 8, d, 16, w.max_context_len), dtype=torch.uint8,
+                         device="cuda")
+    big = pa.decode(q, kp, vp, bt, cl, w.scale, w.max_context_len, workspace=ws_big)
+    pa.sync_status()
+    n = 40  # 40 x 8 items: fewer than the resident CTAs
+    ws_small = torch.zeros(pa.decode_workspace_size(n, hq, 8, d, 16, w.max_context_len), dtype=torch.uint8,
+                           device="cuda")
+    small_out = pa.decode(q[:n].contiguous(), kp, vp, bt[:n].contiguous(), cl[:n].contiguous(), w.scale,
+                          w.max_context_len, workspace=ws_small)
+    pa.sync_status()
+    # the plan wrote the item total (byte offset 4); the unplanned call did not
+    assert int(ws_big[4:8].view(torch.int32).item()) == B * 8
+    assert int(ws_small[4:8].view(torch.int32).item()) == 0
+    # both wrote the range length they used (byte offset 8): no split
+    assert int(ws_small[8:12].view(torch.int32).item()) >= w.max_context_len
+    assert torch.equal(small_out, big[:n])
+    ref, _, _ = oracle_step(w, seqs=range(n))
+    assert_attention_close(as_f64(small_out), ref[:n], "unplanned small batch")
+
+
 @pytest.mark.parametrize("hq,hkv,cache,split", [(96, 8, "bf16", 0), (128, 8, "bf16", 64),
                                                 (16, 1, "e4m3", 32), (48, 4, "f16", 0)])
 def test_decode_more_than_eight_query_heads_per_kv_head(pa, hq, hkv, cache, split):
