@@ -95,13 +95,14 @@ def grow_keys(pw, rate):
     return pw
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "f16"])
-def test_prefill_long_context_growing_scores(pa, dtype):
-    # a chunk late in a long context (many key tiles, both K/V stages reused
-    # many times) with scores that grow along the keys
-    pw = grow_keys(W.prefill(seed=11, ctxs=(1500, 700), nqs=(96, 700), hq=32, hkv=8, bs=16,
+@pytest.mark.parametrize("dtype,bs", [("bf16", 16), ("f16", 16), ("bf16", 32)])
+def test_prefill_long_context_growing_scores(pa, dtype, bs):
+    # a chunk late in a long context (many key tiles, both K/V stages and
+    # every S / O barrier reused many times, the load warp's block ids read
+    # across several 32-entry chunks) with scores that grow along the keys
+    pw = grow_keys(W.prefill(seed=11, ctxs=(1500, 700), nqs=(96, 700), hq=32, hkv=8, bs=bs,
                              dtype=dtype), 1.0 / 48)
-    assert_attention_close(as_f64(run(pa, pw)), ref(pw), f"prefill growing scores {dtype}")
+    assert_attention_close(as_f64(run(pa, pw)), ref(pw), f"prefill growing scores {dtype} bs{bs}")
 
 
 def test_prefill_bad_table_entry_masks_its_block(pa):
