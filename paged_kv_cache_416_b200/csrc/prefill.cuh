@@ -105,6 +105,10 @@ __device__ __forceinline__ uint32_t swz128(int r, int c) {
 
 // One CTA per (query tile, kv head, sequence): grid (ceil(max_query_len / T),
 // Hkv, B) with T = 128 / G tokens; CTAs past a sequence's new tokens exit.
+// Blocks start in index order, x fastest, and block x takes query tile
+// gridDim.x - 1 - x: within a (sequence, kv head) the tiles with the most
+// keys under the causal mask start first, so the grid ends on short tiles
+// (the tiles of one pair still run side by side and share its K / V in L2).
 template <bool kBF16, int BS, int D>
 __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_constant__ PrefillArgs a) {
   using C = PrefillCfg<BS, D>;
@@ -118,7 +122,7 @@ __global__ void __launch_bounds__(kPfThreads, 2) prefill_kernel(const __grid_con
   const int T = kPfRows / G;  // query tokens per CTA
   const int q0 = a.query_start[s];
   const int n = a.query_start[s + 1] - q0;
-  const int i0 = blockIdx.x * T;
+  const int i0 = static_cast<int>(gridDim.x - 1 - blockIdx.x) * T;
   if (n <= 0 || i0 >= n) return;  // the whole CTA, before any TMEM use
   const int nt = min(T, n - i0);
   const int r = tid;                          // row of a row thread
